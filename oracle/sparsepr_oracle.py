@@ -1,0 +1,572 @@
+"""Plain fp64 CPU oracle of the SparsePR sparse attention call.
+
+TEST INFRASTRUCTURE: imported only by tests, the smoke check and the bench's
+CPU-baseline leg; never by the product path.
+
+Sources.  The method is "Partition the Support, Reconstruct the Residual:
+Training-Free Sparse Attention for Video Generation and World Models"
+(Taghavi, Langari, Pandey; arXiv 2608.18484), known here only through web
+summaries.  Citations name the page and the paper section it summarises:
+
+  [paperlayer §X]  paperlayer.ai section-by-section summary, section X
+  [abstract]       the English abstract (paperdance.org card)
+  [gist-nl §X]     gist.science Dutch technical summary, section X
+                   (the Italian and Korean gist.science pages repeat it)
+
+Numerics: every input is the bf16-rounded tensor converted to fp64; all
+arithmetic is fp64.  Library primitives used as single steps: matmul,
+``numpy.linalg.eigh`` (symmetric eigendecomposition), ``numpy.linalg.solve``,
+``numpy.argsort`` / ``lexsort`` (stable sorts).
+
+Readings (the pages leave these steps open; the plainest reading is taken):
+  R1 sampled queries: rows floor(i*N/M_s), i < M_s.
+  R2 key-response weights: top-p eigenvectors of M_K scaled by
+     sqrt(lambda_i / sum_j lambda_j) (Euclidean distance in these coordinates
+     is the sampled-query response-profile distance, truncated to p).
+  R3 k-means init: G distinct rows from a partial Fisher-Yates shuffle driven
+     by splitmix64; T Lloyd iterations, ties to the lowest index, an empty
+     cluster keeps its previous centroid; labels are the T-th assignment.
+  R4 query-response coordinates: u_q = s * Ctilde q over nonempty K/V groups
+     (Ctilde = raw-key group means minus their unweighted mean), divided by
+     sqrt(mean(u_q^2) + 1e-6).
+  R5 route logit: s * qbar_i . c_j + ln|K_j| (qbar_i = mean raw query of group
+     i, c_j = uncentred mean raw key of group j); cells of a query group are
+     ranked by softmax mass (ties to lower j); a cell's entry mass is the
+     cumulative mass ranked before it; tau mode keeps entry mass < tau; budget
+     mode keeps all cells with entry mass <= the largest value v such that the
+     kept cells' true cost sum |Q_i||K_j| plus the probe pairs M*N_k fits in
+     rho_target*N_q*N_k (per head); each group's top cell is always kept.
+  R6 probes: one per nonempty query group, the rest apportioned by largest
+     remainder on the spare capacity |Q_g|-1 (ties to lower g); if M is below
+     the number of nonempty groups, the M largest groups get one each; within a
+     group, members in original-index order at positions
+     floor((t+1/2)|Q_g|/m_g); coverage weight (|Q_g|/m_g) normalised to sum 1.
+  R7 fit: weighted (coverage weights) centring; U_r = leading eigenvectors of
+     the weighted centred residual Gram (= right singular vectors), directions
+     with sigma <= 1e-6 sigma_max dropped; the feature-dependent term is a
+     ridge fit (absolute lambda, unpenalised intercept) of the centred
+     residual's U_r coordinates on the centred sparse output, and only that
+     term is restricted to U_r: the intercept keeps the full weighted mean
+     residual; probe rows keep their exact dense value.
+  R8 rho_exec counts routed cells and, separately, the M*N_k probe pairs.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+__all__ = [
+    "Params", "attention_rows", "dense_attention", "sample_query_indices",
+    "response_metric", "key_response_weights", "splitmix64_stream",
+    "kmeans_init_indices", "kmeans", "kmeans_objective", "group_means",
+    "kv_centroids", "query_response_coords", "group_major_permutation",
+    "route_logits", "route_entry_mass", "route_select", "route_to_csr",
+    "select_probes", "hard_drop_attention", "fit_residual", "apply_correction",
+    "rho_exec", "sparsepr_head", "sparsepr_call",
+]
+
+MASK64 = (1 << 64) - 1
+RMS_EPS = 1e-6
+SIGMA_DROP = 1e-6
+
+
+@dataclasses.dataclass
+class Params:
+    """Method parameters of one call (the oracle's own copy)."""
+
+    Ms: int
+    p: int
+    Gk: int
+    Gq: int
+    iters: int = 10
+    route_mode: str = "tau"  # "tau" | "budget"
+    tau: float = 0.9
+    rho_target: float = 0.25
+    M: int = 64
+    r: int = 8
+    lam: float = 1e-3
+    seed: int = 0
+    scale: float | None = None  # default 1/sqrt(d)
+    weight_power: float = 0.5
+
+
+# ---------------------------------------------------------------------------
+# Dense attention (the operator SparsePR approximates) [abstract]
+# ---------------------------------------------------------------------------
+def attention_rows(Qr, K, V, scale):
+    """softmax(scale * Qr K^T) V for the given query rows, in fp64.
+
+    Textbook softmax attention with the row maximum subtracted before exp.
+    """
+    S = scale * (np.asarray(Qr, np.float64) @ np.asarray(K, np.float64).T)
+    S = S - S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P = P / P.sum(axis=1, keepdims=True)
+    return P @ np.asarray(V, np.float64)
+
+
+def dense_attention(Q, K, V, scale, chunk=2048):
+    """Full dense attention, row by row (rows are independent)."""
+    out = np.empty((Q.shape[0], V.shape[1]), np.float64)
+    for s in range(0, Q.shape[0], chunk):
+        out[s:s + chunk] = attention_rows(Q[s:s + chunk], K, V, scale)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Response-Coupled Partitioning [paperlayer §4, App. B, B.1, B.2; gist-nl §2A]
+# ---------------------------------------------------------------------------
+def sample_query_indices(N, Ms):
+    """Deterministic sampled queries [paperlayer App. B.1]; reading R1."""
+    return np.array([(i * N) // Ms for i in range(Ms)], dtype=np.int64)
+
+
+def response_metric(Qs):
+    """M_K = Q_s^T Q_s / M_s  [gist-nl §2A]."""
+    Qs = np.asarray(Qs, np.float64)
+    return Qs.T @ Qs / Qs.shape[0]
+
+
+def key_response_weights(MK, p, weight_power=0.5):
+    """Key-response projection W (d x p) [paperlayer App. B.1]; reading R2.
+
+    Columns are the top-p eigenvectors of M_K (descending eigenvalue), each
+    scaled by (lambda_i / sum_j lambda_j) ** weight_power.  Returns (W, lam)
+    with lam the eigenvalues in descending order.
+    """
+    lam, U = np.linalg.eigh(np.asarray(MK, np.float64))
+    order = np.argsort(-lam, kind="stable")
+    lam, U = lam[order], U[:, order]
+    lam = np.maximum(lam, 0.0)
+    tot = lam.sum()
+    wts = (lam[:p] / tot) ** weight_power if tot > 0 else np.zeros(p)
+    return U[:, :p] * wts[None, :], lam
+
+
+def splitmix64_stream(state):
+    """splitmix64 (Steele, Lea & Flood, OOPSLA 2014): yields 64-bit outputs."""
+    x = state & MASK64
+    while True:
+        x = (x + 0x9E3779B97F4A7C15) & MASK64
+        z = x
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & MASK64
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & MASK64
+        yield z ^ (z >> 31)
+
+
+def kmeans_init_indices(n, G, seed, bh, which):
+    """G distinct row indices for k-means init (reading R3).
+
+    Partial Fisher-Yates over 0..n-1: for i < G, j = i + (draw mod (n - i)),
+    swap a[i], a[j]; the stream starts at
+    seed XOR ((2*bh + which + 1) * 0xD1B54A32D192ED03) mod 2^64,
+    which = 0 for keys, 1 for queries.
+    """
+    if G > n:
+        raise ValueError("more groups than rows")
+    state = (seed ^ (((2 * bh + which + 1) * 0xD1B54A32D192ED03) & MASK64)) & MASK64
+    rng = splitmix64_stream(state)
+    a = {}
+    out = []
+    for i in range(G):
+        j = i + next(rng) % (n - i)
+        ai, aj = a.get(i, i), a.get(j, j)
+        a[i], a[j] = aj, ai
+        out.append(a[i])
+    return np.array(out, dtype=np.int64)
+
+
+def _sqdist(X, C):
+    """Squared Euclidean distances, ||x||^2 - 2 x.c + ||c||^2, fp64."""
+    return (X * X).sum(1)[:, None] - 2.0 * (X @ C.T) + (C * C).sum(1)[None, :]
+
+
+def kmeans(X, G, iters, init_idx):
+    """Lloyd's k-means with a fixed iteration count (reading R3).
+
+    Each iteration assigns every row to its nearest centroid (ties to the lower
+    index; numpy's argmin returns the first minimum) and then replaces each
+    centroid by the mean of its rows; an empty cluster keeps its centroid.
+    Returns (labels, centroids, objective, objective_per_iteration).
+    """
+    X = np.asarray(X, np.float64)
+    C = X[np.asarray(init_idx)].copy()
+    lab = np.zeros(X.shape[0], np.int64)
+    hist = []
+    for _ in range(iters):
+        lab = np.argmin(_sqdist(X, C), axis=1)
+        C = group_means(X, lab, G, fallback=C)
+        hist.append(kmeans_objective(X, lab, C))
+    return lab, C, (hist[-1] if hist else kmeans_objective(X, lab, C)), hist
+
+
+def kmeans_objective(X, lab, C):
+    """sum_n ||x_n - c_{lab_n}||^2."""
+    D = np.asarray(X, np.float64) - C[lab]
+    return float((D * D).sum())
+
+
+def group_means(X, lab, G, fallback=None):
+    """Mean row per group; groups with no rows take ``fallback`` (or NaN)."""
+    X = np.asarray(X, np.float64)
+    out = np.full((G, X.shape[1]), np.nan) if fallback is None else np.array(fallback, np.float64)
+    for g in range(G):
+        m = lab == g
+        if m.any():
+            out[g] = X[m].mean(axis=0)
+    return out
+
+
+def kv_centroids(K, lab_k, Gk):
+    """Raw-key mean per K/V group and group sizes [paperlayer App. B.2]."""
+    counts = np.bincount(lab_k, minlength=Gk).astype(np.int64)
+    return group_means(K, lab_k, Gk), counts
+
+
+def query_response_coords(Q, C, counts_k, scale, eps=RMS_EPS):
+    """Query-response coordinates [paperlayer App. B.2, C.1]; reading R4.
+
+    The logits of each query against the equally weighted, centred, nonempty
+    K/V-group centroids, divided by their RMS.  Returns (U_hat, rms, Ctilde).
+    """
+    ne = counts_k > 0
+    Cne = C[ne]
+    Ct = Cne - Cne.mean(axis=0, keepdims=True)
+    u = scale * (np.asarray(Q, np.float64) @ Ct.T)
+    rms = np.sqrt((u * u).mean(axis=1) + eps)
+    return u / rms[:, None], rms, Ct
+
+
+def group_major_permutation(lab, G):
+    """Stable group-major order and group offsets [paperlayer §4].
+
+    perm[i] is the original index of the row at permuted position i; rows of
+    one group keep their original relative order.
+    """
+    perm = np.argsort(np.asarray(lab), kind="stable")
+    counts = np.bincount(lab, minlength=G)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    return perm.astype(np.int64), off
+
+
+# ---------------------------------------------------------------------------
+# Routing [paperlayer §4 "Sparse Execution"]; reading R5
+# ---------------------------------------------------------------------------
+def route_logits(qbar, C, counts_k, scale):
+    """Centroid logit plus log group size, over nonempty K/V groups.
+
+    Returns an array [Gq, Gk] with -inf in columns of empty K/V groups.
+    """
+    Gk = C.shape[0]
+    L = np.full((qbar.shape[0], Gk), -np.inf)
+    ne = counts_k > 0
+    L[:, ne] = scale * (qbar @ C[ne].T) + np.log(counts_k[ne].astype(np.float64))[None, :]
+    return L
+
+
+def route_entry_mass(L):
+    """Per query group: softmax mass of each cell and its entry mass.
+
+    Cells are ranked by mass, descending, ties to the lower K/V index; a
+    cell's entry mass is the total mass ranked before it.  Columns with -inf
+    logits (empty K/V groups) get mass 0 and entry mass +inf (never routed).
+    """
+    Gq, Gk = L.shape
+    pi = np.zeros((Gq, Gk))
+    e = np.full((Gq, Gk), np.inf)
+    for i in range(Gq):
+        fin = np.isfinite(L[i])
+        if not fin.any():
+            continue
+        row = L[i][fin] - L[i][fin].max()
+        w = np.exp(row)
+        w = w / w.sum()
+        js = np.nonzero(fin)[0]
+        order = np.lexsort((js, -w))
+        before = np.concatenate([[0.0], np.cumsum(w[order])[:-1]])
+        pi[i, js] = w
+        e[i, js[order]] = before
+    return pi, e
+
+
+def route_select(e, counts_q, counts_k, mode, tau=0.9, rho_target=0.25, M=0):
+    """Boolean cell mask [Gq, Gk]; reading R5.  Empty query groups keep none.
+
+    Budget mode: the budget is rho_target*N_q*N_k - M*N_k pairs, compared in
+    fp64 against integer costs.
+    """
+    live = (counts_q > 0)[:, None] & (counts_k > 0)[None, :]
+    top = live & (e == 0.0)
+    if mode == "tau":
+        return (live & (e < tau)) | top
+    if mode != "budget":
+        raise ValueError(mode)
+    Nq, Nk = int(counts_q.sum()), int(counts_k.sum())
+    budget = rho_target * Nq * Nk - M * Nk
+    cost = counts_q[:, None].astype(np.float64) * counts_k[None, :]
+    # Kept cost as a function of the threshold v is the cumulative cost of
+    # live cells in ascending entry-mass order, read at the last cell with
+    # entry mass v; it is monotone, so the feasible values form a prefix.
+    ev, cv = e[live], cost[live]
+    order = np.argsort(ev, kind="stable")
+    ev, cv = ev[order], cv[order]
+    cum = np.cumsum(cv)
+    last = np.r_[ev[1:] != ev[:-1], True] if len(ev) else np.zeros(0, bool)
+    ok = np.nonzero(last & (cum <= budget))[0]
+    if len(ok) == 0:
+        return top
+    best = ev[ok.max()]
+    return (live & (e <= best)) | top
+
+
+def route_to_csr(mask):
+    """CSR of selected K/V groups per query group, columns ascending."""
+    row_ptr = np.concatenate([[0], np.cumsum(mask.sum(axis=1))]).astype(np.int64)
+    col_idx = np.nonzero(mask)[1].astype(np.int64)  # row-major: ascending j per row
+    return row_ptr, col_idx
+
+
+# ---------------------------------------------------------------------------
+# Probe selection [paperlayer §4, App. A.2; gist-nl §2B]; reading R6
+# ---------------------------------------------------------------------------
+def select_probes(counts_q, q_off, perm_q, M):
+    """Stratified probe rows and coverage weights.
+
+    Returns (probe_pos, probe_idx, weights, m_g): permuted positions, original
+    row indices (both ordered by group, then position), weights summing to 1,
+    and the per-group probe counts.
+    """
+    counts_q = np.asarray(counts_q, np.int64)
+    G = counts_q.shape[0]
+    N = int(counts_q.sum())
+    m = np.zeros(G, np.int64)
+    ne = np.nonzero(counts_q > 0)[0]
+    if M > N:
+        raise ValueError("more probes than rows")
+    if M > 0:
+        if M >= len(ne):
+            m[ne] = 1
+            R = M - len(ne)
+            S = N - len(ne)
+            if R > 0:
+                num = R * (counts_q - 1)
+                num[counts_q == 0] = 0
+                fl = num // S
+                rem = num % S
+                m += fl
+                left = R - int(fl.sum())
+                cand = [g for g in range(G) if rem[g] > 0]
+                cand.sort(key=lambda g: (-rem[g], g))
+                for g in cand[:left]:
+                    m[g] += 1
+        else:
+            order = sorted(ne.tolist(), key=lambda g: (-counts_q[g], g))
+            m[order[:M]] = 1
+    pos, wt = [], []
+    covered = int(counts_q[m > 0].sum())
+    for g in range(G):
+        for t in range(int(m[g])):
+            pos.append(int(q_off[g]) + ((2 * t + 1) * int(counts_q[g])) // (2 * int(m[g])))
+            wt.append((counts_q[g] / m[g]) / covered)
+    pos = np.array(pos, np.int64)
+    return pos, np.asarray(perm_q)[pos] if len(pos) else pos, np.array(wt, np.float64), m
+
+
+# ---------------------------------------------------------------------------
+# Routed attention under renormalized hard drop [paperlayer §1, §4]
+# ---------------------------------------------------------------------------
+def hard_drop_attention(Q, K, V, lab_q, lab_k, row_ptr, col_idx, scale, rows=None):
+    """Each query attends, with softmax renormalised over the retained keys,
+    to the union of the K/V groups routed to its query group.
+
+    ``rows`` restricts the output to the given original query indices (the
+    result then has one row per entry of ``rows``).  Rows of a query group
+    with no routed cell get zeros.
+    """
+    lab_q = np.asarray(lab_q)
+    lab_k = np.asarray(lab_k)
+    want = np.arange(Q.shape[0]) if rows is None else np.asarray(rows)
+    out = np.zeros((len(want), V.shape[1]))
+    gq = lab_q[want]
+    for i in np.unique(gq):
+        sel = np.nonzero(gq == i)[0]
+        cols = col_idx[row_ptr[i]:row_ptr[i + 1]]
+        if len(cols) == 0:
+            continue
+        keys = np.nonzero(np.isin(lab_k, cols))[0]
+        out[sel] = attention_rows(Q[want[sel]], K[keys], V[keys], scale)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Probe-Fitted Residual Reconstruction [paperlayer §4, App. A, A.3;
+# gist-nl §2B]; reading R7
+# ---------------------------------------------------------------------------
+def fit_residual(X, D, w, r, lam, sigma_drop=SIGMA_DROP):
+    """Fit the call-specific affine residual map on the probes.
+
+    X = sparse outputs of the probes (M x d), D = their dense outputs,
+    w = coverage weights (sum 1), R = D - X, Rbar = sum_t w_t R_t.
+    U_r holds the leading right singular vectors of the weighted, centred
+    residual W^1/2 (R - Rbar), i.e. the leading eigenvectors of its Gram
+    matrix, dropping directions with sigma <= sigma_drop * sigma_max.
+    The feature-dependent part is fitted inside that subspace by weighted
+    ridge on centred data: B = (Xc^T W Xc + lam I)^-1 Xc^T W (Rc U_r).
+    The estimator is R(x) = b + x B U_r^T with the full-width intercept
+    b = Rbar - xbar B U_r^T (only the feature-dependent term is restricted).
+    Returns (U, B, b, sigma): U is d x r_eff, B is d x r_eff, b has d entries,
+    sigma the singular values (descending).
+    """
+    X = np.asarray(X, np.float64)
+    R = np.asarray(D, np.float64) - X
+    w = np.asarray(w, np.float64)
+    d = X.shape[1]
+    Rbar = w @ R
+    Rc = R - Rbar
+    Gram = Rc.T @ (w[:, None] * Rc)
+    ev, U = np.linalg.eigh(Gram)
+    order = np.argsort(-ev, kind="stable")
+    ev, U = np.maximum(ev[order], 0.0), U[:, order]
+    sigma = np.sqrt(ev)
+    keep = 0
+    if sigma[0] > 0:
+        keep = int(min(r, np.count_nonzero(sigma > sigma_drop * sigma[0])))
+    U = U[:, :keep]
+    xbar = w @ X
+    Xc = X - xbar
+    Yc = Rc @ U
+    A = Xc.T @ (w[:, None] * Xc) + lam * np.eye(d)
+    B = np.linalg.solve(A, Xc.T @ (w[:, None] * Yc))
+    b = Rbar - (xbar @ B) @ U.T
+    return U, B, b, sigma
+
+
+def apply_correction(X, U, B, b):
+    """Estimated dense rows: x + b + x B U^T  [gist-nl §2B "Correctie"]."""
+    X = np.asarray(X, np.float64)
+    return X + b[None, :] + (X @ B) @ U.T
+
+
+def rho_exec(counts_q, counts_k, row_ptr, col_idx, M):
+    """Executed-pair density including probe rows [paperlayer §4, App. C.3].
+
+    Returns (routed_pairs, probe_pairs, rho).
+    """
+    routed = 0
+    for i in range(len(counts_q)):
+        for j in col_idx[row_ptr[i]:row_ptr[i + 1]]:
+            routed += int(counts_q[i]) * int(counts_k[j])
+    Nq, Nk = int(np.sum(counts_q)), int(np.sum(counts_k))
+    probe = int(M) * Nk
+    return routed, probe, (routed + probe) / (Nq * Nk)
+
+
+# ---------------------------------------------------------------------------
+# Whole call
+# ---------------------------------------------------------------------------
+def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
+                  rows=None, want_dense=False):
+    """One (batch, head) SparsePR call, fp64, following the pages' order.
+
+    Driven mode: ``lab_k`` / ``lab_q`` (and optionally ``csr``) replace the
+    oracle's own clustering (routing) so that everything downstream is
+    recomputed from given assignments.  ``rows`` limits the routed attention
+    and the output to those original rows (probe rows are always computed).
+    Returns a dict of every intermediate.
+    """
+    Q = np.asarray(Q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    N, d = Q.shape
+    s = prm.scale if prm.scale is not None else 1.0 / np.sqrt(d)
+    out = {"scale": s}
+    # Key-response coordinates and paired K/V groups
+    qs_idx = sample_query_indices(N, prm.Ms)
+    MK = response_metric(Q[qs_idx])
+    W, lamk = key_response_weights(MK, prm.p, prm.weight_power)
+    Z = K @ W
+    out.update(MK=MK, W=W, eig_MK=lamk, Z=Z)
+    if lab_k is None:
+        init_k = kmeans_init_indices(K.shape[0], prm.Gk, prm.seed, bh, 0)
+        lab_k, _, _, hist_k = kmeans(Z, prm.Gk, prm.iters, init_k)
+        out["kmeans_k_hist"] = hist_k
+    lab_k = np.asarray(lab_k, np.int64)
+    Cz = group_means(Z, lab_k, prm.Gk)
+    ne_k = np.bincount(lab_k, minlength=prm.Gk) > 0
+    out["obj_k"] = kmeans_objective(Z, lab_k, np.where(ne_k[:, None], Cz, 0.0))
+    C, counts_k = kv_centroids(K, lab_k, prm.Gk)
+    # Query-response coordinates and query groups
+    Uq, rms, Ct = query_response_coords(Q, C, counts_k, s)
+    if lab_q is None:
+        init_q = kmeans_init_indices(N, prm.Gq, prm.seed, bh, 1)
+        lab_q, _, _, hist_q = kmeans(Uq, prm.Gq, prm.iters, init_q)
+        out["kmeans_q_hist"] = hist_q
+    lab_q = np.asarray(lab_q, np.int64)
+    Cu = group_means(Uq, lab_q, prm.Gq)
+    ne_q = np.bincount(lab_q, minlength=prm.Gq) > 0
+    out["obj_q"] = kmeans_objective(Uq, lab_q, np.where(ne_q[:, None], Cu, 0.0))
+    out.update(lab_k=lab_k, lab_q=lab_q, C=C, counts_k=counts_k, rms=rms, Ctilde=Ct,
+               Cu=Cu)
+    # Group-major layouts
+    perm_k, kv_off = group_major_permutation(lab_k, prm.Gk)
+    perm_q, q_off = group_major_permutation(lab_q, prm.Gq)
+    counts_q = np.bincount(lab_q, minlength=prm.Gq).astype(np.int64)
+    qbar = group_means(Q, lab_q, prm.Gq)
+    out.update(perm_k=perm_k, kv_off=kv_off, perm_q=perm_q, q_off=q_off,
+               counts_q=counts_q, qbar=qbar)
+    # Routing
+    L = route_logits(np.nan_to_num(qbar), C, counts_k, s)
+    pi, e = route_entry_mass(L)
+    if csr is None:
+        mask = route_select(e, counts_q, counts_k, prm.route_mode, prm.tau,
+                            prm.rho_target, prm.M)
+        row_ptr, col_idx = route_to_csr(mask)
+    else:
+        row_ptr, col_idx = (np.asarray(a, np.int64) for a in csr)
+    out.update(route_logits=L, route_pi=pi, route_entry=e, row_ptr=row_ptr,
+               col_idx=col_idx)
+    # Probes
+    probe_pos, probe_idx, wts, m_g = select_probes(counts_q, q_off, perm_q, prm.M)
+    routed, probe_pairs, rho = rho_exec(counts_q, counts_k, row_ptr, col_idx, prm.M)
+    out.update(probe_pos=probe_pos, probe_idx=probe_idx, probe_w=wts, probe_m=m_g,
+               routed_pairs=routed, probe_pairs=probe_pairs, rho_exec=rho)
+    # Sparse execution and exact probe rows
+    want = np.arange(N) if rows is None else np.asarray(rows, np.int64)
+    O_sp = hard_drop_attention(Q, K, V, lab_q, lab_k, row_ptr, col_idx, s, rows=want)
+    out["rows"] = want
+    out["O_sp"] = O_sp
+    if prm.M > 0:
+        X = hard_drop_attention(Q, K, V, lab_q, lab_k, row_ptr, col_idx, s, rows=probe_idx)
+        Dn = attention_rows(Q[probe_idx], K, V, s)
+        U, B, b, sig = fit_residual(X, Dn, wts, prm.r, prm.lam)
+        O = apply_correction(O_sp, U, B, b)
+        is_probe = np.isin(want, probe_idx)
+        where = {int(t): k for k, t in enumerate(probe_idx)}
+        for k in np.nonzero(is_probe)[0]:
+            O[k] = Dn[where[int(want[k])]]
+        out.update(probe_sparse=X, probe_dense=Dn, U=U, B=B, b=b, sigma=sig)
+    else:
+        O = O_sp.copy()
+    out["O"] = O
+    if want_dense:
+        out["O_dense"] = dense_attention(Q[want], K, V, s)
+    return out
+
+
+def sparsepr_call(Q, K, V, prm: Params, **kw):
+    """All heads of a [B, H, N, d] call; returns a list of per-head dicts.
+
+    Keyword arrays given per head (lab_k, lab_q, csr, rows) are lists indexed
+    by flat head index b*H + h.
+    """
+    Bn, Hn = Q.shape[:2]
+    res = []
+    for b in range(Bn):
+        for h in range(Hn):
+            bh = b * Hn + h
+            per = {k: (v[bh] if v is not None else None) for k, v in kw.items()
+                   if k in ("lab_k", "lab_q", "csr", "rows")}
+            other = {k: v for k, v in kw.items() if k not in per}
+            res.append(sparsepr_head(Q[b, h], K[b, h], V[b, h], prm, bh=bh, **per, **other))
+    return res
