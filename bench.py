@@ -1,0 +1,352 @@
+#!/usr/bin/env python
+"""Benchmark of the SparsePR sparse attention call on B200.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload mid|hunyuan|wan|sweep|tiny]
+                    [--impl ours|reference]
+
+One step = one whole SparsePR call (partition, route, routed attention with
+exact probe rows, probe-fitted reconstruction and un-permute) over a batch of
+seeded synthetic Voronoi-center video tokens.  The default workload is the
+single-layer mid size: 24 heads x 8192 tokens (8x32x32 grid), d = 128, bf16,
+budget routing at rho_exec = 25% including probes.
+
+Metric: dense-equivalent TFLOP/s = 4 d N^2 (heads) / call time (higher is
+better); the JSON line also carries ms per call, executed-pair TFLOP/s, the
+stage breakdown, the attention kernel's roofline fraction, an end-to-end figure
+through host buffers, and the fp64 CPU oracle timed on this host as a baseline.
+
+Multi-GPU (torchrun): every rank runs its own heads (weak scaling); there is
+no collective on the data path, only a barrier and a max-reduction of the
+timings.  --impl reference times the CPU oracle (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from synthetic import voronoi_qkv, workload  # noqa: E402
+
+METRIC = "SparsePR ms/call & dense-equiv TFLOP/s at ρ_exec≈25%; rel-L2 vs dense"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def shard_heads(BH: int, rank: int, world: int):
+    """Flat head indices of one rank under weak scaling (each rank its own BH heads)."""
+    return list(range(rank * BH, (rank + 1) * BH))
+
+
+def reduce_max(values, world, device):
+    """Element-wise max over ranks of a list of floats (timing only)."""
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+def blas_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def oracle_head_seconds(wl, bh):
+    """Seconds the fp64 oracle takes for one whole head (independent mode)."""
+    from oracle import Params, sparsepr_head
+    prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
+                 tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index)
+    Q, K, V = voronoi_qkv(wl, heads=[bh])
+    q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
+    t0 = time.perf_counter()
+    sparsepr_head(q, k, v, prm, bh=bh)
+    return time.perf_counter() - t0
+
+
+def oracle_baseline(wl, budget_s=10.0):
+    """The oracle as it stands on whole heads of the workload, ~budget_s of CPU work."""
+    heads, t_tot = 0, 0.0
+    while heads < wl.BH and (heads == 0 or t_tot < budget_s):
+        t_tot += oracle_head_seconds(wl, heads)
+        heads += 1
+    flops = 4.0 * wl.d * wl.N * wl.N * heads
+    return {"value": flops / t_tot / 1e12, "unit": "TFLOP/s (dense-equivalent)",
+            "cores": blas_cores(), "kind": "oracle",
+            "sample": f"{heads} of {wl.BH} heads of {wl.name}, whole call, fp64 numpy, "
+                      f"{t_tot:.1f} s"}
+
+
+def config_of(wl, world):
+    return {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} ({'x'.join(map(str, wl.grid))}) "
+                        f"d={wl.d}", "heads_per_gpu": wl.BH, "tokens": wl.N, "head_dim": wl.d,
+            "Ms": wl.Ms, "p": wl.p, "Gk": wl.Gk, "Gq": wl.Gq, "iters": wl.iters,
+            "routing": (f"budget rho_target={wl.rho_target}" if wl.route_mode == "budget"
+                        else f"tau={wl.tau}"),
+            "M": wl.M, "r": wl.r, "lambda": wl.lam, "parallelism": f"heads x{world} (weak)",
+            "l2": "flushed (256 MiB write) before every timed call"}
+
+
+def run_reference(args, wl):
+    """The oracle as the reference arm: one whole head of the workload per step."""
+    world, rank, _ = dist_info()
+    if rank != 0:
+        return 0
+    times = []
+    for s in range(args.warmup + args.steps):
+        t = oracle_head_seconds(wl, s % wl.BH)
+        if s >= args.warmup:
+            times.append(t)
+    t = statistics.mean(times)
+    val = 4.0 * wl.d * wl.N * wl.N / t / 1e12
+    unit = "TFLOP/s (dense-equivalent)"
+    line = {"metric": METRIC, "value": val, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference", "config": config_of(wl, 1),
+            "cpu_baseline": {"value": val, "unit": unit, "cores": blas_cores(), "kind": "oracle",
+                             "sample": f"one whole head of {wl.name} per step"},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, wl):
+    import free_block_sparse_means_b200 as spr
+    world, rank, local = dist_info()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    spr.load_library()
+    heads = shard_heads(wl.BH, rank, world)
+    Qc, Kc, Vc = voronoi_qkv(wl, heads=heads)
+    shape = (wl.B, wl.H, wl.N, wl.d)
+    Qc, Kc, Vc = (t.reshape(shape).contiguous() for t in (Qc, Kc, Vc))
+    Q, K, V = (t.to(dev) for t in (Qc, Kc, Vc))
+    O = torch.empty_like(Q)
+    prm = spr.make_params(Q, K, V, O, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
+                          seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
+                          rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam)
+    ws = spr.alloc_workspace(prm, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call_staged(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        spr.sparsepr_partition(prm, Q, K, V, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        spr.sparsepr_route(prm, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        spr.sparsepr_attend(prm, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        spr.sparsepr_reconstruct(prm, ws, O, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        call_staged()
+    torch.cuda.synchronize(dev)
+    stats, err = spr.sparsepr_get_stats(prm, ws, stream)
+    if err:
+        raise SystemExit(f"device error word {err}")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    n0 = spr.sparsepr_launch_count()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            call_staged(evs[s])
+        torch.cuda.synchronize(dev)
+    n1 = spr.sparsepr_launch_count()
+    if world > 1:
+        torch.distributed.barrier()
+    stage = [[evs[s][i].elapsed_time(evs[s][i + 1]) for i in range(4)] for s in range(args.steps)]
+    per_call = [sum(x) for x in stage]
+    total_ms = sum(per_call)
+    stage_mean = [statistics.mean(x[i] for x in stage) for i in range(4)]
+    mx = reduce_max([total_ms] + stage_mean, world, dev)
+    total_ms_max, stage_max = mx[0], mx[1:]
+    ms_per_call = total_ms_max / args.steps
+    dense_flop = 4.0 * wl.d * wl.N * wl.N * wl.BH  # per rank
+    value = dense_flop * world / (ms_per_call * 1e-3) / 1e12
+    pairs = sum(h["routed_pairs"] + h["probe_pairs"] for h in stats)
+    tile_pairs = sum(h["tile_pairs"] for h in stats)
+    rho = pairs / (wl.N * wl.N * wl.BH)
+    exec_tflops = 4.0 * wl.d * pairs / (ms_per_call * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    attend_ms = stage_max[2]
+    att_achieved = 4.0 * wl.d * pairs / (attend_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": "k_attend (routed cells + probe rows)",
+            "achieved": att_achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": att_achieved / peaks["bf16_tflops"], "peak_source": f"{peak_kind} bf16 burst",
+            "traffic": None, "algorithmic_flop_per_launch": 4.0 * wl.d * pairs,
+            "executed_tile_pairs": tile_pairs, "true_pairs": pairs}
+    # partition: algorithmic HBM bytes (reads of Q, K, V per pass and the permuted copies)
+    part_bytes = float(wl.BH * wl.N * wl.d * 2) * ((wl.iters + 3) + (wl.iters + 2) + 2 * 3)
+    part_gbs = part_bytes / (stage_max[0] * 1e-3) / 1e9
+    # end to end through the public API with host buffers (pinned)
+    Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
+    Oh = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(e2e_steps)]
+    for s in range(e2e_steps):
+        flush.zero_()
+        ee[s][0].record(stream)
+        Q.copy_(Qh, non_blocking=True)
+        K.copy_(Kh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        spr.sparsepr_call(prm, Q, K, V, O, ws, stream)
+        Oh.copy_(O, non_blocking=True)
+        ee[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max([statistics.mean(a.elapsed_time(b) for a, b in ee)], world, dev)[0]
+    h2d = 3 * Q.numel() * 2
+    d2h = O.numel() * 2
+    clocks = clk.summary()
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s (dense-equivalent)",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_call, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 (fp32 accumulate)", "data": "synthetic",
+            "config": config_of(wl, world), "ms_per_call": ms_per_call,
+            "exec_pair_tflops": exec_tflops * world, "rho_exec": rho,
+            "stage_ms": {"partition": stage_max[0], "route": stage_max[1], "attend": stage_max[2],
+                         "reconstruct": stage_max[3]},
+            "roofline": roof,
+            "partition_hbm": {"achieved_gbs": part_gbs, "peak_gbs": peaks["hbm_gbs"],
+                              "frac": part_gbs / peaks["hbm_gbs"], "algorithmic_bytes": part_bytes},
+            "e2e": {"value": dense_flop * world / (e2e_ms * 1e-3) / 1e12,
+                    "unit": "TFLOP/s (dense-equivalent)", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(n1 - n0), "clocks": clocks, "device_error": err}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(wl, budget_s=args.cpu_budget)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mid")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

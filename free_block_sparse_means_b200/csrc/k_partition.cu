@@ -1,0 +1,873 @@
+// Response-Coupled Partitioning on the GPU [paperlayer §4, App. B.1, B.2;
+// gist-nl §2A]: sampled-query metric, its eigen-coordinates, key k-means,
+// paired K/V groups, centred K/V centroids, RMS-normalised query-response
+// coordinates (never materialised: the query k-means works in the head
+// dimension through Ctilde^T Ctilde), query k-means and the stable
+// group-major permutations of Q, K and V.
+#include <float.h>
+
+#include "spr_internal.cuh"
+
+namespace spr {
+
+int padded_p(int p) { return p <= 8 ? 8 : p <= 16 ? 16 : p <= 32 ? 32 : 64; }
+
+// ---------------------------------------------------------------------------
+// M_K = Q_s^T Q_s / M_s with Q_s the rows floor(i N / M_s), i < M_s.
+// Grid (BH, (D/32)^2), one 32x32 output tile per block.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_metric(TensorView Q, int N, int Ms, float* MK) {
+  const int bh = blockIdx.x;
+  const int ti = blockIdx.y / (D / 32), tj = blockIdx.y % (D / 32);
+  __shared__ float As[32][33], Bs[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s0 = 0; s0 < Ms; s0 += 32) {
+    for (int e = threadIdx.x; e < 32 * 32; e += 256) {
+      const int rr = e >> 5, c = e & 31, s = s0 + rr;
+      float a = 0.f, b = 0.f;
+      if (s < Ms) {
+        const int row = (int)(((int64_t)s * N) / Ms);
+        const bf16* q = Q.row(bh, row);
+        a = bf2f(q[ti * 32 + c]);
+        b = bf2f(q[tj * 32 + c]);
+      }
+      As[rr][c] = a;
+      Bs[rr][c] = b;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int rr = 0; rr < 32; ++rr) {
+      const float bv = Bs[rr][tx];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] += As[rr][ty * 4 + k] * bv;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    MK[((size_t)bh * D + ti * 32 + ty * 4 + k) * D + tj * 32 + tx] = acc[k] / (float)Ms;
+}
+
+
+// W[:, k] = u_k sqrt(lambda_k / sum_j lambda_j) for k < p; zero for p <= k < pp.
+__global__ void k_keyweights(const float* evals, const float* evecs, int D, int p, int pp,
+                             float* W) {
+  const int bh = blockIdx.x;
+  __shared__ float tot;
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < D; ++i) t += fmaxf(evals[(size_t)bh * D + i], 0.f);
+    tot = t;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < D * pp; e += blockDim.x) {
+    const int i = e / pp, k = e % pp;
+    float w = 0.f;
+    if (k < p && tot > 0.f)
+      w = evecs[((size_t)bh * D + i) * D + k] * sqrtf(fmaxf(evals[(size_t)bh * D + k], 0.f) / tot);
+    W[(size_t)bh * D * pp + e] = w;
+  }
+}
+
+// z_n = W^T k_n  (key-response coordinates).
+template <int D, int PP>
+__global__ void __launch_bounds__(256) k_project(TensorView K, int N, const float* W, float* Z) {
+  __shared__ __align__(16) float Ws[D * PP];
+  const int bh = blockIdx.y;
+  for (int e = threadIdx.x; e < D * PP; e += 256) Ws[e] = W[(size_t)bh * D * PP + e];
+  __syncthreads();
+  for (int n = blockIdx.x * 256 + threadIdx.x; n < N; n += gridDim.x * 256) {
+    const uint4* srow = reinterpret_cast<const uint4*>(K.row(bh, n));
+    float acc[PP];
+#pragma unroll
+    for (int k = 0; k < PP; ++k) acc[k] = 0.f;
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 raw = srow[c];
+      const bf16* v = reinterpret_cast<const bf16*>(&raw);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float x = bf2f(v[e]);
+        const float4* w = reinterpret_cast<const float4*>(&Ws[(c * 8 + e) * PP]);
+#pragma unroll
+        for (int k = 0; k < PP / 4; ++k) {
+          const float4 ww = w[k];
+          acc[4 * k] += x * ww.x;
+          acc[4 * k + 1] += x * ww.y;
+          acc[4 * k + 2] += x * ww.z;
+          acc[4 * k + 3] += x * ww.w;
+        }
+      }
+    }
+    float4* dst = reinterpret_cast<float4*>(Z + ((size_t)bh * N + n) * PP);
+#pragma unroll
+    for (int k = 0; k < PP / 4; ++k)
+      dst[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k-means initial rows: partial Fisher-Yates over 0..N-1 driven by splitmix64
+// (Steele, Lea & Flood 2014).  Stream state: seed XOR ((2 bh + which + 1) *
+// 0xD1B54A32D192ED03).  One block per (bh, which); a small open-addressing map
+// stores the displaced entries of the virtual identity array.
+// ---------------------------------------------------------------------------
+__global__ void k_init_idx(int N, int Gk, int Gq, uint64_t seed, int32_t* init_k,
+                           int32_t* init_q) {
+  constexpr int CAP = 2048;
+  __shared__ int keys[CAP], vals[CAP];
+  const int bh = blockIdx.x, which = blockIdx.y;
+  const int G = which ? Gq : Gk;
+  int32_t* out = (which ? init_q : init_k) + (size_t)bh * G;
+  for (int i = threadIdx.x; i < CAP; i += blockDim.x) keys[i] = -1;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  auto slot = [&](int k) {
+    uint32_t h = (uint32_t)k * 2654435761u;
+    int s = (int)(h & (CAP - 1));
+    while (keys[s] != -1 && keys[s] != k) s = (s + 1) & (CAP - 1);
+    return s;
+  };
+  auto get = [&](int k) {
+    const int s = slot(k);
+    return keys[s] == k ? vals[s] : k;
+  };
+  auto put = [&](int k, int v) {
+    const int s = slot(k);
+    keys[s] = k;
+    vals[s] = v;
+  };
+  uint64_t x = seed ^ ((uint64_t)(2 * bh + which + 1) * 0xD1B54A32D192ED03ull);
+  for (int i = 0; i < G; ++i) {
+    x += 0x9E3779B97F4A7C15ull;
+    uint64_t z = x;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    z ^= z >> 31;
+    const int j = i + (int)(z % (uint64_t)(N - i));
+    const int ai = get(i), aj = get(j);
+    put(i, aj);
+    put(j, ai);
+    out[i] = aj;
+  }
+}
+
+__global__ void k_init_centk(const float* Z, int N, int G, int PP, const int32_t* init,
+                             float* cent) {
+  const int bh = blockIdx.x;
+  for (int e = threadIdx.x; e < G * PP; e += blockDim.x) {
+    const int g = e / PP, k = e % PP;
+    cent[(size_t)bh * G * PP + e] = Z[((size_t)bh * N + init[(size_t)bh * G + g]) * PP + k];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Key assignment in eigen-coordinates: argmin_g ||z - c_g||^2 (ties to the
+// lowest g).  One block per CHUNK rows; also the chunk's label histogram.
+// ---------------------------------------------------------------------------
+template <int PP, int RPT>
+__global__ void __launch_bounds__(CHUNK / RPT) k_assign_z(const float* Z, int N, int G,
+                                                          const float* cent, int32_t* lab,
+                                                          int32_t* chunk_cnt, int nchunk) {
+  extern __shared__ __align__(16) float asm_[];
+  float* C = asm_;
+  float* cn = C + G * PP;
+  int* hist = reinterpret_cast<int*>(cn + G);
+  const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
+  constexpr int NT = CHUNK / RPT;
+  for (int e = tid; e < G * PP; e += NT) C[e] = cent[(size_t)bh * G * PP + e];
+  for (int g = tid; g < G; g += NT) hist[g] = 0;
+  __syncthreads();
+  for (int g = tid; g < G; g += NT) {
+    float s = 0.f;
+    for (int k = 0; k < PP; ++k) s += C[g * PP + k] * C[g * PP + k];
+    cn[g] = s;
+  }
+  __syncthreads();
+  float z[RPT][PP];
+  int n[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    n[r] = chunk * CHUNK + tid + r * NT;
+    const float4* src = reinterpret_cast<const float4*>(Z + ((size_t)bh * N + (n[r] < N ? n[r] : 0)) * PP);
+#pragma unroll
+    for (int k = 0; k < PP / 4; ++k) {
+      const float4 v = src[k];
+      z[r][4 * k] = v.x;
+      z[r][4 * k + 1] = v.y;
+      z[r][4 * k + 2] = v.z;
+      z[r][4 * k + 3] = v.w;
+    }
+  }
+  float best[RPT];
+  int arg[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    best[r] = FLT_MAX;
+    arg[r] = 0;
+  }
+  for (int g = 0; g < G; ++g) {
+    const float4* c4 = reinterpret_cast<const float4*>(C + g * PP);
+    float dot[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) dot[r] = 0.f;
+#pragma unroll
+    for (int k = 0; k < PP / 4; ++k) {
+      const float4 c = c4[k];
+#pragma unroll
+      for (int r = 0; r < RPT; ++r)
+        dot[r] += z[r][4 * k] * c.x + z[r][4 * k + 1] * c.y + z[r][4 * k + 2] * c.z +
+                  z[r][4 * k + 3] * c.w;
+    }
+    const float cg = cn[g];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      const float sc = cg - 2.f * dot[r];
+      if (sc < best[r]) {
+        best[r] = sc;
+        arg[r] = g;
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RPT; ++r)
+    if (n[r] < N) {
+      lab[(size_t)bh * N + n[r]] = arg[r];
+      atomicAdd(&hist[arg[r]], 1);
+    }
+  __syncthreads();
+  for (int g = tid; g < G; g += NT) chunk_cnt[((size_t)bh * nchunk + chunk) * G + g] = hist[g];
+}
+
+// ---------------------------------------------------------------------------
+// Per (bh, g): base of each chunk within the group (exclusive scan over
+// chunks), group sizes, and group offsets (exclusive scan over g).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_chunk_scan(const int32_t* chunk_cnt, int nchunk, int G,
+                                                    int N, int32_t* cbase, int32_t* off,
+                                                    int32_t* counts) {
+  __shared__ int wsum[8];
+  const int bh = blockIdx.x, g = threadIdx.x;
+  int tot = 0;
+  if (g < G) {
+    for (int c = 0; c < nchunk; ++c) {
+      const size_t i = ((size_t)bh * nchunk + c) * G + g;
+      cbase[i] = tot;
+      tot += chunk_cnt[i];
+    }
+    counts[(size_t)bh * G + g] = tot;
+  }
+  // block exclusive scan of tot over g
+  int v = tot;
+  const int lane = g & 31, w = g >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) wsum[w] = v;
+  __syncthreads();
+  int before = 0;
+  for (int i = 0; i < w; ++i) before += wsum[i];
+  if (g < G) off[(size_t)bh * (G + 1) + g] = before + v - tot;
+  if (g == 0) off[(size_t)bh * (G + 1) + G] = N;
+}
+
+// Stable scatter: perm[off[g] + chunk base + rank among equal labels before
+// this row in the chunk] = row.
+__global__ void __launch_bounds__(1024) k_scatter(const int32_t* lab, int N, int G, int nchunk,
+                                                  const int32_t* cbase, const int32_t* off,
+                                                  int32_t* perm, Header* hdr) {
+  __shared__ int cnt[32][MAX_GROUPS];
+  const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
+  const int w = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < 32 * G; e += 1024) cnt[e / G][e % G] = 0;
+  __syncthreads();
+  const int n = chunk * CHUNK + tid;
+  int g = n < N ? lab[(size_t)bh * N + n] : -1;
+  if (g >= G || g < -1) {
+    set_error(hdr, ERR_INDEX, 1, bh, n);
+    g = -1;
+  }
+  const unsigned mask = __match_any_sync(0xffffffffu, g);
+  const int rank_w = __popc(mask & ((1u << lane) - 1u));
+  if (g >= 0 && (__ffs(mask) - 1) == lane) cnt[w][g] = __popc(mask);
+  __syncthreads();
+  if (g >= 0) {
+    int before = 0;
+    for (int i = 0; i < w; ++i) before += cnt[i][g];
+    const int pos = off[(size_t)bh * (G + 1) + g] + cbase[((size_t)bh * nchunk + chunk) * G + g] +
+                    before + rank_w;
+    if (pos < 0 || pos >= N)
+      set_error(hdr, ERR_INDEX, 2, bh, pos);
+    else
+      perm[(size_t)bh * N + pos] = n;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Segmented sums over the members of each group (fixed order, fp64
+// accumulation, deterministic).  Modes:
+//   SEG_Z       rows of Z (fp32, PP wide) at perm[i]          -> k-means update
+//   SEG_QSCALED rows (s / rms_n) q_n at n = perm[i]           -> k-means update
+//   SEG_BF16    rows i of a contiguous permuted bf16 buffer     -> means
+// keep_empty: an empty group keeps out's previous row, else it is zeroed.
+// ---------------------------------------------------------------------------
+enum { SEG_Z = 0, SEG_QSCALED = 1, SEG_BF16 = 2 };
+
+struct SegArgs {
+  const float* Z;
+  TensorView Q;
+  const float* rms;
+  float scale;
+  const bf16* Xp;
+  const int32_t* perm;
+  const int32_t* off;
+  int N, G;
+  float* out;
+  int keep_empty;
+};
+
+template <int MODE, int DD>
+__global__ void __launch_bounds__(128) k_segsum(SegArgs a) {
+  constexpr int NV = (MODE == SEG_Z) ? (DD + 31) / 32 : DD / 32;  // values per lane
+  __shared__ double red[4][DD];
+  const int bh = blockIdx.y, g = blockIdx.x, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int start = a.off[(size_t)bh * (a.G + 1) + g], end = a.off[(size_t)bh * (a.G + 1) + g + 1];
+  double acc[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) acc[v] = 0.0;
+  for (int i = start + w; i < end; i += 4) {
+    if (MODE == SEG_Z) {
+      const int row = a.perm[(size_t)bh * a.N + i];
+      const float* src = a.Z + ((size_t)bh * a.N + row) * DD;
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+        if (lane + 32 * v < DD) acc[v] += (double)src[lane + 32 * v];
+    } else {
+      const bf16* src;
+      float sc = 1.f;
+      if (MODE == SEG_QSCALED) {
+        const int row = a.perm[(size_t)bh * a.N + i];
+        src = a.Q.row(bh, row);
+        sc = a.scale / a.rms[(size_t)bh * a.N + row];
+      } else {
+        src = a.Xp + ((size_t)bh * a.N + i) * DD;
+      }
+#pragma unroll
+      for (int v = 0; v < NV / 2; ++v) {
+        const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(src)[lane + 32 * v];
+        acc[2 * v] += (double)(sc * __low2float(x));
+        acc[2 * v + 1] += (double)(sc * __high2float(x));
+      }
+    }
+  }
+  if (MODE == SEG_Z) {
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
+      if (lane + 32 * v < DD) red[w][lane + 32 * v] = acc[v];
+  } else {
+#pragma unroll
+    for (int v = 0; v < NV / 2; ++v) {
+      red[w][2 * (lane + 32 * v)] = acc[2 * v];
+      red[w][2 * (lane + 32 * v) + 1] = acc[2 * v + 1];
+    }
+  }
+  __syncthreads();
+  const int cnt = end - start;
+  for (int k = threadIdx.x; k < DD; k += 128) {
+    const double s = red[0][k] + red[1][k] + red[2][k] + red[3][k];
+    float* o = a.out + ((size_t)bh * a.G + g) * DD + k;
+    if (cnt > 0)
+      *o = (float)(s / cnt);
+    else if (!a.keep_empty)
+      *o = 0.f;
+  }
+}
+
+// Key objective with the final centroids: sum_n ||z_n - c_{lab_n}||^2 (fp64
+// partial per chunk).
+template <int PP>
+__global__ void __launch_bounds__(256) k_obj_z(const float* Z, int N, int G, const float* cent,
+                                               const int32_t* lab, int nchunk, double* part) {
+  __shared__ double red[8];
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  double acc = 0.0;
+  for (int n = chunk * CHUNK + threadIdx.x; n < min(N, (chunk + 1) * CHUNK); n += 256) {
+    const int g = lab[(size_t)bh * N + n];
+    const float* z = Z + ((size_t)bh * N + n) * PP;
+    const float* c = cent + ((size_t)bh * G + g) * PP;
+    float s = 0.f;
+    for (int k = 0; k < PP; ++k) {
+      const float t = z[k] - c[k];
+      s += t * t;
+    }
+    acc += s;
+  }
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < 8; ++i) s += red[i];
+    part[((size_t)bh * 2 + 0) * (nchunk + 1) + chunk] = s;
+  }
+}
+
+// Permuted copy of bf16 rows: dst[bh, i, :] = src.row(bh, perm[bh, i]).
+template <int D>
+__global__ void __launch_bounds__(256) k_gather_rows(TensorView src, const int32_t* perm, int N,
+                                                     int BH, bf16* dst) {
+  constexpr int LANES = D / 8;  // uint4 per row
+  const int64_t total = (int64_t)BH * N * LANES;
+  for (int64_t e = (int64_t)blockIdx.x * 256 + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * 256) {
+    const int64_t rowi = e / LANES;
+    const int c = (int)(e % LANES);
+    const int bh = (int)(rowi / N), i = (int)(rowi % N);
+    const int n = perm[rowi];
+    reinterpret_cast<uint4*>(dst)[e] = reinterpret_cast<const uint4*>(src.row(bh, n))[c];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Centred nonempty K/V centroids [paperlayer App. B.2]: Ctilde rows (compacted,
+// ascending group index) = c_j - mean over nonempty j of c_j.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_center(const float* Craw, const int32_t* counts, int G,
+                                                int D, float* Ct, spr_head_stats* stats) {
+  __shared__ int idx[MAX_GROUPS];
+  __shared__ int nne;
+  const int bh = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int k = 0;
+    for (int j = 0; j < G; ++j)
+      if (counts[(size_t)bh * G + j] > 0) idx[k++] = j;
+    nne = k;
+    stats[bh].gk_nonempty = k;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += 256) {
+    double s = 0.0;
+    for (int t = 0; t < nne; ++t) s += Craw[((size_t)bh * G + idx[t]) * D + c];
+    const float mean = nne ? (float)(s / nne) : 0.f;
+    for (int t = 0; t < G; ++t)
+      Ct[((size_t)bh * G + t) * D + c] =
+          t < nne ? Craw[((size_t)bh * G + idx[t]) * D + c] - mean : 0.f;
+  }
+}
+
+// A = Ctilde^T Ctilde (D x D) and its bf16 hi/lo split for the tensor-core
+// quadratic form.  Grid (BH, (D/32)^2).
+__global__ void __launch_bounds__(256) k_amat(const float* Ct, int G, int D,
+                                              const spr_head_stats* stats, float* A, bf16* split,
+                                              int split_rows) {
+  __shared__ float As[32][33], Bs[32][33];
+  const int bh = blockIdx.x, nt = D / 32;
+  const int ti = blockIdx.y / nt, tj = blockIdx.y % nt;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int nne = stats[bh].gk_nonempty;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int t0 = 0; t0 < nne; t0 += 32) {
+    for (int e = threadIdx.x; e < 1024; e += 256) {
+      const int rr = e >> 5, c = e & 31, t = t0 + rr;
+      As[rr][c] = t < nne ? Ct[((size_t)bh * G + t) * D + ti * 32 + c] : 0.f;
+      Bs[rr][c] = t < nne ? Ct[((size_t)bh * G + t) * D + tj * 32 + c] : 0.f;
+    }
+    __syncthreads();
+    for (int rr = 0; rr < 32; ++rr) {
+      const float bv = Bs[rr][tx];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] += As[rr][ty * 4 + k] * bv;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = ti * 32 + ty * 4 + k, j = tj * 32 + tx;
+    const float v = acc[k];
+    A[((size_t)bh * D + i) * D + j] = v;
+    const bf16 hi = __float2bfloat16_rn(v);
+    const bf16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    // split layout [BH][2][split_rows][D]; row = output column j, k-index = i
+    split[(((size_t)bh * 2 + 0) * split_rows + j) * D + i] = hi;
+    split[(((size_t)bh * 2 + 1) * split_rows + j) * D + i] = lo;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core row GEMM over the queries of one head (mma.sync m16n8k16 bf16,
+// fp32 accumulation) with the B operand split into bf16 hi + lo so that the
+// products carry ~16 bits of the fp32 B.
+//   QUAD  : B = A (D x D); per row qAq -> rms = sqrt(s^2 qAq / G'k + eps),
+//           ||u_hat||^2 = s^2 qAq / rms^2  (query-response RMS, reading R4)
+//   assign: B rows = Bq_g = A a_g; score_g = (s / rms_n) q.Bq_g - beta_g;
+//           label = argmax (ties to the lowest g)  (query k-means assignment
+//           in factored form: u.m_g - ||m_g||^2 / 2 with m_g = Ctilde a_g)
+// One block per CHUNK rows (8 sub-tiles of 128), 8 warps x 16 rows.
+// ---------------------------------------------------------------------------
+struct RowGemmArgs {
+  TensorView Q;
+  int N, G, nchunk, split_rows;
+  const bf16* bsplit;   // [BH][2][split_rows][D]
+  const float* beta;    // [BH][G]
+  float scale;
+  const spr_head_stats* stats;
+  float* rms;
+  float* un2;
+  int32_t* lab;
+  int32_t* chunk_cnt;
+  double* part;
+  Header* hdr;
+};
+
+template <int D, bool QUAD>
+__global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  extern __shared__ __align__(128) uint8_t rsm[];
+  const int NC = QUAD ? D : ((a.G + 31) / 32) * 32;  // padded B rows
+  uint8_t* Bhi = rsm;
+  uint8_t* Blo = Bhi + NC * D * 2;
+  uint8_t* Qs = Blo + NC * D * 2;
+  float* betas = reinterpret_cast<float*>(Qs + ATT_BM * D * 2);
+  int* hist = reinterpret_cast<int*>(betas + MAX_GROUPS);
+  double* red = reinterpret_cast<double*>(hist + MAX_GROUPS);
+  const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int nrows_b = QUAD ? D : a.G;
+  // B operand, swizzled rows
+  const bf16* bsrc = a.bsplit + (size_t)bh * 2 * a.split_rows * D;
+  for (int e = tid; e < NC * CH; e += 256) {
+    const int r = e / CH, c = e % CH;
+    uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
+    if (r < nrows_b) {
+      hi = reinterpret_cast<const uint4*>(bsrc + (size_t)r * D)[c];
+      lo = reinterpret_cast<const uint4*>(bsrc + ((size_t)a.split_rows + r) * D)[c];
+    }
+    *reinterpret_cast<uint4*>(Bhi + swz<CH>(r, c)) = hi;
+    *reinterpret_cast<uint4*>(Blo + swz<CH>(r, c)) = lo;
+  }
+  if (!QUAD)
+    for (int g = tid; g < MAX_GROUPS; g += 256) {
+      betas[g] = g < a.G ? a.beta[(size_t)bh * a.G + g] : 0.f;
+      hist[g] = 0;
+    }
+  const float gk = QUAD ? (float)max(1, a.stats[bh].gk_nonempty) : 1.f;
+  double un2acc = 0.0;
+  for (int sub = 0; sub < CHUNK / ATT_BM; ++sub) {
+    const int row0 = chunk * CHUNK + sub * ATT_BM;
+    if (row0 >= a.N) break;
+    __syncthreads();  // previous tile consumed
+    for (int e = tid; e < ATT_BM * CH; e += 256) {
+      const int r = e / CH, c = e % CH, n = row0 + r;
+      const bf16* src = a.Q.row(bh, n < a.N ? n : 0) + c * 8;
+      cp_async16(Qs + swz<CH>(r, c), src, n < a.N ? 16 : 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    // A fragments for this warp's 16 rows
+    uint32_t af[D / 16][4];
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int c = ks * 2 + (lane >> 4);
+      ldsm_x4(af[ks][0], af[ks][1], af[ks][2], af[ks][3], Qs + swz<CH>(r, c));
+    }
+    const int r_lo = row0 + warp * 16 + gid, r_hi = r_lo + 8;
+    float alpha_lo = 1.f, alpha_hi = 1.f;
+    if (!QUAD) {
+      alpha_lo = r_lo < a.N ? a.scale / a.rms[(size_t)bh * a.N + r_lo] : 0.f;
+      alpha_hi = r_hi < a.N ? a.scale / a.rms[(size_t)bh * a.N + r_hi] : 0.f;
+    }
+    float best_lo = -FLT_MAX, best_hi = -FLT_MAX, quad_lo = 0.f, quad_hi = 0.f;
+    int arg_lo = 0, arg_hi = 0;
+    for (int nc = 0; nc < NC; nc += 32) {
+      float acc[4][4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {  // two n-tile pairs of 16 columns
+          const int brow = nc + pr * 16 + (lane & 7) + (lane >> 4) * 8;
+          const int bc = ks * 2 + ((lane >> 3) & 1);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(b0, b1, b2, b3, Bhi + swz<CH>(brow, bc));
+          mma16816(acc[pr * 2], af[ks], b0, b1);
+          mma16816(acc[pr * 2 + 1], af[ks], b2, b3);
+          ldsm_x4(b0, b1, b2, b3, Blo + swz<CH>(brow, bc));
+          mma16816(acc[pr * 2], af[ks], b0, b1);
+          mma16816(acc[pr * 2 + 1], af[ks], b2, b3);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int col = nc + t * 8 + 2 * tig;
+        if (QUAD) {
+          // q values at (row, col), (row, col+1) from the swizzled tile
+          const int rl = warp * 16 + gid, rh = rl + 8;
+          const bf16* ql = reinterpret_cast<const bf16*>(Qs + swz<CH>(rl, col / 8)) + (col & 7);
+          const bf16* qh = reinterpret_cast<const bf16*>(Qs + swz<CH>(rh, col / 8)) + (col & 7);
+          quad_lo += acc[t][0] * bf2f(ql[0]) + acc[t][1] * bf2f(ql[1]);
+          quad_hi += acc[t][2] * bf2f(qh[0]) + acc[t][3] * bf2f(qh[1]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int g = col + e;
+            if (g < a.G) {
+              const float sl = alpha_lo * acc[t][e] - betas[g];
+              const float sh = alpha_hi * acc[t][2 + e] - betas[g];
+              if (sl > best_lo) { best_lo = sl; arg_lo = g; }
+              if (sh > best_hi) { best_hi = sh; arg_hi = g; }
+            }
+          }
+        }
+      }
+    }
+    if (QUAD) {
+      quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 1);
+      quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 2);
+      quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 1);
+      quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 2);
+      if (tig == 0) {
+        const float s2 = a.scale * a.scale;
+        if (r_lo < a.N) {
+          const float ms = s2 * fmaxf(quad_lo, 0.f) / gk;
+          const float rr = sqrtf(ms + 1e-6f);
+          a.rms[(size_t)bh * a.N + r_lo] = rr;
+          const float u2 = s2 * fmaxf(quad_lo, 0.f) / (rr * rr);
+          a.un2[(size_t)bh * a.N + r_lo] = u2;
+          un2acc += u2;
+        }
+        if (r_hi < a.N) {
+          const float ms = s2 * fmaxf(quad_hi, 0.f) / gk;
+          const float rr = sqrtf(ms + 1e-6f);
+          a.rms[(size_t)bh * a.N + r_hi] = rr;
+          const float u2 = s2 * fmaxf(quad_hi, 0.f) / (rr * rr);
+          a.un2[(size_t)bh * a.N + r_hi] = u2;
+          un2acc += u2;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        const float bl = __shfl_xor_sync(0xffffffffu, best_lo, o);
+        const int al = __shfl_xor_sync(0xffffffffu, arg_lo, o);
+        if (bl > best_lo || (bl == best_lo && al < arg_lo)) { best_lo = bl; arg_lo = al; }
+        const float bhv = __shfl_xor_sync(0xffffffffu, best_hi, o);
+        const int ah = __shfl_xor_sync(0xffffffffu, arg_hi, o);
+        if (bhv > best_hi || (bhv == best_hi && ah < arg_hi)) { best_hi = bhv; arg_hi = ah; }
+      }
+      if (tig == 0) {
+        if (r_lo < a.N) {
+          a.lab[(size_t)bh * a.N + r_lo] = arg_lo;
+          atomicAdd(&hist[arg_lo], 1);
+        }
+        if (r_hi < a.N) {
+          a.lab[(size_t)bh * a.N + r_hi] = arg_hi;
+          atomicAdd(&hist[arg_hi], 1);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (QUAD) {
+    un2acc = warp_sum(un2acc);
+    if (lane == 0) red[warp] = un2acc;
+    __syncthreads();
+    if (tid == 0) {
+      double s = 0.0;
+      for (int i = 0; i < 8; ++i) s += red[i];
+      a.part[((size_t)bh * 2 + 1) * (a.nchunk + 1) + chunk] = s;
+    }
+  } else {
+    for (int g = tid; g < a.G; g += 256)
+      a.chunk_cnt[((size_t)bh * a.nchunk + chunk) * a.G + g] = hist[g];
+  }
+}
+
+// Initial query centroids: a_g = (s / rms_n) q_n at the seeded rows.
+__global__ void k_init_centq(TensorView Q, int N, int G, int D, const int32_t* init,
+                             const float* rms, float scale, float* centq) {
+  const int bh = blockIdx.x;
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+    const int g = e / D, c = e % D;
+    const int n = init[(size_t)bh * G + g];
+    centq[(size_t)bh * G * D + e] = scale / rms[(size_t)bh * N + n] * bf2f(Q.row(bh, n)[c]);
+  }
+}
+
+// Bq_g = A a_g, beta_g = a_g . Bq_g / 2 (= ||m_g||^2 / 2), bf16 hi/lo split of Bq.
+// Grid (BH, G), D threads.  Also n_g * a_g^T A a_g into part for the objective.
+__global__ void k_qprep(const float* A, const float* centq, int G, int D, const int32_t* counts,
+                        float* beta, bf16* split, int split_rows, double* qterm) {
+  __shared__ float av[128];
+  __shared__ float red[4];
+  const int bh = blockIdx.x, g = blockIdx.y, i = threadIdx.x;
+  av[i] = centq[((size_t)bh * G + g) * D + i];
+  __syncthreads();
+  float s = 0.f;
+  const float* Ab = A + (size_t)bh * D * D;
+  for (int j = 0; j < D; ++j) s += Ab[(size_t)j * D + i] * av[j];  // A symmetric
+  const bf16 hi = __float2bfloat16_rn(s);
+  const bf16 lo = __float2bfloat16_rn(s - __bfloat162float(hi));
+  split[(((size_t)bh * 2 + 0) * split_rows + g) * D + i] = hi;
+  split[(((size_t)bh * 2 + 1) * split_rows + g) * D + i] = lo;
+  float t = warp_sum(s * av[i]);
+  if ((i & 31) == 0) red[i >> 5] = t;
+  __syncthreads();
+  if (i == 0) {
+    float q = 0.f;
+    for (int w = 0; w < D / 32; ++w) q += red[w];
+    beta[(size_t)bh * G + g] = 0.5f * q;
+    if (qterm) qterm[(size_t)bh * G + g] = (double)counts[(size_t)bh * G + g] * (double)q;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host orchestration of stage 1.
+// ---------------------------------------------------------------------------
+template <int D>
+static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs& P,
+                               const TensorView& Q, const TensorView& K, const TensorView& V,
+                               cudaStream_t st) {
+  const int BH = L.BH, N = p.N, nchunk = L.nchunk, pp = padded_p(p.p);
+  const float scale = p.scale > 0.f ? p.scale : 1.f / sqrtf((float)D);
+  const int sms = num_sms();
+  cudaError_t e;
+  // Key-response coordinates
+  spr_launch(k_metric<D>, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, Q, N, p.Ms, P.MK);
+  if ((e = launch_eig(P.MK, BH, D, P.eval, P.evec, st)) != cudaSuccess) return e;
+  spr_launch(k_keyweights, BH, 256, 0, st, P.eval, P.evec, D, p.p, pp, P.W);
+  const int pgrid = min((N + 255) / 256, max(1, 4 * sms / BH + 1));
+#define PROJ(PPV) spr_launch(k_project<D, PPV>, dim3(pgrid, BH), 256, 0, st, K, N, P.W, P.Z)
+  if (pp == 8) PROJ(8); else if (pp == 16) PROJ(16); else if (pp == 32) PROJ(32); else PROJ(64);
+#undef PROJ
+  spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
+  spr_launch(k_init_centk, BH, 256, 0, st, P.Z, N, p.Gk, pp, P.initk, P.centk);
+  // Key k-means
+  const size_t asmem = (size_t)p.Gk * pp * 4 + p.Gk * 4 + p.Gk * 4;
+  for (int it = 0; it < p.iters; ++it) {
+#define ASG(PPV, RPT)                                                                      \
+  do {                                                                                     \
+    cudaFuncSetAttribute(k_assign_z<PPV, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                         (int)asmem);                                                      \
+    spr_launch(k_assign_z<PPV, RPT>, dim3(nchunk, BH), CHUNK / RPT, asmem, st,                     \
+        P.Z, N, p.Gk, P.centk, P.labk, P.chunk, nchunk);                                   \
+  } while (0)
+    if (pp == 8) ASG(8, 4); else if (pp == 16) ASG(16, 4); else if (pp == 32) ASG(32, 2); else ASG(64, 1);
+#undef ASG
+    spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gk, N, P.cbase, P.kvoff, P.counts);
+    spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labk, N, p.Gk, nchunk, P.cbase, P.kvoff,
+                                                 P.permk, P.hdr);
+    SegArgs sa{};
+    sa.Z = P.Z;
+    sa.perm = P.permk;
+    sa.off = P.kvoff;
+    sa.N = N;
+    sa.G = p.Gk;
+    sa.out = P.centk;
+    sa.keep_empty = 1;
+#define SEGZ(PPV) spr_launch(k_segsum<SEG_Z, PPV>, dim3(p.Gk, BH), 128, 0, st, sa)
+    if (pp == 8) SEGZ(8); else if (pp == 16) SEGZ(16); else if (pp == 32) SEGZ(32); else SEGZ(64);
+#undef SEGZ
+  }
+#define OBJZ(PPV) \
+  spr_launch(k_obj_z<PPV>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.labk, nchunk, P.part)
+  if (pp == 8) OBJZ(8); else if (pp == 16) OBJZ(16); else if (pp == 32) OBJZ(32); else OBJZ(64);
+#undef OBJZ
+  // Paired K/V groups: permuted keys and values, raw-key centroids
+  const int ggrid = sms * 8;
+  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
+  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
+  {
+    SegArgs sa{};
+    sa.Xp = P.Kp;
+    sa.off = P.kvoff;
+    sa.N = N;
+    sa.G = p.Gk;
+    sa.out = P.Craw;
+    sa.keep_empty = 0;
+    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gk, BH), 128, 0, st, sa);
+  }
+  // P.counts holds |K_j| now; keep a copy of key counts in kv_off differences.
+  spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
+  const int split_rows = p.Gq > D ? p.Gq : D;
+  spr_launch(k_amat, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, P.Ct, p.Gk, D, P.stats, P.Amat, P.bq16,
+                                                         split_rows);
+  // Query-response RMS (tensor-core quadratic form)
+  RowGemmArgs ra{};
+  ra.Q = Q;
+  ra.N = N;
+  ra.G = p.Gq;
+  ra.nchunk = nchunk;
+  ra.split_rows = split_rows;
+  ra.bsplit = P.bq16;
+  ra.beta = P.beta;
+  ra.scale = scale;
+  ra.stats = P.stats;
+  ra.rms = P.rms;
+  ra.un2 = P.un2;
+  ra.lab = P.labq;
+  ra.chunk_cnt = P.chunk;
+  ra.part = P.part;
+  ra.hdr = P.hdr;
+  {
+    const size_t sm = (size_t)2 * D * D * 2 + ATT_BM * D * 2 + MAX_GROUPS * 8 + 64;
+    cudaFuncSetAttribute(k_rowgemm<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    spr_launch(k_rowgemm<D, true>, dim3(nchunk, BH), 256, sm, st, ra);
+  }
+  // Query k-means in the head dimension
+  spr_launch(k_init_centq, BH, 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale, P.centq);
+  const int ncq = ((p.Gq + 31) / 32) * 32;
+  const size_t smq = (size_t)2 * ncq * D * 2 + ATT_BM * D * 2 + MAX_GROUPS * 8 + 64;
+  cudaFuncSetAttribute(k_rowgemm<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq);
+  for (int it = 0; it < p.iters; ++it) {
+    spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
+                                          split_rows, nullptr);
+    spr_launch(k_rowgemm<D, false>, dim3(nchunk, BH), 256, smq, st, ra);
+    spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gq, N, P.cbase, P.qoff, P.counts);
+    spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labq, N, p.Gq, nchunk, P.cbase, P.qoff,
+                                                 P.permq, P.hdr);
+    SegArgs sa{};
+    sa.Q = Q;
+    sa.rms = P.rms;
+    sa.scale = scale;
+    sa.perm = P.permq;
+    sa.off = P.qoff;
+    sa.N = N;
+    sa.G = p.Gq;
+    sa.out = P.centq;
+    sa.keep_empty = 1;
+    spr_launch(k_segsum<SEG_QSCALED, D>, dim3(p.Gq, BH), 128, 0, st, sa);
+  }
+  // objective terms n_g a_g^T A a_g with the final centroids (into part's tail)
+  spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
+                                        split_rows, P.part + (size_t)BH * 2 * (nchunk + 1));
+  // Group-major queries and raw query means
+  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, Q, P.permq, N, BH, P.Qp);
+  {
+    SegArgs sa{};
+    sa.Xp = P.Qp;
+    sa.off = P.qoff;
+    sa.N = N;
+    sa.G = p.Gq;
+    sa.out = P.qbar;
+    sa.keep_empty = 0;
+    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gq, BH), 128, 0, st, sa);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_partition(const spr_params& p, const Layout& L, const Ptrs& P,
+                             const TensorView& Q, const TensorView& K, const TensorView& V,
+                             cudaStream_t st) {
+  if (p.d == 64) return partition_d<64>(p, L, P, Q, K, V, st);
+  return partition_d<128>(p, L, P, Q, K, V, st);
+}
+
+}  // namespace spr

@@ -1,0 +1,207 @@
+// Internal declarations shared by the SparsePR CUDA sources (not part of the
+// public C ABI).  Workspace layout, launch helpers and device utilities.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sparsepr.h"
+
+namespace spr {
+
+typedef __nv_bfloat16 bf16;
+
+constexpr int CHUNK = 1024;        // rows per histogram chunk (k-means, permutation)
+constexpr int MAX_GROUPS = 256;    // Gk, Gq upper bound
+constexpr int MAX_P = 64;          // eigen-coordinate upper bound
+constexpr int MAX_PROBES = 4096;   // M upper bound
+constexpr int ATT_BM = 128;        // query rows per attention work item
+
+// Device error word codes (first error wins; info words carry details).
+enum : int32_t {
+  ERR_NONE = 0,
+  ERR_INDEX = 1,       // an index read from the workspace is out of range
+  ERR_WORKLIST = 2,    // attention work list overflow
+  ERR_NUMERIC = 3,     // non-finite value where the method needs a finite one
+  ERR_TIMEOUT = 4,     // a bounded wait gave up
+};
+
+// Workspace buffers.
+enum Buf : int {
+  B_HDR, B_STATS, B_MK, B_EVAL, B_EVEC, B_W, B_Z, B_INITK, B_INITQ, B_CENTK,
+  B_LABK, B_LABQ, B_CHUNK, B_CBASE, B_COUNTS, B_PERMK, B_KVOFF, B_PERMQ, B_QOFF,
+  B_KP, B_VP, B_QP, B_CRAW, B_CT, B_AMAT, B_RMS, B_UN2, B_CENTQ, B_BQ16, B_BETA,
+  B_QBAR, B_LOGIT, B_ENTRY, B_TOP, B_SEL, B_ROWPTR, B_COLIDX, B_RUNPTR, B_RUNS, B_PPOS,
+  B_PIDX, B_PW, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
+  B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_COUNT_
+};
+
+struct Layout {
+  size_t off[B_COUNT_];
+  size_t bytes[B_COUNT_];
+  size_t total;
+  int BH, N, d, nchunk, max_items, part_slots;
+};
+
+// Header block at the start of the workspace.
+struct Header {
+  int32_t err;          // ERR_* of the first fault
+  int32_t err_info[3];
+  uint32_t work_next;   // attention work-list cursor
+  int32_t n_items;      // attention work items
+  int32_t pad[10];
+};
+
+bool make_layout(const spr_params* p, Layout* L);
+// Eigen-coordinate count rounded up to 8, 16, 32 or 64 (zero-padded columns).
+int padded_p(int p);
+
+// Pointers of one call, resolved from the workspace base.
+struct Ptrs {
+  Header* hdr;
+  spr_head_stats* stats;
+  float *MK, *eval, *evec, *W, *Z, *centk, *Craw, *Ct, *Amat, *rms, *un2, *centq, *beta,
+      *qbar, *logit, *entry, *pw, *osp, *odn, *fitU, *fitB, *fitBv, *gram, *axx, *rxbar,
+      *proj;
+  double* part;
+  int32_t *initk, *initq, *labk, *labq, *chunk, *cbase, *counts, *permk, *kvoff, *permq,
+      *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx;
+  int2* runs;
+  int4* items;
+  uint8_t *sel, *top;
+  bf16 *Kp, *Vp, *Qp, *bq16, *qprobe;
+};
+
+Ptrs resolve(const Layout& L, void* ws);
+
+// Strided input view of one tensor (elements).
+struct TensorView {
+  const bf16* base;
+  int64_t sb, sh, sn;
+  int H;
+  __host__ __device__ const bf16* row(int bh, int n) const {
+    int b = bh / H, h = bh - b * H;
+    return base + b * sb + h * sh + (int64_t)n * sn;
+  }
+};
+
+// ---- stage launchers (host) ----
+cudaError_t launch_partition(const spr_params& p, const Layout& L, const Ptrs& P,
+                             const TensorView& Q, const TensorView& K, const TensorView& V,
+                             cudaStream_t st);
+cudaError_t launch_route(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st);
+cudaError_t launch_attend(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st);
+cudaError_t launch_reconstruct(const spr_params& p, const Layout& L, const Ptrs& P,
+                               bf16* O, cudaStream_t st);
+// Symmetric eigensolver: `count` matrices n x n (fp32, row-major) -> eigenvalues
+// descending and eigenvectors as columns, same order.
+cudaError_t launch_eig(const float* A, int count, int n, float* evals, float* evecs,
+                       cudaStream_t st);
+int num_sms();
+
+// Every kernel launch of the library goes through spr_launch, which counts it
+// (sparsepr_launch_count reports the total).
+void note_launch();
+#ifdef __CUDACC__
+template <typename... KArgs, typename... Args>
+inline void spr_launch(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  k<<<grid, block, smem, st>>>(args...);
+  note_launch();
+}
+#endif
+
+}  // namespace spr
+
+// ------------------------------------------------------------------------
+// Device helpers
+// ------------------------------------------------------------------------
+#ifdef __CUDACC__
+namespace spr {
+
+__device__ __forceinline__ void set_error(Header* h, int code, int a = 0, int b = 0, int c = 0) {
+  if (atomicCAS(&h->err, 0, code) == 0) {
+    h->err_info[0] = a;
+    h->err_info[1] = b;
+    h->err_info[2] = c;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte asynchronous global->shared copy; src_bytes = 0 zero-fills.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
+               "l"(gmem), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                        const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                          const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D (fp32)
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// exp2 through the hardware approximation instruction.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Byte offset of 16-byte chunk `c` of row `r` in a row-major bf16 tile with
+// `CH` chunks per row, XOR-swizzled so that 8 consecutive rows at the same
+// logical chunk hit 8 distinct bank groups.
+template <int CH>
+__device__ __forceinline__ int swz(int r, int c) {
+  return (r * CH + (c ^ (r & 7))) * 16;
+}
+
+__device__ __forceinline__ float bf2f(bf16 v) { return __bfloat162float(v); }
+
+}  // namespace spr
+#endif

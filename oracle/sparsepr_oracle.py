@@ -32,9 +32,11 @@ Readings (the pages leave these steps open; the plainest reading is taken):
   R5 route logit: s * qbar_i . c_j + ln|K_j| (qbar_i = mean raw query of group
      i, c_j = uncentred mean raw key of group j); cells of a query group are
      ranked by softmax mass (ties to lower j); a cell's entry mass is the
-     cumulative mass ranked before it; tau mode keeps entry mass < tau; budget
-     mode keeps all cells with entry mass <= the largest value v such that the
-     kept cells' true cost sum |Q_i||K_j| plus the probe pairs M*N_k fits in
+     cumulative mass ranked before it and its tail mass the mass ranked at or
+     after it (1 - entry, summed from the small end so that peaked rows keep
+     their tails distinct); tau mode keeps entry mass < tau; budget mode keeps
+     all cells with tail mass >= the smallest value t such that the kept
+     cells' true cost sum |Q_i||K_j| plus the probe pairs M*N_k fits in
      rho_target*N_q*N_k (per head); each group's top cell is always kept.
   R6 probes: one per nonempty query group, the rest apportioned by largest
      remainder on the spare capacity |Q_g|-1 (ties to lower g); if M is below
@@ -61,7 +63,7 @@ __all__ = [
     "response_metric", "key_response_weights", "splitmix64_stream",
     "kmeans_init_indices", "kmeans", "kmeans_objective", "group_means",
     "kv_centroids", "query_response_coords", "group_major_permutation",
-    "route_logits", "route_entry_mass", "route_select", "route_to_csr",
+    "route_logits", "route_masses", "route_select", "route_to_csr",
     "select_probes", "hard_drop_attention", "fit_residual", "apply_correction",
     "rho_exec", "sparsepr_head", "sparsepr_call",
 ]
@@ -265,16 +267,22 @@ def route_logits(qbar, C, counts_k, scale):
     return L
 
 
-def route_entry_mass(L):
-    """Per query group: softmax mass of each cell and its entry mass.
+def route_masses(L):
+    """Per query group: softmax mass of each cell, its entry and tail mass.
 
-    Cells are ranked by mass, descending, ties to the lower K/V index; a
-    cell's entry mass is the total mass ranked before it.  Columns with -inf
-    logits (empty K/V groups) get mass 0 and entry mass +inf (never routed).
+    Cells are ranked by mass, descending, ties to the lower K/V index.  A
+    cell's entry mass e is the total mass ranked before it; its tail mass is
+    the total mass ranked at or after it (1 - e in exact arithmetic), summed
+    from the smallest cell upward so that tiny tails keep their relative
+    precision.  Columns with -inf logits (empty K/V groups) get mass 0, entry
+    mass +inf and tail 0, and are never routed.  Returns (pi, e, tail, top)
+    with top marking each row's first-ranked cell.
     """
     Gq, Gk = L.shape
     pi = np.zeros((Gq, Gk))
     e = np.full((Gq, Gk), np.inf)
+    tail = np.zeros((Gq, Gk))
+    top = np.zeros((Gq, Gk), bool)
     for i in range(Gq):
         fin = np.isfinite(L[i])
         if not fin.any():
@@ -284,40 +292,45 @@ def route_entry_mass(L):
         w = w / w.sum()
         js = np.nonzero(fin)[0]
         order = np.lexsort((js, -w))
-        before = np.concatenate([[0.0], np.cumsum(w[order])[:-1]])
+        ranked = w[order]
         pi[i, js] = w
-        e[i, js[order]] = before
-    return pi, e
+        e[i, js[order]] = np.concatenate([[0.0], np.cumsum(ranked)[:-1]])
+        tail[i, js[order]] = np.cumsum(ranked[::-1])[::-1]
+        top[i, js[order[0]]] = True
+    return pi, e, tail, top
 
 
-def route_select(e, counts_q, counts_k, mode, tau=0.9, rho_target=0.25, M=0):
+def route_select(tail, top, counts_q, counts_k, mode, tau=0.9, rho_target=0.25, M=0):
     """Boolean cell mask [Gq, Gk]; reading R5.  Empty query groups keep none.
 
-    Budget mode: the budget is rho_target*N_q*N_k - M*N_k pairs, compared in
-    fp64 against integer costs.
+    Tau mode keeps cells whose entry mass is below tau, i.e. whose tail mass
+    exceeds 1 - tau.  Budget mode keeps every live cell whose tail mass is at
+    least t*, the smallest tail value for which the kept cells' true cost fits
+    the budget rho_target*N_q*N_k - M*N_k (fp64 against integer costs).  Each
+    group's top cell is always kept.
     """
     live = (counts_q > 0)[:, None] & (counts_k > 0)[None, :]
-    top = live & (e == 0.0)
+    top = top & live
     if mode == "tau":
-        return (live & (e < tau)) | top
+        return (live & (tail > 1.0 - tau)) | top
     if mode != "budget":
         raise ValueError(mode)
     Nq, Nk = int(counts_q.sum()), int(counts_k.sum())
     budget = rho_target * Nq * Nk - M * Nk
     cost = counts_q[:, None].astype(np.float64) * counts_k[None, :]
-    # Kept cost as a function of the threshold v is the cumulative cost of
-    # live cells in ascending entry-mass order, read at the last cell with
-    # entry mass v; it is monotone, so the feasible values form a prefix.
-    ev, cv = e[live], cost[live]
-    order = np.argsort(ev, kind="stable")
-    ev, cv = ev[order], cv[order]
+    # Kept cost as a function of the threshold t is the cumulative cost of
+    # live cells in descending tail order, read at the last cell with tail t;
+    # it is monotone, so the feasible thresholds form a prefix.
+    tv, cv = tail[live], cost[live]
+    order = np.argsort(-tv, kind="stable")
+    tv, cv = tv[order], cv[order]
     cum = np.cumsum(cv)
-    last = np.r_[ev[1:] != ev[:-1], True] if len(ev) else np.zeros(0, bool)
+    last = np.r_[tv[1:] != tv[:-1], True] if len(tv) else np.zeros(0, bool)
     ok = np.nonzero(last & (cum <= budget))[0]
     if len(ok) == 0:
         return top
-    best = ev[ok.max()]
-    return (live & (e <= best)) | top
+    best = tv[ok.max()]
+    return (live & (tail >= best)) | top
 
 
 def route_to_csr(mask):
@@ -517,14 +530,14 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
                counts_q=counts_q, qbar=qbar)
     # Routing
     L = route_logits(np.nan_to_num(qbar), C, counts_k, s)
-    pi, e = route_entry_mass(L)
+    pi, e, tail, top = route_masses(L)
     if csr is None:
-        mask = route_select(e, counts_q, counts_k, prm.route_mode, prm.tau,
+        mask = route_select(tail, top, counts_q, counts_k, prm.route_mode, prm.tau,
                             prm.rho_target, prm.M)
         row_ptr, col_idx = route_to_csr(mask)
     else:
         row_ptr, col_idx = (np.asarray(a, np.int64) for a in csr)
-    out.update(route_logits=L, route_pi=pi, route_entry=e, row_ptr=row_ptr,
+    out.update(route_logits=L, route_pi=pi, route_entry=e, route_tail=tail, row_ptr=row_ptr,
                col_idx=col_idx)
     # Probes
     probe_pos, probe_idx, wts, m_g = select_probes(counts_q, q_off, perm_q, prm.M)

@@ -1,0 +1,175 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path through the C ABI
+on seeded synthetic inputs, read its intermediates out of the workspace, and
+recompute everything downstream of its cluster labels with the oracle
+(driven mode), then compare.
+
+Bars (from the method's contract): integer and indexing results bit-exact on
+the GPU's labels; k-means objectives within 1e-4 relative; the final output
+within 5e-3 per-head relative L2 (bf16 inputs, fp32 accumulation, bf16
+output).  Routing decisions that sit on a floating-point near-tie (a tail
+mass within 1e-4 relative of the cut, or two cells of one query group whose
+masses agree to 1e-5) may differ; such cells are counted and the GPU's routed
+cells are then handed to the oracle.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import free_block_sparse_means_b200 as spr
+from oracle import Params, sparsepr_head
+from synthetic import voronoi_qkv
+
+OUT_TOL = 5e-3
+OBJ_TOL = 1e-4
+TIE_E = 3e-4
+TIE_PI = 1e-5
+
+
+def oracle_params(wl, **kw) -> Params:
+    d = dict(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
+             tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index)
+    d.update(kw)
+    return Params(**d)
+
+
+def run_gpu(wl, N=None, heads=None, inputs=None):
+    """Run sparsepr_call on cuda:0; return a dict of CPU numpy results."""
+    Q, K, V = inputs if inputs is not None else voronoi_qkv(wl, heads=heads, N=N)
+    Qd, Kd, Vd = (t.cuda() for t in (Q, K, V))
+    Od = torch.empty_like(Qd)
+    prm = spr.make_params(Qd, Kd, Vd, Od, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
+                          seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
+                          rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam)
+    ws = spr.alloc_workspace(prm)
+    spr.sparsepr_call(prm, Qd, Kd, Vd, Od, ws)
+    stats, err = spr.sparsepr_get_stats(prm, ws)
+    assert err == 0
+    return collect(prm, ws, Q, K, V, Od, stats)
+
+
+def collect(prm, ws, Q, K, V, Od, stats):
+    B, H, N, d = prm.B, prm.H, prm.N, prm.d
+    BH, Gk, Gq, M = B * H, prm.Gk, prm.Gq, prm.M
+    pp = 8 if prm.p <= 8 else 16 if prm.p <= 16 else 32 if prm.p <= 32 else 64
+
+    def view(name, dtype, shape):
+        return spr.workspace_tensor(prm, ws, name, dtype, shape).cpu().numpy()
+
+    i32, f32 = torch.int32, torch.float32
+    out = dict(
+        prm=prm, stats=stats,
+        Q=Q.reshape(BH, N, d), K=K.reshape(BH, N, d), V=V.reshape(BH, N, d),
+        O=Od.float().cpu().reshape(BH, N, d).numpy().astype(np.float64),
+        lab_k=view("lab_k", i32, (BH, N)), lab_q=view("lab_q", i32, (BH, N)),
+        perm_k=view("perm_k", i32, (BH, N)), perm_q=view("perm_q", i32, (BH, N)),
+        kv_off=view("kv_off", i32, (BH, Gk + 1)), q_off=view("q_off", i32, (BH, Gq + 1)),
+        row_ptr=view("row_ptr", i32, (BH, Gq + 1)), col_idx=view("col_idx", i32, (BH, Gq * Gk)),
+        tail=view("tail", f32, (BH, Gq, Gk)),
+        w_key=view("w_key", f32, (BH, d, pp)), cent_k=view("cent_k", f32, (BH, Gk, pp)),
+        o_sparse=view("o_sparse", f32, (BH, N, d)),
+    )
+    if M > 0:
+        out.update(probe_pos=view("probe_pos", i32, (BH, M)), probe_idx=view("probe_idx", i32, (BH, M)),
+                   probe_w=view("probe_w", f32, (BH, M)), o_probe=view("o_probe", f32, (BH, M, d)))
+    return out
+
+
+def rel_l2(a, b):
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
+
+
+def gpu_csr(g, bh):
+    rp = g["row_ptr"][bh].astype(np.int64)
+    return rp, g["col_idx"][bh][: rp[-1]].astype(np.int64)
+
+
+def mask_from_csr(rp, ci, Gq, Gk):
+    m = np.zeros((Gq, Gk), bool)
+    for i in range(Gq):
+        m[i, ci[rp[i]:rp[i + 1]]] = True
+    return m
+
+
+def fragile_cells(orc, wl, gpu_thr, live):
+    """Cells whose routing decision sits on a floating-point near-tie: a tail
+    mass within TIE_E (relative) of either side's cut, or a mass that agrees
+    with another cell of its row to TIE_PI."""
+    tail, pi = orc["route_tail"], orc["route_pi"]
+    fr = np.zeros(tail.shape, bool)
+    if wl.route_mode == "tau":
+        fr |= live & (np.abs(tail - (1.0 - wl.tau)) < TIE_E)
+    else:
+        keep = orc["_mask"] & live
+        thr = tail[keep].min() if keep.any() else 1.0
+        for t in (thr, gpu_thr):
+            fr |= live & (np.abs(tail - t) <= TIE_E * max(t, 1e-30))
+    for i in range(tail.shape[0]):
+        row = pi[i]
+        srt = np.sort(row[row > 0])
+        close = np.nonzero(np.diff(srt) < TIE_PI * max(srt.max() if len(srt) else 1.0, 1e-30))[0]
+        for c in close:
+            for v in (srt[c], srt[c + 1]):
+                fr[i] |= np.isclose(row, v, rtol=0, atol=0)
+    return fr
+
+
+def check_head(g, wl, bh, rows=None, report=None):
+    """Driven-mode oracle for one head and every comparison of the contract."""
+    prm = oracle_params(wl)
+    q, k, v = (g[n][bh].double().numpy() for n in ("Q", "K", "V"))
+    lab_k, lab_q = g["lab_k"][bh].astype(np.int64), g["lab_q"][bh].astype(np.int64)
+    orc = sparsepr_head(q, k, v, prm, bh=bh, lab_k=lab_k, lab_q=lab_q, rows=rows)
+    # --- integer / indexing work: bit-exact on the GPU's labels
+    assert (g["perm_k"][bh] == orc["perm_k"]).all(), "perm_k"
+    assert (g["kv_off"][bh] == orc["kv_off"]).all(), "kv_off"
+    assert (g["perm_q"][bh] == orc["perm_q"]).all(), "perm_q"
+    assert (g["q_off"][bh] == orc["q_off"]).all(), "q_off"
+    rp, ci = gpu_csr(g, bh)
+    gm = mask_from_csr(rp, ci, wl.Gq, wl.Gk)
+    om = mask_from_csr(orc["row_ptr"], orc["col_idx"], wl.Gq, wl.Gk)
+    orc["_mask"] = om
+    live = (orc["counts_q"] > 0)[:, None] & (orc["counts_k"] > 0)[None, :]
+    # tail masses agree to fp32 accuracy on live cells; dead cells are marked -1
+    t_g, t_o = g["tail"][bh].astype(np.float64), orc["route_tail"]
+    assert ((t_g < 0) == ~live).all(), "tail liveness"
+    assert (np.abs(t_g - t_o)[live] <= 1e-3 * np.maximum(t_o[live], 1e-3)).all(), "tail mass"
+    near = 0
+    if not (gm == om).all():
+        fr = fragile_cells(orc, wl, g["stats"][bh]["route_threshold"], live)
+        diff = gm != om
+        assert not (diff & ~fr).any(), f"route differs off near-ties at {np.argwhere(diff & ~fr)[:5]}"
+        near = int(diff.sum())
+        orc = sparsepr_head(q, k, v, prm, bh=bh, lab_k=lab_k, lab_q=lab_q, csr=(rp, ci), rows=rows)
+    st = g["stats"][bh]
+    assert st["routed_pairs"] == orc["routed_pairs"], "routed pairs"
+    assert st["probe_pairs"] == orc["probe_pairs"], "probe pairs"
+    assert st["nnz_cells"] == len(orc["col_idx"]), "nnz"
+    assert st["rho_exec"] == orc["rho_exec"], "rho_exec"
+    if wl.M > 0:
+        assert (g["probe_pos"][bh] == orc["probe_pos"]).all(), "probe_pos"
+        assert (g["probe_idx"][bh] == orc["probe_idx"]).all(), "probe_idx"
+        np.testing.assert_allclose(g["probe_w"][bh], orc["probe_w"], rtol=1e-6)
+    # --- k-means objectives on the GPU's labels
+    ek = abs(st["obj_k"] - orc["obj_k"]) / max(orc["obj_k"], 1e-30)
+    eq = abs(st["obj_q"] - orc["obj_q"]) / max(orc["obj_q"], 1e-30)
+    # --- floating-point outputs
+    want = orc["rows"]
+    inv = np.empty_like(g["perm_q"][bh])
+    inv[g["perm_q"][bh]] = np.arange(len(inv))
+    osp_gpu = g["o_sparse"][bh][inv[want]].astype(np.float64)
+    e_sp = rel_l2(osp_gpu, orc["O_sp"])
+    e_out = rel_l2(g["O"][bh][want], orc["O"])
+    res = dict(bh=bh, near_ties=near, obj_k_rel=ek, obj_q_rel=eq, hard_drop_rel=e_sp, out_rel=e_out)
+    if wl.M > 0:
+        res["probe_rel"] = rel_l2(g["o_probe"][bh].astype(np.float64), orc["probe_dense"])
+    if report is not None:
+        report.append(res)
+    assert ek <= OBJ_TOL, f"key objective rel err {ek}"
+    assert eq <= OBJ_TOL, f"query objective rel err {eq}"
+    assert e_sp <= OUT_TOL, f"hard-drop output rel-L2 {e_sp}"
+    assert e_out <= OUT_TOL, f"output rel-L2 {e_out}"
+    if wl.M > 0:
+        assert res["probe_rel"] <= OUT_TOL, f"probe rows rel-L2 {res['probe_rel']}"
+    return res, orc

@@ -1,0 +1,110 @@
+"""GPU parity of the SparsePR call (CUDA path through the C ABI) against the
+fp64 oracle run on the GPU's own cluster labels.
+
+Sizes: the tiny workload (1 head, 1024 tokens, d=64, tau routing); the
+mid workload at full sequence length on two heads (budget routing, several
+tiles and chunks); ragged lengths that end mid-tile and mid-chunk for d=64
+and d=128; degenerate cases (one group, every cell routed, no probes, r=0,
+singleton-heavy groups).
+"""
+import numpy as np
+import pytest
+import torch
+
+import free_block_sparse_means_b200 as spr
+from gpu_support import check_head, oracle_params, rel_l2, run_gpu
+from oracle import dense_attention
+from synthetic import workload
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_full_parity():
+    wl = workload("tiny")
+    g = run_gpu(wl)
+    res, orc = check_head(g, wl, 0)
+    assert res["near_ties"] == 0
+
+
+def test_mid_two_heads_full_length():
+    wl = workload("mid", H=2)
+    g = run_gpu(wl)
+    for bh in range(2):
+        res, _ = check_head(g, wl, bh)
+        st = g["stats"][bh]
+        assert 0.2 < st["rho_exec"] <= 0.25 + 1e-9, st["rho_exec"]
+
+
+@pytest.mark.parametrize("d,grid,mode", [(128, (3, 17, 29), "tau"), (64, (2, 23, 31), "budget"),
+                                         (128, (1, 7, 19), "budget")])
+def test_ragged_lengths(d, grid, mode):
+    n = grid[0] * grid[1] * grid[2]
+    wl = workload("mid", H=2, d=d, grid=grid, centers=24, Gk=24, Gq=20, Ms=min(300, n), p=16,
+                  M=min(100, n // 2), r=8, route_mode=mode, tau=0.85, rho_target=0.3)
+    g = run_gpu(wl)
+    for bh in range(2):
+        check_head(g, wl, bh)
+
+
+def test_every_cell_routed_is_dense_attention():
+    wl = workload("tiny", tau=2.0, M=0)
+    g = run_gpu(wl)
+    q, k, v = (g[n][0].double().numpy() for n in ("Q", "K", "V"))
+    dense = dense_attention(q, k, v, 1 / np.sqrt(64))
+    assert rel_l2(g["O"][0], dense) < 5e-3
+    assert g["stats"][0]["rho_exec"] == 1.0
+
+
+def test_single_group_and_no_probes():
+    wl = workload("tiny", Gk=1, Gq=1, M=0)
+    g = run_gpu(wl)
+    res, _ = check_head(g, wl, 0)
+    assert g["stats"][0]["nnz_cells"] == 1
+    assert g["stats"][0]["gk_nonempty"] == 1
+
+
+def test_zero_rank_fit_and_many_small_groups():
+    wl = workload("tiny", grid=(1, 10, 20), Gk=150, Gq=160, Ms=200, M=170, r=0, tau=0.6)
+    g = run_gpu(wl)
+    check_head(g, wl, 0)
+    assert g["stats"][0]["r_eff"] == 0
+
+
+def test_stage_entry_points_match_fused_call():
+    wl = workload("mid", H=1, grid=(2, 32, 32))
+    from synthetic import voronoi_qkv
+    Q, K, V = (t.cuda() for t in voronoi_qkv(wl))
+    O1, O2 = torch.empty_like(Q), torch.empty_like(Q)
+    prm = spr.make_params(Q, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, seed=wl.index,
+                          route_mode=wl.route_mode, rho_target=wl.rho_target, M=wl.M, r=wl.r,
+                          lam=wl.lam)
+    ws = spr.alloc_workspace(prm)
+    spr.sparsepr_call(prm, Q, K, V, O1, ws)
+    spr.sparsepr_partition(prm, Q, K, V, ws)
+    spr.sparsepr_route(prm, ws)
+    spr.sparsepr_attend(prm, ws)
+    spr.sparsepr_attend(prm, ws)  # re-running a stage is allowed
+    spr.sparsepr_reconstruct(prm, ws, O2)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2)  # deterministic
+    stats, err = spr.sparsepr_get_stats(prm, ws)
+    assert err == 0 and stats[0]["tile_pairs"] >= stats[0]["routed_pairs"]
+
+
+def test_strided_inputs_and_output():
+    """[B, N, H, d] layout (token-major), as DiT blocks hold it."""
+    wl = workload("mid", B=2, H=2, grid=(2, 16, 32), centers=32, Gk=32, Gq=32, Ms=256, M=64, r=8)
+    from synthetic import voronoi_qkv
+    Q, K, V = voronoi_qkv(wl)
+    g_ref = run_gpu(wl, inputs=(Q, K, V))
+    Qt, Kt, Vt = (t.transpose(1, 2).contiguous().transpose(1, 2).cuda() for t in (Q, K, V))
+    Ot = torch.empty(Q.shape[0], Q.shape[2], Q.shape[1], Q.shape[3], dtype=torch.bfloat16,
+                     device="cuda").transpose(1, 2)
+    prm = spr.make_params(Qt, Kt, Vt, Ot, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, seed=wl.index,
+                          route_mode=wl.route_mode, rho_target=wl.rho_target, M=wl.M, r=wl.r,
+                          lam=wl.lam)
+    ws = spr.alloc_workspace(prm)
+    spr.sparsepr_call(prm, Qt, Kt, Vt, Ot, ws)
+    torch.cuda.synchronize()
+    got = Ot.float().cpu().reshape(-1, wl.N, wl.d).numpy()
+    assert np.array_equal(got, g_ref["O"].astype(np.float32))

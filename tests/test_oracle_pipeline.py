@@ -12,7 +12,7 @@ exact attention mass the group's mean query puts on that group.
 import numpy as np
 import pytest
 
-from oracle import Params, dense_attention, route_entry_mass, route_logits, sparsepr_head
+from oracle import Params, dense_attention, route_logits, route_masses, sparsepr_head
 from synthetic import voronoi_qkv, workload
 
 
@@ -97,7 +97,7 @@ def test_route_logit_is_exact_mass_for_collapsed_groups():
     lab = np.repeat(np.arange(Gk), sizes)
     qbar = rng.normal(size=(2, d))
     s = 0.8
-    pi, _ = route_entry_mass(route_logits(qbar, cent, sizes, s))
+    pi, _, _, _ = route_masses(route_logits(qbar, cent, sizes, s))
     for i in range(2):
         w = np.exp(s * keys @ qbar[i])
         for j in range(Gk):

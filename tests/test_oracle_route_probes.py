@@ -12,7 +12,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
-from oracle import (Params, dense_attention, rho_exec, route_entry_mass, route_logits,
+from oracle import (Params, dense_attention, rho_exec, route_logits, route_masses,
                     route_select, route_to_csr, select_probes, sparsepr_head)
 
 
@@ -21,7 +21,7 @@ def test_entry_mass_explicit_sort():
     L = rng.normal(size=(4, 6))
     L[1, 2] = -np.inf
     L[3, :] = 0.0  # all equal: ties go to the lower index
-    pi, e = route_entry_mass(L)
+    pi, e, tail, top = route_masses(L)
     for i in range(4):
         fin = [j for j in range(6) if np.isfinite(L[i, j])]
         w = {j: np.exp(L[i, j]) for j in fin}
@@ -31,8 +31,10 @@ def test_entry_mass_explicit_sort():
         for j in order:
             assert abs(e[i, j] - acc) < 1e-14
             assert abs(pi[i, j] - w[j] / z) < 1e-14
+            assert abs(tail[i, j] - sum(w[t] / z for t in order[order.index(j):])) < 1e-14
+            assert top[i, j] == (j == order[0])
             acc += w[j] / z
-    assert e[1, 2] == np.inf
+    assert e[1, 2] == np.inf and tail[1, 2] == 0.0
     np.testing.assert_allclose(e[3], np.arange(6) / 6, atol=1e-15)
 
 
@@ -41,11 +43,20 @@ def test_tau_limits():
     L = rng.normal(size=(5, 7)) * 3
     cq = np.array([3, 0, 2, 5, 1])
     ck = np.array([2, 2, 0, 4, 1, 3, 1])
-    _, e = route_entry_mass(route_logits(rng.normal(size=(5, 3)), rng.normal(size=(7, 3)), ck, 1.0))
-    allm = route_select(e, cq, ck, "tau", tau=1.5)
+    _, e, tail, top = route_masses(route_logits(rng.normal(size=(5, 3)), rng.normal(size=(7, 3)), ck, 1.0))
+    allm = route_select(tail, top, cq, ck, "tau", tau=1.5)
     assert (allm == ((cq > 0)[:, None] & (ck > 0)[None, :])).all()
-    top = route_select(e, cq, ck, "tau", tau=1e-12)
-    assert top.sum(1).tolist() == [1, 0, 1, 1, 1]
+    topm = route_select(tail, top, cq, ck, "tau", tau=1e-12)
+    assert topm.sum(1).tolist() == [1, 0, 1, 1, 1]
+
+
+def test_tail_keeps_peaked_rows_ordered():
+    """Entry masses of a very peaked row all round to 1.0; tails stay distinct."""
+    L = np.array([[0.0, -40.0, -45.0, -50.0, -60.0]])
+    pi, e, tail, top = route_masses(L)
+    assert (e[0, 1:] == 1.0).all()
+    assert tail[0, 1] > tail[0, 2] > tail[0, 3] > tail[0, 4] > 0
+    np.testing.assert_allclose(tail[0, 4], np.exp(-60.0) / np.exp(L[0]).sum(), rtol=1e-12)
 
 
 def test_budget_brute_force():
@@ -57,17 +68,17 @@ def test_budget_brute_force():
         if cq.sum() == 0 or ck.sum() == 0:
             continue
         L = route_logits(rng.normal(size=(Gq, 3)), rng.normal(size=(Gk, 3)) * 2, ck, 1.0)
-        _, e = route_entry_mass(L)
+        _, e, tail, top = route_masses(L)
         rho, M = float(rng.uniform(0.05, 0.9)), int(rng.integers(0, 3))
-        got = route_select(e, cq, ck, "budget", rho_target=rho, M=M)
+        got = route_select(tail, top, cq, ck, "budget", rho_target=rho, M=M)
         live = (cq > 0)[:, None] & (ck > 0)[None, :]
         budget = rho * cq.sum() * ck.sum() - M * ck.sum()
         best = None
-        for v in sorted(set(e[live].tolist())):
-            keep = live & (e <= v)
+        for v in sorted(set(tail[live].tolist()), reverse=True):
+            keep = live & (tail >= v)
             if (cq[:, None] * ck[None, :])[keep].sum() <= budget:
                 best = keep
-        want = live & (e == 0.0) if best is None else best | (live & (e == 0.0))
+        want = live & top if best is None else best | (live & top)
         assert (got == want).all()
 
 
@@ -75,10 +86,11 @@ def test_budget_exact_equality_is_feasible():
     """A threshold whose kept cost equals the budget exactly is taken."""
     cq = np.array([2, 2])
     ck = np.array([2, 2])
-    e = np.array([[0.0, 0.3], [0.6, 0.0]])
-    got = route_select(e, cq, ck, "budget", rho_target=0.75, M=0)  # budget 12 = 3 cells
+    tail = np.array([[1.0, 0.7], [0.4, 1.0]])
+    top = np.array([[True, False], [False, True]])
+    got = route_select(tail, top, cq, ck, "budget", rho_target=0.75, M=0)  # budget 12 = 3 cells
     assert got.tolist() == [[True, True], [False, True]]
-    got = route_select(e, cq, ck, "budget", rho_target=0.75, M=1)  # budget 8: top cells only
+    got = route_select(tail, top, cq, ck, "budget", rho_target=0.75, M=1)  # budget 8: top cells only
     assert got.tolist() == [[True, False], [False, True]]
 
 
