@@ -24,6 +24,7 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_HDR] = sizeof(Header);
   sz[B_STATS] = BH * sizeof(spr_head_stats);
   sz[B_MK] = BH * d * d * 4;
+  sz[B_TRACE] = BH * 4;
   sz[B_EVAL] = BH * d * 4;
   sz[B_EVEC] = BH * d * d * 4;
   sz[B_W] = BH * d * P * 4;
@@ -63,6 +64,7 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_PPOS] = BH * (M ? M : 1) * 4;
   sz[B_PIDX] = BH * (M ? M : 1) * 4;
   sz[B_PW] = BH * (M ? M : 1) * 4;
+  sz[B_PSLOT] = BH * N * 4;
   sz[B_QPROBE] = BH * (M ? M : 1) * d * 2;
   sz[B_ITEMS] = max_items * 16;
   sz[B_OSP] = BH * N * d * 4;
@@ -73,7 +75,7 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_GRAM] = BH * d * d * 4;
   sz[B_AXX] = BH * d * d * 4;
   sz[B_RXBAR] = BH * 2 * d * 4;
-  sz[B_PROJ] = BH * (M ? M : 1) * d * 4;
+  sz[B_PROJ] = BH * (M ? (M + 63) / 64 : 1) * d * (p->r > 0 ? p->r : 1) * 4;  // fit rhs partials
   sz[B_PART] = part_slots * 8;
   size_t off = 0;
   for (int i = 0; i < B_COUNT_; ++i) {
@@ -98,6 +100,7 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.hdr = AT(Header*, B_HDR);
   P.stats = AT(spr_head_stats*, B_STATS);
   P.MK = AT(float*, B_MK);
+  P.trace = AT(float*, B_TRACE);
   P.eval = AT(float*, B_EVAL);
   P.evec = AT(float*, B_EVEC);
   P.W = AT(float*, B_W);
@@ -137,6 +140,7 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.ppos = AT(int32_t*, B_PPOS);
   P.pidx = AT(int32_t*, B_PIDX);
   P.pw = AT(float*, B_PW);
+  P.pslot = AT(int32_t*, B_PSLOT);
   P.qprobe = AT(bf16*, B_QPROBE);
   P.items = AT(int4*, B_ITEMS);
   P.osp = AT(float*, B_OSP);

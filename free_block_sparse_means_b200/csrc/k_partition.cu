@@ -52,16 +52,11 @@ __global__ void __launch_bounds__(256) k_metric(TensorView Q, int N, int Ms, flo
 
 
 // W[:, k] = u_k sqrt(lambda_k / sum_j lambda_j) for k < p; zero for p <= k < pp.
-__global__ void k_keyweights(const float* evals, const float* evecs, int D, int p, int pp,
-                             float* W) {
+// The eigenvalue sum of the positive semidefinite M_K is its trace.
+__global__ void k_keyweights(const float* evals, const float* evecs, const float* trace, int D,
+                             int p, int pp, float* W) {
   const int bh = blockIdx.x;
-  __shared__ float tot;
-  if (threadIdx.x == 0) {
-    float t = 0.f;
-    for (int i = 0; i < D; ++i) t += fmaxf(evals[(size_t)bh * D + i], 0.f);
-    tot = t;
-  }
-  __syncthreads();
+  const float tot = trace[bh];
   for (int e = threadIdx.x; e < D * pp; e += blockDim.x) {
     const int i = e / pp, k = e % pp;
     float w = 0.f;
@@ -330,54 +325,78 @@ struct SegArgs {
 };
 
 template <int MODE, int DD>
-__global__ void __launch_bounds__(128) k_segsum(SegArgs a) {
+__device__ __forceinline__ void seg_row(const SegArgs& a, int bh, int i, int lane, float* v) {
+  constexpr int NV = (MODE == SEG_Z) ? (DD + 31) / 32 : DD / 32;
+  if (MODE == SEG_Z) {
+    const int row = a.perm[(size_t)bh * a.N + i];
+    const float* src = a.Z + ((size_t)bh * a.N + row) * DD;
+#pragma unroll
+    for (int q = 0; q < NV; ++q) v[q] = (lane + 32 * q < DD) ? src[lane + 32 * q] : 0.f;
+  } else {
+    const bf16* src;
+    float sc = 1.f;
+    if (MODE == SEG_QSCALED) {
+      const int row = a.perm[(size_t)bh * a.N + i];
+      src = a.Q.row(bh, row);
+      sc = a.scale / a.rms[(size_t)bh * a.N + row];
+    } else {
+      src = a.Xp + ((size_t)bh * a.N + i) * DD;
+    }
+#pragma unroll
+    for (int q = 0; q < NV / 2; ++q) {
+      const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(src)[lane + 32 * q];
+      v[2 * q] = sc * __low2float(x);
+      v[2 * q + 1] = sc * __high2float(x);
+    }
+  }
+}
+
+// 8 warps; warp w sums rows start + w + 8 t in ascending t, with four rows'
+// loads in flight, then the warps' partial sums are added in warp order.
+template <int MODE, int DD>
+__global__ void __launch_bounds__(256) k_segsum(SegArgs a) {
   constexpr int NV = (MODE == SEG_Z) ? (DD + 31) / 32 : DD / 32;  // values per lane
-  __shared__ double red[4][DD];
+  constexpr int NW = 8, UN = 4;
+  __shared__ double red[NW][DD];
   const int bh = blockIdx.y, g = blockIdx.x, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int start = a.off[(size_t)bh * (a.G + 1) + g], end = a.off[(size_t)bh * (a.G + 1) + g + 1];
   double acc[NV];
 #pragma unroll
-  for (int v = 0; v < NV; ++v) acc[v] = 0.0;
-  for (int i = start + w; i < end; i += 4) {
-    if (MODE == SEG_Z) {
-      const int row = a.perm[(size_t)bh * a.N + i];
-      const float* src = a.Z + ((size_t)bh * a.N + row) * DD;
+  for (int q = 0; q < NV; ++q) acc[q] = 0.0;
+  for (int i0 = start + w; i0 < end; i0 += NW * UN) {
+    float v[UN][NV];
 #pragma unroll
-      for (int v = 0; v < NV; ++v)
-        if (lane + 32 * v < DD) acc[v] += (double)src[lane + 32 * v];
-    } else {
-      const bf16* src;
-      float sc = 1.f;
-      if (MODE == SEG_QSCALED) {
-        const int row = a.perm[(size_t)bh * a.N + i];
-        src = a.Q.row(bh, row);
-        sc = a.scale / a.rms[(size_t)bh * a.N + row];
+    for (int u = 0; u < UN; ++u) {
+      const int i = i0 + u * NW;
+      if (i < end) {
+        seg_row<MODE, DD>(a, bh, i, lane, v[u]);
       } else {
-        src = a.Xp + ((size_t)bh * a.N + i) * DD;
-      }
 #pragma unroll
-      for (int v = 0; v < NV / 2; ++v) {
-        const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(src)[lane + 32 * v];
-        acc[2 * v] += (double)(sc * __low2float(x));
-        acc[2 * v + 1] += (double)(sc * __high2float(x));
+        for (int q = 0; q < NV; ++q) v[u][q] = 0.f;
       }
     }
+#pragma unroll
+    for (int u = 0; u < UN; ++u)
+#pragma unroll
+      for (int q = 0; q < NV; ++q) acc[q] += (double)v[u][q];
   }
   if (MODE == SEG_Z) {
 #pragma unroll
-    for (int v = 0; v < NV; ++v)
-      if (lane + 32 * v < DD) red[w][lane + 32 * v] = acc[v];
+    for (int q = 0; q < NV; ++q)
+      if (lane + 32 * q < DD) red[w][lane + 32 * q] = acc[q];
   } else {
 #pragma unroll
-    for (int v = 0; v < NV / 2; ++v) {
-      red[w][2 * (lane + 32 * v)] = acc[2 * v];
-      red[w][2 * (lane + 32 * v) + 1] = acc[2 * v + 1];
+    for (int q = 0; q < NV / 2; ++q) {
+      red[w][2 * (lane + 32 * q)] = acc[2 * q];
+      red[w][2 * (lane + 32 * q) + 1] = acc[2 * q + 1];
     }
   }
   __syncthreads();
   const int cnt = end - start;
-  for (int k = threadIdx.x; k < DD; k += 128) {
-    const double s = red[0][k] + red[1][k] + red[2][k] + red[3][k];
+  for (int k = threadIdx.x; k < DD; k += NW * 32) {
+    double s = 0.0;
+#pragma unroll
+    for (int q = 0; q < NW; ++q) s += red[q][k];
     float* o = a.out + ((size_t)bh * a.G + g) * DD + k;
     if (cnt > 0)
       *o = (float)(s / cnt);
@@ -741,8 +760,8 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   cudaError_t e;
   // Key-response coordinates
   spr_launch(k_metric<D>, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, Q, N, p.Ms, P.MK);
-  if ((e = launch_eig(P.MK, BH, D, P.eval, P.evec, st)) != cudaSuccess) return e;
-  spr_launch(k_keyweights, BH, 256, 0, st, P.eval, P.evec, D, p.p, pp, P.W);
+  if ((e = launch_eig(P.MK, BH, D, p.p, P.eval, P.evec, P.trace, st)) != cudaSuccess) return e;
+  spr_launch(k_keyweights, BH, 256, 0, st, P.eval, P.evec, P.trace, D, p.p, pp, P.W);
   const int pgrid = min((N + 255) / 256, max(1, 4 * sms / BH + 1));
 #define PROJ(PPV) spr_launch(k_project<D, PPV>, dim3(pgrid, BH), 256, 0, st, K, N, P.W, P.Z)
   if (pp == 8) PROJ(8); else if (pp == 16) PROJ(16); else if (pp == 32) PROJ(32); else PROJ(64);
@@ -772,7 +791,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
     sa.G = p.Gk;
     sa.out = P.centk;
     sa.keep_empty = 1;
-#define SEGZ(PPV) spr_launch(k_segsum<SEG_Z, PPV>, dim3(p.Gk, BH), 128, 0, st, sa)
+#define SEGZ(PPV) spr_launch(k_segsum<SEG_Z, PPV>, dim3(p.Gk, BH), 256, 0, st, sa)
     if (pp == 8) SEGZ(8); else if (pp == 16) SEGZ(16); else if (pp == 32) SEGZ(32); else SEGZ(64);
 #undef SEGZ
   }
@@ -792,7 +811,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
     sa.G = p.Gk;
     sa.out = P.Craw;
     sa.keep_empty = 0;
-    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gk, BH), 128, 0, st, sa);
+    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gk, BH), 256, 0, st, sa);
   }
   // P.counts holds |K_j| now; keep a copy of key counts in kv_off differences.
   spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
@@ -843,7 +862,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
     sa.G = p.Gq;
     sa.out = P.centq;
     sa.keep_empty = 1;
-    spr_launch(k_segsum<SEG_QSCALED, D>, dim3(p.Gq, BH), 128, 0, st, sa);
+    spr_launch(k_segsum<SEG_QSCALED, D>, dim3(p.Gq, BH), 256, 0, st, sa);
   }
   // objective terms n_g a_g^T A a_g with the final centroids (into part's tail)
   spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
@@ -858,7 +877,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
     sa.G = p.Gq;
     sa.out = P.qbar;
     sa.keep_empty = 0;
-    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gq, BH), 128, 0, st, sa);
+    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gq, BH), 256, 0, st, sa);
   }
   return cudaGetLastError();
 }

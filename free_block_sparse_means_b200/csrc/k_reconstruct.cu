@@ -78,32 +78,90 @@ __global__ void __launch_bounds__(1024) k_fit_moments(const float* osp, const fl
   }
 }
 
-// Subspace, ridge solve and the full-width map.  Grid BH, 512 threads.
+// Residual directions kept by the fit: the leading r eigenvalues of the Gram
+// above 1e-6 of the largest (sigma above 1e-3 sigma_max, the fp32 noise floor).
+__device__ __forceinline__ int fit_rank(const float* ev, int D, int r) {
+  const float l0 = fmaxf(ev[0], 0.f);
+  int k = 0;
+  if (l0 > 0.f)
+    while (k < r && k < D && fmaxf(ev[k], 0.f) > 1e-6f * l0) ++k;
+  return k;
+}
+
+constexpr int FIT_TM = 64;  // probes per right-hand-side block
+
+// Partial right-hand sides of the ridge system for one block of FIT_TM probes:
+// part[i][k] = sum_t w_t (x_t - xbar)_i ((r_t - Rbar) . u_k), k < r_eff, stride R.
+// Grid (BH, ceil(M / FIT_TM)), 256 threads.  Dynamic smem: Rs, Xs (TM x D),
+// Us (D x R), Ps (TM x R).
+template <int D>
+__global__ void __launch_bounds__(256) k_fit_rhs(const float* osp, const float* odn,
+                                                 const int32_t* ppos, const float* pw, int N,
+                                                 int M, int r, int R, const float* evals,
+                                                 const float* evecs, const float* rxbar,
+                                                 float* part) {
+  extern __shared__ __align__(16) float rsm[];
+  float* Rs = rsm;
+  float* Xs = Rs + FIT_TM * D;
+  float* Us = Xs + FIT_TM * D;
+  float* Ps = Us + D * R;
+  __shared__ float ws[FIT_TM];
+  const int bh = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, t0 = c * FIT_TM;
+  const int re = fit_rank(evals + (size_t)bh * D, D, r);
+  const float* rbar = rxbar + (size_t)bh * 2 * D;
+  const float* xbar = rbar + D;
+  for (int e = tid; e < FIT_TM * D; e += 256) {
+    const int tt = e / D, col = e % D, t = t0 + tt;
+    float rv = 0.f, xv = 0.f;
+    if (t < M) {
+      const float x = osp[((size_t)bh * N + ppos[(size_t)bh * M + t]) * D + col];
+      rv = odn[((size_t)bh * M + t) * D + col] - x - rbar[col];
+      xv = x - xbar[col];
+    }
+    Rs[e] = rv;
+    Xs[e] = xv;
+  }
+  for (int e = tid; e < D * R; e += 256) {
+    const int i = e / R, k = e % R;
+    Us[e] = k < re ? evecs[((size_t)bh * D + i) * D + k] : 0.f;
+  }
+  for (int e = tid; e < FIT_TM; e += 256) ws[e] = (t0 + e < M) ? pw[(size_t)bh * M + t0 + e] : 0.f;
+  __syncthreads();
+  for (int e = tid; e < FIT_TM * R; e += 256) {
+    const int tt = e / R, k = e % R;
+    float s = 0.f;
+    if (k < re)
+      for (int col = 0; col < D; ++col) s += Rs[tt * D + col] * Us[col * R + k];
+    Ps[e] = ws[tt] * s;
+  }
+  __syncthreads();
+  float* out = part + ((size_t)bh * gridDim.y + c) * D * R;
+  for (int e = tid; e < D * R; e += 256) {
+    const int i = e / R, k = e % R;
+    float s = 0.f;
+    if (k < re)
+      for (int tt = 0; tt < FIT_TM; ++tt) s += Xs[tt * D + i] * Ps[tt * R + k];
+    out[e] = s;
+  }
+}
+
+// Subspace, ridge solve and the intercept.  Grid BH, 512 threads.
 // Dynamic smem: A (D x (D+1)) Cholesky factor, Bm (D x D) right-hand sides.
 template <int D>
-__global__ void __launch_bounds__(512) k_fit_solve(const float* osp, const float* odn,
-                                                   const int32_t* ppos, const float* pw, int N,
-                                                   int M, int r, const float* evals,
+__global__ void __launch_bounds__(512) k_fit_solve(int r, int R, int nchunk, const float* evals,
                                                    const float* evecs, const float* axx,
-                                                   const float* rxbar, float* proj, float* fitU,
-                                                   float* fitB, float* fitBv,
+                                                   const float* rxbar, const float* part,
+                                                   float* fitU, float* fitB, float* fitBv,
                                                    spr_head_stats* stats, Header* hdr) {
   extern __shared__ __align__(16) float fsm[];
   constexpr int LD = D + 1;
   float* A = fsm;             // D x LD
   float* Bm = A + D * LD;     // D x D  (rhs, then B)
-  __shared__ int reff_s;
   __shared__ float rbar[D], xbar[D];
   const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
   const float* U = evecs + (size_t)bh * D * D;
-  if (tid == 0) {
-    const float l0 = fmaxf(evals[(size_t)bh * D], 0.f);
-    int k = 0;
-    if (l0 > 0.f)
-      while (k < r && k < D && fmaxf(evals[(size_t)bh * D + k], 0.f) > 1e-6f * l0) ++k;
-    reff_s = k;
-    stats[bh].r_eff = k;
-  }
+  const int re = fit_rank(evals + (size_t)bh * D, D, r);
+  if (tid == 0) stats[bh].r_eff = re;
   for (int c = tid; c < D; c += nt) {
     rbar[c] = rxbar[(size_t)bh * 2 * D + c];
     xbar[c] = rxbar[(size_t)bh * 2 * D + D + c];
@@ -112,75 +170,82 @@ __global__ void __launch_bounds__(512) k_fit_solve(const float* osp, const float
     A[(e / D) * LD + (e % D)] = axx[(size_t)bh * D * D + e];
     fitU[(size_t)bh * D * D + e] = U[e];
   }
-  __syncthreads();
-  const int re = reff_s;
-  // proj[t][k] = (R_t - Rbar) . U_k
-  for (int e = tid; e < M * re; e += nt) {
-    const int t = e / re, k = e % re;
-    const float* xr = osp + ((size_t)bh * N + ppos[(size_t)bh * M + t]) * D;
-    const float* dr = odn + ((size_t)bh * M + t) * D;
-    float s = 0.f;
-    for (int c = 0; c < D; ++c) s += (dr[c] - xr[c] - rbar[c]) * U[c * D + k];
-    proj[((size_t)bh * M + t) * D + k] = s;
-  }
-  __syncthreads();
-  // rhs[i][k] = sum_t w_t (X_t - xbar)_i proj[t][k]
-  for (int e = tid; e < D * re; e += nt) {
+  for (int e = tid; e < D * re; e += nt) {  // sum the probe blocks in a fixed order
     const int i = e / re, k = e % re;
     float s = 0.f;
-    for (int t = 0; t < M; ++t) {
-      const float x = osp[((size_t)bh * N + ppos[(size_t)bh * M + t]) * D + i] - xbar[i];
-      s += pw[(size_t)bh * M + t] * x * proj[((size_t)bh * M + t) * D + k];
-    }
+    for (int c = 0; c < nchunk; ++c) s += part[(((size_t)bh * nchunk + c) * D + i) * R + k];
     Bm[i * D + k] = s;
   }
   __syncthreads();
-  // Cholesky A = L L^T (lower triangle in place), right-looking.
+  // Cholesky A = L L^T, right-looking, one barrier per column: step k updates
+  // the trailing block from the unscaled column k and scales column k - 1.
+  const int warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
   for (int k = 0; k < D; ++k) {
-    if (tid == 0) {
-      float v = A[k * LD + k];
-      if (!(v > 0.f)) {
-        if (!isfinite(v)) set_error(hdr, ERR_NUMERIC, 10, bh, k);
-        v = FLT_MIN * 1e10f;
-      }
-      A[k * LD + k] = sqrtf(v);
+    float akk = A[k * LD + k];
+    if (!(akk > 0.f)) {
+      if (tid == 0 && !isfinite(akk)) set_error(hdr, ERR_NUMERIC, 10, bh, k);
+      akk = FLT_MIN * 1e10f;
+    }
+    const float inv = 1.f / akk;
+    for (int i = k + 1 + warp; i < D; i += nw) {
+      const float aik = A[i * LD + k] * inv;
+      for (int j = k + 1 + lane; j <= i; j += 32) A[i * LD + j] -= aik * A[j * LD + k];
+    }
+    if (k > 0) {
+      float ap = A[(k - 1) * LD + k - 1];
+      if (!(ap > 0.f)) ap = FLT_MIN * 1e10f;
+      const float dp = sqrtf(ap);
+      for (int i = k + tid; i < D; i += nt) A[i * LD + k - 1] /= dp;
     }
     __syncthreads();
-    const float dkk = A[k * LD + k];
-    for (int i = k + 1 + tid; i < D; i += nt) A[i * LD + k] /= dkk;
-    __syncthreads();
-    const int m = D - k - 1;
-    for (int e = tid; e < m * m; e += nt) {
-      const int i = k + 1 + e / m, j = k + 1 + e % m;
-      if (j <= i) A[i * LD + j] -= A[i * LD + k] * A[j * LD + k];
-    }
-    __syncthreads();
-  }
-  // Solve L L^T B = rhs, one column per thread.
-  for (int k = tid; k < re; k += nt) {
-    for (int i = 0; i < D; ++i) {
-      float s = Bm[i * D + k];
-      for (int j = 0; j < i; ++j) s -= A[i * LD + j] * Bm[j * D + k];
-      Bm[i * D + k] = s / A[i * LD + i];
-    }
-    for (int i = D - 1; i >= 0; --i) {
-      float s = Bm[i * D + k];
-      for (int j = i + 1; j < D; ++j) s -= A[j * LD + i] * Bm[j * D + k];
-      Bm[i * D + k] = s / A[i * LD + i];
+    if (k > 0 && tid == 0) {
+      float ap = A[(k - 1) * LD + k - 1];
+      A[(k - 1) * LD + k - 1] = sqrtf(ap > 0.f ? ap : FLT_MIN * 1e10f);
     }
   }
   __syncthreads();
-  // Full map F = B U_r^T (d x d) and intercept b = Rbar - xbar F.
+  {
+    float ap = A[(D - 1) * LD + D - 1];
+    if (tid == 0) A[(D - 1) * LD + D - 1] = sqrtf(ap > 0.f ? ap : FLT_MIN * 1e10f);
+  }
+  __syncthreads();
+  // Solve L L^T B = rhs: one warp per column, lanes split each inner product.
+  {
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int k = warp; k < re; k += nt / 32) {
+      for (int i = 0; i < D; ++i) {
+        float s = 0.f;
+        for (int j = lane; j < i; j += 32) s += A[i * LD + j] * Bm[j * D + k];
+        s = warp_sum(s);
+        if (lane == 0) Bm[i * D + k] = (Bm[i * D + k] - s) / A[i * LD + i];
+        __syncwarp();
+      }
+      for (int i = D - 1; i >= 0; --i) {
+        float s = 0.f;
+        for (int j = i + 1 + lane; j < D; j += 32) s += A[j * LD + i] * Bm[j * D + k];
+        s = warp_sum(s);
+        if (lane == 0) Bm[i * D + k] = (Bm[i * D + k] - s) / A[i * LD + i];
+        __syncwarp();
+      }
+    }
+  }
+  __syncthreads();
+  // B (d x r_eff, stride d) and the full-width intercept b = Rbar - (xbar B) U_r^T.
+  __shared__ float xb[D];
   for (int e = tid; e < D * D; e += nt) {
-    const int i = e / D, j = e % D;
+    const int i = e / D, k = e % D;
+    fitB[(size_t)bh * D * D + e] = k < re ? Bm[i * D + k] : 0.f;
+  }
+  for (int k = tid; k < D; k += nt) {
     float s = 0.f;
-    for (int k = 0; k < re; ++k) s += Bm[i * D + k] * U[j * D + k];
-    fitB[(size_t)bh * D * D + e] = s;
+    if (k < re)
+      for (int i = 0; i < D; ++i) s += xbar[i] * Bm[i * D + k];
+    xb[k] = s;
   }
   __syncthreads();
   for (int j = tid; j < D; j += nt) {
     float s = 0.f;
-    for (int i = 0; i < D; ++i) s += xbar[i] * fitB[(size_t)bh * D * D + i * D + j];
+    for (int k = 0; k < re; ++k) s += xb[k] * U[j * D + k];
     fitBv[(size_t)bh * D + j] = rbar[j] - s;
   }
 }
@@ -194,27 +259,35 @@ __global__ void k_fit_zero(float* fitB, float* fitBv, int D, int BH) {
   }
 }
 
-// O[orig row] = x + b + x F (unprobed) or the dense probe row; bf16 output in
-// the original query order.  Grid (blocks per head, BH), 256 threads, one warp
-// per permuted row.  Dynamic smem: F (D x D fp32).
+// O[orig row] = x + b + (x B) U_r^T (unprobed) or the dense probe row; bf16
+// output in the original query order.  Grid (blocks per head, BH), 256
+// threads, one warp per permuted row.  Dynamic smem: B as [D][R] and U_r as
+// [R][D] (R = the rank bound of the call).
 template <int D>
 __global__ void __launch_bounds__(256) k_apply(const float* osp, const float* odn,
-                                               const int32_t* ppos, const int32_t* permq,
-                                               const float* fitB, const float* fitBv, int N, int M,
-                                               int B_, int H, int64_t sb, int64_t sh, int64_t sn,
-                                               bf16* O, int do_fit, Header* hdr) {
-  extern __shared__ __align__(16) float Fs[];
+                                               const int32_t* pslot, const int32_t* permq,
+                                               const float* fitB, const float* fitU,
+                                               const float* fitBv, const spr_head_stats* stats,
+                                               int R, int N, int M, int H, int64_t sb, int64_t sh,
+                                               int64_t sn, bf16* O, int do_fit, Header* hdr) {
+  extern __shared__ __align__(16) float fsh[];
+  float* Bs = fsh;          // [D][R]
+  float* Us = fsh + D * R;  // [R][D]
   __shared__ float bv[D];
   constexpr int V = D / 32;  // values per lane
   const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int re = do_fit ? min(stats[bh].r_eff, R) : 0;
   if (do_fit) {
-    for (int e = tid; e < D * D; e += 256) Fs[e] = fitB[(size_t)bh * D * D + e];
+    for (int e = tid; e < D * R; e += 256) {
+      const int i = e / R, k = e % R;
+      Bs[e] = k < re ? fitB[((size_t)bh * D + i) * D + k] : 0.f;
+      Us[k * D + i] = k < re ? fitU[((size_t)bh * D + i) * D + k] : 0.f;
+    }
     for (int e = tid; e < D; e += 256) bv[e] = fitBv[(size_t)bh * D + e];
   }
   __syncthreads();
   const int b = bh / H, h = bh - b * H;
   bf16* ob = O + b * sb + h * sh;
-  const int32_t* pp = ppos + (size_t)bh * M;
   for (int pos = blockIdx.x * 8 + warp; pos < N; pos += gridDim.x * 8) {
     const float* xr = osp + ((size_t)bh * N + pos) * D;
     float x[V];
@@ -226,14 +299,10 @@ __global__ void __launch_bounds__(256) k_apply(const float* osp, const float* od
       x[0] = v.x; x[1 % V] = v.y;
     }
     // probe slot lookup (ppos ascending)
-    int slot = -1;
-    if (M > 0) {
-      int lo = 0, hi = M - 1;
-      while (lo <= hi) {
-        const int mid = (lo + hi) >> 1, v = pp[mid];
-        if (v == pos) { slot = mid; break; }
-        if (v < pos) lo = mid + 1; else hi = mid - 1;
-      }
+    const int slot = M > 0 ? pslot[(size_t)bh * N + pos] : -1;
+    if (slot >= M) {
+      set_error(hdr, ERR_INDEX, 21, bh, slot);
+      continue;
     }
     float y[V];
     if (slot >= 0) {
@@ -243,11 +312,20 @@ __global__ void __launch_bounds__(256) k_apply(const float* osp, const float* od
     } else if (do_fit) {
 #pragma unroll
       for (int k = 0; k < V; ++k) y[k] = x[k] + bv[lane * V + k];
+      // t = x B (lanes over the rank index, up to 4 per lane)
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
       for (int i = 0; i < D; ++i) {
         const float xi = __shfl_sync(0xffffffffu, x[i % V], i / V);
-        const float* fr = Fs + i * D + lane * V;
 #pragma unroll
-        for (int k = 0; k < V; ++k) y[k] += xi * fr[k];
+        for (int q = 0; q < 4; ++q)
+          if (lane + 32 * q < re) t[q] += xi * Bs[i * R + lane + 32 * q];
+      }
+      // y += t U_r^T
+      for (int k = 0; k < re; ++k) {
+        const float tk = __shfl_sync(0xffffffffu, t[k >> 5], k & 31);
+        const float* ur = Us + k * D + lane * V;
+#pragma unroll
+        for (int v = 0; v < V; ++v) y[v] += tk * ur[v];
       }
     } else {
 #pragma unroll
@@ -268,7 +346,6 @@ __global__ void __launch_bounds__(256) k_apply(const float* osp, const float* od
       *reinterpret_cast<uint32_t*>(dst) = pack_bf16(y[0], y[1 % V]);
     }
   }
-  (void)B_;
 }
 
 // Per-head accounting: probe pairs, rho_exec, k-means objectives.
@@ -296,22 +373,27 @@ static cudaError_t reconstruct_d(const spr_params& p, const Layout& L, const Ptr
   if (M > 0) {
     spr_launch(k_fit_moments<D>, BH, 1024, 0, st, P.osp, P.odn, P.ppos, P.pw, N, M, (float)p.lambda,
                                           P.gram, P.axx, P.rxbar);
-    cudaError_t e = launch_eig(P.gram, BH, D, P.eval, P.evec, st);
+    cudaError_t e = launch_eig(P.gram, BH, D, p.r > 0 ? p.r : 1, P.eval, P.evec, nullptr, st);
     if (e != cudaSuccess) return e;
+    const int R = p.r > 0 ? p.r : 1, nchunk = (M + FIT_TM - 1) / FIT_TM;
+    const size_t smr = (size_t)(2 * FIT_TM * D + D * R + FIT_TM * R) * 4;
+    cudaFuncSetAttribute(k_fit_rhs<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smr);
+    spr_launch(k_fit_rhs<D>, dim3(BH, nchunk), 256, smr, st, P.osp, P.odn, P.ppos, P.pw, N, M,
+               p.r, R, P.eval, P.evec, P.rxbar, P.proj);
     const size_t sm = (size_t)(D * (D + 1) + D * D) * 4;
     cudaFuncSetAttribute(k_fit_solve<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    spr_launch(k_fit_solve<D>, BH, 512, sm, st, P.osp, P.odn, P.ppos, P.pw, N, M, p.r, P.eval, P.evec,
-                                        P.axx, P.rxbar, P.proj, P.fitU, P.fitB, P.fitBv, P.stats,
-                                        P.hdr);
+    spr_launch(k_fit_solve<D>, BH, 512, sm, st, p.r, R, nchunk, P.eval, P.evec, P.axx, P.rxbar,
+               P.proj, P.fitU, P.fitB, P.fitBv, P.stats, P.hdr);
   } else {
     spr_launch(k_fit_zero, num_sms(), 256, 0, st, P.fitB, P.fitBv, D, BH);
   }
-  const size_t sm = (size_t)D * D * 4;
+  const int R = p.r > 0 ? p.r : 1;
+  const size_t sm = (size_t)2 * D * R * 4;
   cudaFuncSetAttribute(k_apply<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   const int bph = max(1, min((N + 7) / 8, (num_sms() * 4 + BH - 1) / BH));
-  spr_launch(k_apply<D>, dim3(bph, BH), 256, sm, st, P.osp, P.odn, P.ppos, P.permq, P.fitB, P.fitBv, N,
-                                             M, p.B, p.H, p.o_strides[0], p.o_strides[1],
-                                             p.o_strides[2], O, M > 0, P.hdr);
+  spr_launch(k_apply<D>, dim3(bph, BH), 256, sm, st, P.osp, P.odn, P.pslot, P.permq, P.fitB,
+             P.fitU, P.fitBv, P.stats, R, N, M, p.H, p.o_strides[0], p.o_strides[1],
+             p.o_strides[2], O, M > 0, P.hdr);
   spr_launch(k_stats, (BH + 127) / 128, 128, 0, st, P.stats, P.part, P.part + (size_t)BH * 2 * (L.nchunk + 1),
                                             L.nchunk, p.Gq, N, M, BH);
   return cudaGetLastError();

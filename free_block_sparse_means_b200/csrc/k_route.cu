@@ -278,9 +278,11 @@ __global__ void __launch_bounds__(256) k_route_csr(const uint8_t* sel, const int
 }
 
 // Stratified probes with coverage weights (reading R6).  Grid BH, block 256.
+// pslot[bh][pos] receives the probe slot of each probed permuted position (the
+// caller fills it with -1 first).
 __global__ void __launch_bounds__(256) k_probes(const int32_t* qoff, const int32_t* permq, int Gq,
                                                 int N, int M, int32_t* ppos, int32_t* pidx,
-                                                float* pw, spr_head_stats* stats) {
+                                                float* pw, int32_t* pslot, spr_head_stats* stats) {
   __shared__ int sh[32];
   __shared__ long long shl[32];
   __shared__ long long rems[MAX_GROUPS];
@@ -332,6 +334,7 @@ __global__ void __launch_bounds__(256) k_probes(const int32_t* qoff, const int32
       ppos[(size_t)bh * M + base + t] = pos;
       pidx[(size_t)bh * M + base + t] = permq[(size_t)bh * N + pos];
       pw[(size_t)bh * M + base + t] = w;
+      pslot[(size_t)bh * N + pos] = base + t;
     }
   }
 }
@@ -410,7 +413,10 @@ cudaError_t launch_route(const spr_params& p, const Layout& L, const Ptrs& P, cu
                p.N, p.M, p.rho_target, P.sel, P.stats);
   spr_launch(k_route_csr, BH, 256, 0, st, P.sel, P.qoff, P.kvoff, p.Gq, p.Gk, P.rowptr, P.colidx,
                                   P.runptr, P.runs, P.stats);
-  spr_launch(k_probes, BH, 256, 0, st, P.qoff, P.permq, p.Gq, p.N, p.M, P.ppos, P.pidx, P.pw, P.stats);
+  if (cudaMemsetAsync(P.pslot, 0xFF, (size_t)BH * p.N * sizeof(int32_t), st) != cudaSuccess)
+    return cudaGetLastError();
+  spr_launch(k_probes, BH, 256, 0, st, P.qoff, P.permq, p.Gq, p.N, p.M, P.ppos, P.pidx, P.pw,
+             P.pslot, P.stats);
   if (p.M > 0) {
     const int grid = num_sms() * 4;
     if (D == 64)

@@ -29,11 +29,11 @@ enum : int32_t {
 
 // Workspace buffers.
 enum Buf : int {
-  B_HDR, B_STATS, B_MK, B_EVAL, B_EVEC, B_W, B_Z, B_INITK, B_INITQ, B_CENTK,
+  B_HDR, B_STATS, B_MK, B_TRACE, B_EVAL, B_EVEC, B_W, B_Z, B_INITK, B_INITQ, B_CENTK,
   B_LABK, B_LABQ, B_CHUNK, B_CBASE, B_COUNTS, B_PERMK, B_KVOFF, B_PERMQ, B_QOFF,
   B_KP, B_VP, B_QP, B_CRAW, B_CT, B_AMAT, B_RMS, B_UN2, B_CENTQ, B_BQ16, B_BETA,
   B_QBAR, B_LOGIT, B_ENTRY, B_TOP, B_SEL, B_ROWPTR, B_COLIDX, B_RUNPTR, B_RUNS, B_PPOS,
-  B_PIDX, B_PW, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
+  B_PIDX, B_PW, B_PSLOT, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
   B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_COUNT_
 };
 
@@ -61,12 +61,12 @@ int padded_p(int p);
 struct Ptrs {
   Header* hdr;
   spr_head_stats* stats;
-  float *MK, *eval, *evec, *W, *Z, *centk, *Craw, *Ct, *Amat, *rms, *un2, *centq, *beta,
+  float *MK, *trace, *eval, *evec, *W, *Z, *centk, *Craw, *Ct, *Amat, *rms, *un2, *centq, *beta,
       *qbar, *logit, *entry, *pw, *osp, *odn, *fitU, *fitB, *fitBv, *gram, *axx, *rxbar,
       *proj;
   double* part;
   int32_t *initk, *initq, *labk, *labq, *chunk, *cbase, *counts, *permk, *kvoff, *permq,
-      *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx;
+      *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx, *pslot;
   int2* runs;
   int4* items;
   uint8_t *sel, *top;
@@ -94,10 +94,11 @@ cudaError_t launch_route(const spr_params& p, const Layout& L, const Ptrs& P, cu
 cudaError_t launch_attend(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st);
 cudaError_t launch_reconstruct(const spr_params& p, const Layout& L, const Ptrs& P,
                                bf16* O, cudaStream_t st);
-// Symmetric eigensolver: `count` matrices n x n (fp32, row-major) -> eigenvalues
-// descending and eigenvectors as columns, same order.
-cudaError_t launch_eig(const float* A, int count, int n, float* evals, float* evecs,
-                       cudaStream_t st);
+// Leading eigenpairs of `count` symmetric n x n matrices (fp32, row-major):
+// evals[m * n + k] for the K largest (descending), evecs[(m * n + row) * n + k]
+// the matching unit eigenvectors as columns, trace[m] the trace (may be null).
+cudaError_t launch_eig(const float* A, int count, int n, int K, float* evals, float* evecs,
+                       float* trace, cudaStream_t st);
 int num_sms();
 
 // Every kernel launch of the library goes through spr_launch, which counts it

@@ -193,8 +193,9 @@ typedef enum {
   SPR_VIEW_TAIL = 18,    /* [BH, Gq, Gk] fp32 tail mass of each cell: softmax mass of
                             the cells ranked at or after it (-1: empty group) */
   SPR_VIEW_FIT_U = 19,   /* [BH, d, d] fp32 residual basis (first r_eff cols) */
-  SPR_VIEW_FIT_B = 20,   /* [BH, d, d] fp32 full map B U_r^T */
-  SPR_VIEW_FIT_BVEC = 21,/* [BH, d] fp32 intercept Rbar - xbar B U_r^T */
+  SPR_VIEW_FIT_B = 20,   /* [BH, d, d] fp32 ridge coefficients B (first r_eff
+                            columns); the correction of a row x is b + (x B) U_r^T */
+  SPR_VIEW_FIT_BVEC = 21,/* [BH, d] fp32 intercept b = Rbar - (xbar B) U_r^T */
   SPR_VIEW_COUNT = 22
 } spr_view;
 

@@ -38,9 +38,13 @@ def test_mid_two_heads_full_length():
 @pytest.mark.parametrize("d,grid,mode", [(128, (3, 17, 29), "tau"), (64, (2, 23, 31), "budget"),
                                          (128, (1, 7, 19), "budget")])
 def test_ragged_lengths(d, grid, mode):
+    # More probes than head dimensions: with M <= d the ridge system is
+    # underdetermined and lambda = 1e-3 lets fp32-level differences in the
+    # probe rows move the correction by percents (the method's conditioning,
+    # not the kernels'), so these cases keep M > d.
     n = grid[0] * grid[1] * grid[2]
     wl = workload("mid", H=2, d=d, grid=grid, centers=24, Gk=24, Gq=20, Ms=min(300, n), p=16,
-                  M=min(100, n // 2), r=8, route_mode=mode, tau=0.85, rho_target=0.3)
+                  M=min(n - 1, 2 * d), r=8, route_mode=mode, tau=0.85, rho_target=0.3)
     g = run_gpu(wl)
     for bh in range(2):
         check_head(g, wl, bh)
