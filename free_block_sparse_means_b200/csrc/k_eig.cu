@@ -13,7 +13,8 @@
 //      one warp evaluates the Sturm count (number of eigenvalues below x, i.e.
 //      negative pivots of T - xI = L D L^T) at G points per step.
 //   3. Eigenvectors of T by inverse iteration on (T - lambda I) with partial
-//      pivoting, then modified Gram-Schmidt in descending eigenvalue order.
+//      pivoting, then orthonormalised in descending eigenvalue order by
+//      Cholesky QR (Y Y^T = L L^T, Y <- L^-1 Y).
 //   4. Back-transformation x = H_0 H_1 ... H_{n-3} y.
 // Outputs: evals[m][k] (descending, k < K), evecs[m][row][k] (stride n), and
 // the trace of each matrix.
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
   float* tau = tb2 + NN;         // reflector scales
   float* lam = tau + NN;         // eigenvalues (K)
   float* pw = lam + NN;          // p = tau A22 v
-  float* misc = pw + NN;         // [4]
+  float* misc = pw + NN;         // [8], then the Cholesky-QR Gram matrix
   const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* src = Ain + (size_t)m * NN * NN;
   for (int e = tid; e < NN * NN; e += EIG_THREADS) {
@@ -96,12 +97,19 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
     const float t = tau[k];
     if (t != 0.f) {
       const float* v = Vh + k * NN;
-      // p = t A22 v, one warp per row
-      for (int row = r0 + warp; row < NN; row += EIG_THREADS / 32) {
-        float s = 0.f;
-        for (int j = r0 + lane; j < NN; j += 32) s += A[row * LD + j] * v[j];
-        s = warp_sum(s);
-        if (lane == 0) pw[row] = t * s;
+      // p = t A22 v, one thread per row; A22 is kept exactly symmetric, so the
+      // thread reads its column (consecutive threads, consecutive addresses)
+      if (tid >= r0 && tid < NN) {
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        int j = r0;
+        for (; j + 3 < NN; j += 4) {
+          s0 += A[j * LD + tid] * v[j];
+          s1 += A[(j + 1) * LD + tid] * v[j + 1];
+          s2 += A[(j + 2) * LD + tid] * v[j + 2];
+          s3 += A[(j + 3) * LD + tid] * v[j + 3];
+        }
+        for (; j < NN; ++j) s0 += A[j * LD + tid] * v[j];
+        pw[tid] = t * ((s0 + s1) + (s2 + s3));
       }
       __syncthreads();
       float kk = 0.f;  // (t / 2) p.v, every warp for itself
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
     for (int i = 0; i < NN - 1; ++i) {
       const float sdn = tb[i], gn = ta[i + 1] - l, hn = (i + 1 < NN - 1) ? tb[i + 1] : 0.f;
       if (fabsf(g) >= fabsf(sdn)) {
-        const float mult = (g != 0.f) ? sdn / g : 0.f;
+        const float mult = (g != 0.f) ? __fdividef(sdn, g) : 0.f;
         ud[i] = g;
         us[i] = h;
         uf[i] = 0.f;
@@ -194,7 +202,7 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
         g = gn - mult * h;
         h = hn;
       } else {
-        const float mult = g / sdn;
+        const float mult = __fdividef(g, sdn);
         ud[i] = sdn;
         us[i] = gn;
         uf[i] = hn;
@@ -218,9 +226,10 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
         }
         y[i + 1] -= ml[i] * y[i];
       }
-      y[NN - 1] /= ud[NN - 1];  // back: U^-1
-      y[NN - 2] = (y[NN - 2] - us[NN - 2] * y[NN - 1]) / ud[NN - 2];
-      for (int i = NN - 3; i >= 0; --i) y[i] = (y[i] - us[i] * y[i + 1] - uf[i] * y[i + 2]) / ud[i];
+      y[NN - 1] = __fdividef(y[NN - 1], ud[NN - 1]);  // back: U^-1
+      y[NN - 2] = __fdividef(y[NN - 2] - us[NN - 2] * y[NN - 1], ud[NN - 2]);
+      for (int i = NN - 3; i >= 0; --i)
+        y[i] = __fdividef(y[i] - us[i] * y[i + 1] - uf[i] * y[i + 2], ud[i]);
       float nrm = 0.f;
       for (int i = 0; i < NN; ++i) nrm += y[i] * y[i];
       const float inv = nrm > 0.f ? rsqrtf(nrm) : 0.f;
@@ -229,23 +238,39 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
     for (int i = 0; i < NN; ++i) Y[e * LD + i] = y[i];
   }
   __syncthreads();
-  // modified Gram-Schmidt in descending eigenvalue order (one warp)
-  if (warp == 0) {
+  // Orthonormalise in descending eigenvalue order by Cholesky QR (the same
+  // basis as Gram-Schmidt in that order): Gm = Y Y^T = L L^T, Y <- L^-1 Y.
+  float* Gm = misc + 8;  // K x (K + 1)
+  const int GL = K + 1;
+  for (int e = tid; e < K * K; e += EIG_THREADS) {
+    const int a = e / K, b = e % K;
+    if (b <= a) {
+      float s = 0.f;
+      for (int i = 0; i < NN; ++i) s += Y[a * LD + i] * Y[b * LD + i];
+      Gm[a * GL + b] = s;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {  // Cholesky of Gm, lanes over rows
     for (int kq = 0; kq < K; ++kq) {
-      float* yk = Y + kq * LD;
-      for (int j = 0; j < kq; ++j) {
-        const float* yj = Y + j * LD;
-        float d = 0.f;
-        for (int i = lane; i < NN; i += 32) d += yj[i] * yk[i];
-        d = warp_sum(d);
-        for (int i = lane; i < NN; i += 32) yk[i] -= d * yj[i];
-      }
-      float n2 = 0.f;
-      for (int i = lane; i < NN; i += 32) n2 += yk[i] * yk[i];
-      n2 = warp_sum(n2);
-      const float inv = n2 > 0.f ? rsqrtf(n2) : 0.f;
-      for (int i = lane; i < NN; i += 32) yk[i] *= inv;
+      const float dkk = sqrtf(fmaxf(Gm[kq * GL + kq], 1e-30f));
       __syncwarp();
+      for (int i = kq + 1 + lane; i < K; i += 32) Gm[i * GL + kq] /= dkk;
+      if (lane == 0) Gm[kq * GL + kq] = dkk;
+      __syncwarp();
+      for (int i = kq + 1 + lane; i < K; i += 32) {
+        const float lik = Gm[i * GL + kq];
+        for (int j = kq + 1; j <= i; ++j) Gm[i * GL + j] -= lik * Gm[j * GL + kq];
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < NN; i += EIG_THREADS) {  // forward substitution per column of Y
+    for (int a = 0; a < K; ++a) {
+      float s = Y[a * LD + i];
+      for (int b = 0; b < a; ++b) s -= Gm[a * GL + b] * Y[b * LD + i];
+      Y[a * LD + i] = s / Gm[a * GL + a];
     }
   }
   __syncthreads();
@@ -274,7 +299,8 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
 template <int NN>
 static cudaError_t eig_n(const float* A, int count, int K, float* ev, float* evec, float* trace,
                          cudaStream_t st) {
-  const size_t smem = (size_t)(NN * (NN + 1) + NN * NN + 7 * NN + 8) * 4;
+  // A / Y, reflectors, T and scratch vectors, misc, Cholesky-QR Gram (K <= NN)
+  const size_t smem = (size_t)(NN * (NN + 1) + NN * NN + 6 * NN + 8 + NN * (NN + 1)) * 4;
   cudaError_t e = cudaFuncSetAttribute(k_eig_top<NN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

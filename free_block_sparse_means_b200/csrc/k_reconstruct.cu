@@ -261,8 +261,11 @@ __global__ void k_fit_zero(float* fitB, float* fitBv, int D, int BH) {
 
 // O[orig row] = x + b + (x B) U_r^T (unprobed) or the dense probe row; bf16
 // output in the original query order.  Grid (blocks per head, BH), 256
-// threads, one warp per permuted row.  Dynamic smem: B as [D][R] and U_r as
-// [R][D] (R = the rank bound of the call).
+// threads; each block takes tiles of APPLY_TR consecutive permuted rows:
+// T = X B (tile x r) and Y = X + b + T U_r^T from shared memory.
+// Dynamic smem: B as [D][R], U_r as [R][D], the X tile and T.
+constexpr int APPLY_TR = 32;
+
 template <int D>
 __global__ void __launch_bounds__(256) k_apply(const float* osp, const float* odn,
                                                const int32_t* pslot, const int32_t* permq,
@@ -271,79 +274,77 @@ __global__ void __launch_bounds__(256) k_apply(const float* osp, const float* od
                                                int R, int N, int M, int H, int64_t sb, int64_t sh,
                                                int64_t sn, bf16* O, int do_fit, Header* hdr) {
   extern __shared__ __align__(16) float fsh[];
-  float* Bs = fsh;          // [D][R]
-  float* Us = fsh + D * R;  // [R][D]
+  constexpr int XL = D + 4;  // padded row of the X tile
+  float* Bs = fsh;                    // [D][R]
+  float* Us = Bs + D * R;             // [R][D]
+  float* Xs = Us + R * D;             // [APPLY_TR][XL]
+  float* Ts = Xs + APPLY_TR * XL;     // [APPLY_TR][R]
   __shared__ float bv[D];
-  constexpr int V = D / 32;  // values per lane
-  const int bh = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ int slot_s[APPLY_TR], orig_s[APPLY_TR];
+  const int bh = blockIdx.y, tid = threadIdx.x;
   const int re = do_fit ? min(stats[bh].r_eff, R) : 0;
-  if (do_fit) {
-    for (int e = tid; e < D * R; e += 256) {
-      const int i = e / R, k = e % R;
-      Bs[e] = k < re ? fitB[((size_t)bh * D + i) * D + k] : 0.f;
-      Us[k * D + i] = k < re ? fitU[((size_t)bh * D + i) * D + k] : 0.f;
-    }
-    for (int e = tid; e < D; e += 256) bv[e] = fitBv[(size_t)bh * D + e];
+  for (int e = tid; e < D * R; e += 256) {
+    const int i = e / R, k = e % R;
+    Bs[e] = k < re ? fitB[((size_t)bh * D + i) * D + k] : 0.f;
+    Us[k * D + i] = k < re ? fitU[((size_t)bh * D + i) * D + k] : 0.f;
   }
-  __syncthreads();
+  for (int e = tid; e < D; e += 256) bv[e] = do_fit ? fitBv[(size_t)bh * D + e] : 0.f;
   const int b = bh / H, h = bh - b * H;
   bf16* ob = O + b * sb + h * sh;
-  for (int pos = blockIdx.x * 8 + warp; pos < N; pos += gridDim.x * 8) {
-    const float* xr = osp + ((size_t)bh * N + pos) * D;
-    float x[V];
-    if (V == 4) {
-      const float4 v = reinterpret_cast<const float4*>(xr)[lane];
-      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3 % V] = v.w;
-    } else {
-      const float2 v = reinterpret_cast<const float2*>(xr)[lane];
-      x[0] = v.x; x[1 % V] = v.y;
+  const int ntile = (N + APPLY_TR - 1) / APPLY_TR;
+  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x) {
+    const int pos0 = tile * APPLY_TR;
+    __syncthreads();  // previous tile fully consumed
+    for (int e = tid; e < APPLY_TR * (D / 4); e += 256) {
+      const int r = e / (D / 4), c4 = e % (D / 4), pos = pos0 + r;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (pos < N) v = reinterpret_cast<const float4*>(osp + ((size_t)bh * N + pos) * D)[c4];
+      *reinterpret_cast<float4*>(Xs + r * XL + c4 * 4) = v;
     }
-    // probe slot lookup (ppos ascending)
-    const int slot = M > 0 ? pslot[(size_t)bh * N + pos] : -1;
-    if (slot >= M) {
-      set_error(hdr, ERR_INDEX, 21, bh, slot);
-      continue;
-    }
-    float y[V];
-    if (slot >= 0) {
-      const float* dr = odn + ((size_t)bh * M + slot) * D;
-#pragma unroll
-      for (int k = 0; k < V; ++k) y[k] = dr[lane * V + k];
-    } else if (do_fit) {
-#pragma unroll
-      for (int k = 0; k < V; ++k) y[k] = x[k] + bv[lane * V + k];
-      // t = x B (lanes over the rank index, up to 4 per lane)
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int i = 0; i < D; ++i) {
-        const float xi = __shfl_sync(0xffffffffu, x[i % V], i / V);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (lane + 32 * q < re) t[q] += xi * Bs[i * R + lane + 32 * q];
+    if (tid < APPLY_TR) {
+      const int pos = pos0 + tid;
+      int slot = -1, orig = -1;
+      if (pos < N) {
+        slot = M > 0 ? pslot[(size_t)bh * N + pos] : -1;
+        orig = permq[(size_t)bh * N + pos];
+        if (slot >= M || orig < 0 || orig >= N) {
+          set_error(hdr, ERR_INDEX, 20, bh, pos);
+          orig = -1;
+        }
       }
-      // y += t U_r^T
-      for (int k = 0; k < re; ++k) {
-        const float tk = __shfl_sync(0xffffffffu, t[k >> 5], k & 31);
-        const float* ur = Us + k * D + lane * V;
-#pragma unroll
-        for (int v = 0; v < V; ++v) y[v] += tk * ur[v];
+      slot_s[tid] = slot;
+      orig_s[tid] = orig;
+    }
+    __syncthreads();
+    if (re > 0) {
+      for (int e = tid; e < APPLY_TR * re; e += 256) {
+        const int r = e / re, k = e % re;
+        float s = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; ++i) s += Xs[r * XL + i] * Bs[i * R + k];
+        Ts[r * R + k] = s;
       }
-    } else {
-#pragma unroll
-      for (int k = 0; k < V; ++k) y[k] = x[k];
+      __syncthreads();
     }
-    const int orig = permq[(size_t)bh * N + pos];
-    if (orig < 0 || orig >= N) {
-      set_error(hdr, ERR_INDEX, 20, bh, orig);
-      continue;
-    }
-    bf16* dst = ob + (int64_t)orig * sn + lane * V;
-    if (V == 4) {
-      uint2 u;
-      u.x = pack_bf16(y[0], y[1 % V]);
-      u.y = pack_bf16(y[2 % V], y[3 % V]);
-      *reinterpret_cast<uint2*>(dst) = u;
-    } else {
-      *reinterpret_cast<uint32_t*>(dst) = pack_bf16(y[0], y[1 % V]);
+    for (int e = tid; e < APPLY_TR * (D / 2); e += 256) {
+      const int r = e / (D / 2), j = 2 * (e % (D / 2));
+      const int orig = orig_s[r];
+      if (orig < 0) continue;
+      float y0, y1;
+      if (slot_s[r] >= 0) {
+        const float* dr = odn + ((size_t)bh * M + slot_s[r]) * D + j;
+        y0 = dr[0];
+        y1 = dr[1];
+      } else {
+        y0 = Xs[r * XL + j] + bv[j];
+        y1 = Xs[r * XL + j + 1] + bv[j + 1];
+        for (int k = 0; k < re; ++k) {
+          const float tk = Ts[r * R + k];
+          y0 += tk * Us[k * D + j];
+          y1 += tk * Us[k * D + j + 1];
+        }
+      }
+      *reinterpret_cast<uint32_t*>(ob + (int64_t)orig * sn + j) = pack_bf16(y0, y1);
     }
   }
 }
@@ -388,9 +389,9 @@ static cudaError_t reconstruct_d(const spr_params& p, const Layout& L, const Ptr
     spr_launch(k_fit_zero, num_sms(), 256, 0, st, P.fitB, P.fitBv, D, BH);
   }
   const int R = p.r > 0 ? p.r : 1;
-  const size_t sm = (size_t)2 * D * R * 4;
+  const size_t sm = (size_t)(2 * D * R + APPLY_TR * (D + 4) + APPLY_TR * R) * 4;
   cudaFuncSetAttribute(k_apply<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  const int bph = max(1, min((N + 7) / 8, (num_sms() * 4 + BH - 1) / BH));
+  const int bph = max(1, min((N + APPLY_TR - 1) / APPLY_TR, (num_sms() * 4 + BH - 1) / BH));
   spr_launch(k_apply<D>, dim3(bph, BH), 256, sm, st, P.osp, P.odn, P.pslot, P.permq, P.fitB,
              P.fitU, P.fitBv, P.stats, R, N, M, p.H, p.o_strides[0], p.o_strides[1],
              p.o_strides[2], O, M > 0, P.hdr);
