@@ -235,6 +235,7 @@ __global__ void k_attend_reset(Header* hdr, spr_head_stats* stats, int BH) {
 
 cudaError_t launch_attend(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st) {
   spr_launch(k_attend_reset, 1, 256, 0, st, P.hdr, P.stats, L.BH);
+  if (attend_tc_enabled(p.d)) return launch_attend_tc(p, L, P, st);
   AttArgs a;
   a.Qp = P.Qp;
   a.Kp = P.Kp;

@@ -1,0 +1,458 @@
+// Routed attention on the 5th-generation tensor cores (tcgen05, TMEM, TMA) for
+// head dimension 128 [paperlayer §1, §4 "Sparse Execution"; App. A.2].
+//
+// Each work item is a tile of up to 128 query rows (one query group's rows in
+// the group-major layout, or 128 gathered probe rows) plus its key ranges (the
+// merged K/V groups routed to the query group, or [0, N) for probes).  Every
+// row's softmax is renormalised over exactly those keys (hard drop).
+//
+// One persistent CTA per SM, 8 warps, items taken round-robin:
+//   warp 0      TMA producer: Q tile once per item, K and V tiles of 128 keys
+//               into a two-stage ring (128-byte-swizzled boxes of 64 columns).
+//   warp 1      owns TMEM (512 columns: S0, S1, O) and issues the MMAs from one
+//               thread: S = Q K^T (A and B K-major in shared memory) into the
+//               S buffer of the tile, and O += P V with P read from TMEM (the
+//               bf16 probabilities the softmax wrote over S) and V as an
+//               MN-major B operand.
+//   warps 4..7  one thread per query row (= TMEM lane): scaled, masked row
+//               max, exp2, row sums, P back to TMEM; O is rescaled in TMEM only
+//               when the running max grows by more than 2^8 (the final
+//               normalisation uses the same stale max, so this is exact);
+//               epilogue O / l to global memory.
+// Every mbarrier wait is bounded in time; a wait that runs out sets an abort
+// flag that ends every role, the device error word records a timeout, copies
+// and MMAs in flight are drained, and TMEM is freed.
+#include <cudaTypedefs.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "tc_sm100.cuh"
+
+namespace spr {
+
+namespace {
+
+constexpr int TBM = 128, TBN = 128, TD = 128;
+constexpr uint32_t TILE_BYTES = TBN * TD * 2;  // one Q, K or V tile: 32 KB
+constexpr uint32_t BOX_BYTES = TBN * 64 * 2;   // one 64-column swizzled box: 16 KB
+constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, TMEM_COLS = 512;
+constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s
+constexpr size_t SMEM_BYTES = 1024 + 5 * TILE_BYTES + 256;
+
+struct TcArgs {
+  const int4* items;
+  const int32_t* runptr;
+  const int2* runs;
+  int N, M, Gq, Gk;
+  float scale_log2;
+  float* osp;
+  float* odn;
+  Header* hdr;
+  spr_head_stats* stats;
+};
+
+// Key tiles of one item: for each key range [x, y), tiles start at x, x+128, ...
+struct TileIter {
+  const int2* runs;
+  int r, rend, t0;
+  int2 run;
+  bool valid;
+  __device__ void init(const TcArgs& a, const int4& it) {
+    runs = nullptr;
+    r = 0;
+    rend = 1;
+    run = make_int2(0, a.N);
+    if (it.w >= 0) {
+      r = a.runptr[(size_t)it.x * (a.Gq + 1) + it.w];
+      rend = a.runptr[(size_t)it.x * (a.Gq + 1) + it.w + 1];
+      runs = a.runs + (size_t)it.x * a.Gq * a.Gk;
+      run = r < rend ? runs[r] : make_int2(0, 0);
+    }
+    t0 = run.x;
+    valid = r < rend && run.x < run.y;
+  }
+  __device__ void next() {
+    t0 += TBN;
+    if (t0 >= run.y) {
+      ++r;
+      if (r < rend) {
+        run = runs[r];
+        t0 = run.x;
+      } else {
+        valid = false;
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
+
+__global__ void __launch_bounds__(256, 1)
+    k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQprobe,
+                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK[2] = {base + TILE_BYTES, base + 2 * TILE_BYTES};
+  uint8_t* sV[2] = {base + 3 * TILE_BYTES, base + 4 * TILE_BYTES};
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + 5 * TILE_BYTES);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;   // [2]
+  uint64_t* kv_empty = bars + 4;  // [2]
+  uint64_t* s_full = bars + 6;    // [2]
+  uint64_t* p_full = bars + 8;    // [2]
+  uint64_t* o_done = bars + 10;
+  uint64_t* o_free = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(bars + 15);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = a.hdr->n_items;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full, 1);
+    tc::mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(kv_full + s, 1);
+      tc::mbar_init(kv_empty + s, 1);
+      tc::mbar_init(s_full + s, 1);
+      tc::mbar_init(p_full + s, 128);
+    }
+    tc::mbar_init(o_done, 1);
+    tc::mbar_init(o_free, 128);
+    tc::mbar_init(drain, 1);
+    *abort_s = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tmap(&tmQ);
+    tc::prefetch_tmap(&tmQprobe);
+    tc::prefetch_tmap(&tmK);
+    tc::prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_base_s, TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = *tmem_base_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int kv = 0, itc = 0, q_loads = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++itc) {
+        const int4 it = a.items[item];
+        TileIter I;
+        I.init(a, it);
+        if (itc > 0 && !tc::mbar_wait(q_empty, (itc - 1) & 1, abort_s, WAIT_NS)) {
+          ok = false;
+          break;
+        }
+        tc::mbar_expect_tx(q_full, TILE_BYTES);
+        const CUtensorMap* qm = it.w >= 0 ? &tmQ : &tmQprobe;
+        const int qrow = it.w >= 0 ? it.x * a.N + it.y : it.x * a.M + it.y;
+        tc::tma_load_2d(sQ, qm, 0, qrow, q_full);
+        tc::tma_load_2d(sQ + BOX_BYTES, qm, 64, qrow, q_full);
+        ++q_loads;
+        for (; I.valid; I.next(), ++kv) {
+          const int s = kv & 1;
+          if (kv >= 2 && !tc::mbar_wait(kv_empty + s, ((kv >> 1) - 1) & 1, abort_s, WAIT_NS)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_expect_tx(kv_full + s, 2 * TILE_BYTES);
+          const int krow = it.x * a.N + I.t0;
+          tc::tma_load_2d(sK[s], &tmK, 0, krow, kv_full + s);
+          tc::tma_load_2d(sK[s] + BOX_BYTES, &tmK, 64, krow, kv_full + s);
+          tc::tma_load_2d(sV[s], &tmV, 0, krow, kv_full + s);
+          tc::tma_load_2d(sV[s] + BOX_BYTES, &tmV, 64, krow, kv_full + s);
+        }
+      }
+      if (*abort_s) {  // let our copies in flight land before the block exits
+        for (int k = kv - 2; k < kv; ++k)
+          if (k >= 0) tc::mbar_wait_bounded(kv_full + (k & 1), (k >> 1) & 1, 100000000ull);
+        if (q_loads > 0) tc::mbar_wait_bounded(q_full, (q_loads - 1) & 1, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = tc::idesc_bf16(TBM, TBN, 0);
+      const uint32_t idPV = tc::idesc_bf16(TBM, TD, 1);
+      const uint32_t q_addr = smem_u32(sQ);
+      int kv = 0, pg = 0, itc = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++itc) {
+        const int4 it = a.items[item];
+        TileIter Is, Ip;
+        Is.init(a, it);
+        Ip.init(a, it);
+        if (!tc::mbar_wait(q_full, itc & 1, abort_s, WAIT_NS)) break;
+        int kv_s = kv, sg = pg;
+        auto issue_s = [&]() -> bool {
+          const int s = kv_s & 1;
+          if (!tc::mbar_wait(kv_full + s, (kv_s >> 1) & 1, abort_s, WAIT_NS)) return false;
+          tc::tc_fence_after();
+          const uint32_t d = tbase + ((sg & 1) ? S_COL1 : S_COL0);
+          const uint32_t k_addr = smem_u32(sK[s]);
+#pragma unroll
+          for (int ks = 0; ks < TD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * BOX_BYTES + (ks & 3) * 32;
+            tc::mma_ss(d, tc::smem_desc_sw128(q_addr + off, 16, 1024),
+                       tc::smem_desc_sw128(k_addr + off, 16, 1024), idS, ks > 0);
+          }
+          tc::mma_commit(s_full + (sg & 1));
+          ++kv_s;
+          ++sg;
+          return true;
+        };
+        for (int k = 0; k < 2 && Is.valid && ok; ++k) {
+          ok = issue_s();
+          Is.next();
+        }
+        bool first = true;
+        for (; Ip.valid && ok; Ip.next()) {
+          const int b = pg & 1;
+          if (!tc::mbar_wait(p_full + b, (pg >> 1) & 1, abort_s, WAIT_NS)) {
+            ok = false;
+            break;
+          }
+          if (first && itc > 0 && !tc::mbar_wait(o_free, (itc - 1) & 1, abort_s, WAIT_NS)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const int s = kv & 1;
+          const uint32_t v_addr = smem_u32(sV[s]);
+          const uint32_t p_col = tbase + (b ? S_COL1 : S_COL0);
+#pragma unroll
+          for (int kk = 0; kk < TBN / 16; ++kk)
+            tc::mma_ts(tbase + O_COL, p_col + kk * 8,
+                       tc::smem_desc_sw128(v_addr + kk * 2048, BOX_BYTES, 1024), idPV,
+                       !(first && kk == 0));
+          tc::mma_commit(kv_empty + s);
+          tc::mma_commit(o_done);
+          first = false;
+          ++kv;
+          ++pg;
+          if (Is.valid) {
+            ok = issue_s();
+            Is.next();
+          }
+        }
+        tc::mma_commit(q_empty);
+      }
+      // drain: every MMA issued so far completes before TMEM is released
+      tc::mma_commit(drain);
+      tc::mbar_wait_bounded(drain, 0, WAIT_NS);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int row = threadIdx.x - 128;                 // query row in the tile
+    const uint32_t lane_f = (uint32_t)((warp & 3) * 32) << 16;  // TMEM lane field
+    int pg = 0, pvseen = 0, itc = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++itc) {
+      const int4 it = a.items[item];
+      TileIter I;
+      I.init(a, it);
+      float m = -INFINITY, l = 0.f;
+      bool first = true;
+      int ntiles = 0;
+      for (; I.valid; I.next(), ++pg, ++ntiles) {
+        const int b = pg & 1;
+        const uint32_t scol = tbase + lane_f + (b ? S_COL1 : S_COL0);
+        const bool got_s = tc::mbar_wait(s_full + b, (pg >> 1) & 1, abort_s, WAIT_NS);
+        __syncwarp();  // TMEM loads and stores below are warp-collective
+        if (!__all_sync(0xffffffffu, got_s)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        uint32_t sr[TBN];
+#pragma unroll
+        for (int c = 0; c < TBN / 32; ++c) tc::tmem_ld32(scol + 32 * c, sr + 32 * c);
+        tc::tmem_wait_ld();
+        const int nvalid = min(TBN, I.run.y - I.t0);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < TBN; ++c) {
+          const float x = c < nvalid ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
+          sr[c] = f2u(x);
+          mx = fmaxf(mx, x);
+        }
+        const float mn = fmaxf(m, mx);
+        float m_use = m;
+        bool rescale = false;
+        if (first || mn > m + 8.f) {
+          m_use = mn;
+          rescale = !first;
+        }
+        const float corr = rescale ? ex2(m - m_use) : 1.f;
+        float sum = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pr[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = ex2(__uint_as_float(sr[64 * h + 2 * c]) - m_use);
+            const float p1 = ex2(__uint_as_float(sr[64 * h + 2 * c + 1]) - m_use);
+            sum += p0 + p1;
+            pr[c] = pack_bf16(p0, p1);
+          }
+          __syncwarp();
+          tc::tmem_st32(scol + 32 * h, pr);
+        }
+        if (!first) {  // O holds PV of the previous tile once it is done
+          const bool got_o = tc::mbar_wait(o_done, pvseen & 1, abort_s, WAIT_NS);
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, got_o)) {
+            ok = false;
+            break;
+          }
+          ++pvseen;
+          tc::tc_fence_after();
+          // the rescale is per row, the TMEM access per warp: a warp rescales
+          // when any of its rows needs it (the others multiply by 1)
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int c = 0; c < TD / 32; ++c) {
+              uint32_t o[32];
+              __syncwarp();
+              tc::tmem_ld32(tbase + lane_f + O_COL + 32 * c, o);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = f2u(__uint_as_float(o[e]) * corr);
+              __syncwarp();
+              tc::tmem_st32(tbase + lane_f + O_COL + 32 * c, o);
+            }
+          }
+        }
+        l = l * corr + sum;
+        m = m_use;
+        __syncwarp();
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(p_full + b);
+        first = false;
+      }
+      if (!ok) break;
+      if (ntiles == 0) {  // keep one o_free phase per item
+        tc::mbar_arrive(o_free);
+        continue;
+      }
+      const bool got_o = tc::mbar_wait(o_done, pvseen & 1, abort_s, WAIT_NS);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got_o)) {
+        ok = false;
+        break;
+      }
+      ++pvseen;
+      tc::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float* dst = it.w >= 0 ? a.osp + ((size_t)it.x * a.N + it.y + row) * TD
+                             : a.odn + ((size_t)it.x * a.M + it.y + row) * TD;
+#pragma unroll
+      for (int c = 0; c < TD / 32; ++c) {
+        uint32_t o[32];
+        __syncwarp();
+        tc::tmem_ld32(tbase + lane_f + O_COL + 32 * c, o);
+        tc::tmem_wait_ld();
+        if (row < it.z) {
+          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            d4[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                __uint_as_float(o[4 * e + 2]) * inv,
+                                __uint_as_float(o[4 * e + 3]) * inv);
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(o_free);
+      if (row == 0)
+        atomicAdd(reinterpret_cast<unsigned long long*>(&a.stats[it.x].tile_pairs),
+                  (unsigned long long)ntiles * TBN * TBM);
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (threadIdx.x == 0 && *abort_s) set_error(a.hdr, ERR_TIMEOUT, blockIdx.x, 0, 0);
+  if (warp == 1) {
+    __syncwarp();  // lane 0 comes from the MMA loop, the others from the barrier
+    tc::tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major [rows, 128] bf16 tensor, 64 x 128 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)TD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)TD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)TBN};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// The tcgen05 path serves d = 128 unless SPR_ATTEND=mma selects the mma.sync
+// kernel (kept for d = 64 and for side-by-side checks).
+bool attend_tc_enabled(int d) {
+  if (d != 128) return false;
+  const char* e = getenv("SPR_ATTEND");
+  return !(e && strcmp(e, "mma") == 0);
+}
+
+cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P,
+                             cudaStream_t st) {
+  CUtensorMap mQ, mQp, mK, mV;
+  const uint64_t rows = (uint64_t)L.BH * p.N;
+  if (!make_map(&mQ, P.Qp, rows) || !make_map(&mK, P.Kp, rows) || !make_map(&mV, P.Vp, rows))
+    return cudaErrorInvalidValue;
+  if (!make_map(&mQp, P.qprobe, (uint64_t)L.BH * (p.M > 0 ? p.M : 1))) return cudaErrorInvalidValue;
+  TcArgs a;
+  a.items = P.items;
+  a.runptr = P.runptr;
+  a.runs = P.runs;
+  a.N = p.N;
+  a.M = p.M;
+  a.Gq = p.Gq;
+  a.Gk = p.Gk;
+  const float scale = p.scale > 0.f ? p.scale : 1.f / sqrtf((float)p.d);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.osp = P.osp;
+  a.odn = P.odn;
+  a.hdr = P.hdr;
+  a.stats = P.stats;
+  cudaError_t e = cudaFuncSetAttribute(k_attend_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  spr_launch(k_attend_tc, num_sms(), 256, SMEM_BYTES, st, mQ, mQp, mK, mV, a);
+  return cudaGetLastError();
+}
+
+}  // namespace spr

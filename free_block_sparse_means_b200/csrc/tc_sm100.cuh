@@ -57,12 +57,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > limit_ns) {
+      // time bound, and an iteration bound in case the timer does not advance
+      if (globaltimer() - t0 > limit_ns || it > (1u << 26)) {
         *abort = 1;
         return false;
       }
     }
   }
+}
+
+// Time-bounded wait that ignores the abort flag (used while draining).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it)
+    if (globaltimer() - t0 > limit_ns || it > (1u << 26)) return false;
+  return true;
 }
 
 // ---- TMA ----------------------------------------------------------------------

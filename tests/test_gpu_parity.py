@@ -112,3 +112,36 @@ def test_strided_inputs_and_output():
     torch.cuda.synchronize()
     got = Ot.float().cpu().reshape(-1, wl.N, wl.d).numpy()
     assert np.array_equal(got, g_ref["O"].astype(np.float32))
+
+
+def _osp_with(impl, wl):
+    import os
+    from synthetic import voronoi_qkv
+    old = os.environ.get("SPR_ATTEND")
+    os.environ["SPR_ATTEND"] = impl
+    try:
+        return run_gpu(wl, inputs=voronoi_qkv(wl))
+    finally:
+        if old is None:
+            del os.environ["SPR_ATTEND"]
+        else:
+            os.environ["SPR_ATTEND"] = old
+
+
+def test_tcgen05_small_d128():
+    """Smallest d = 128 case first: one head, 256 tokens, short key ranges."""
+    wl = workload("mid", H=1, grid=(1, 8, 32), centers=8, Gk=8, Gq=8, Ms=128, M=160, r=8)
+    g = run_gpu(wl)
+    check_head(g, wl, 0)
+
+
+def test_tcgen05_matches_mma_sync():
+    """The tcgen05 kernel and the mma.sync kernel agree on the same partition."""
+    wl = workload("mid", H=2, grid=(4, 32, 32))
+    a = _osp_with("tc", wl)
+    b = _osp_with("mma", wl)
+    assert (a["perm_q"] == b["perm_q"]).all() and (a["row_ptr"] == b["row_ptr"]).all()
+    assert rel_l2(a["o_sparse"].astype(np.float64), b["o_sparse"].astype(np.float64)) < 2e-3
+    assert rel_l2(a["o_probe"].astype(np.float64), b["o_probe"].astype(np.float64)) < 2e-3
+    assert rel_l2(a["O"], b["O"]) < 5e-3
+    assert a["stats"][0]["tile_pairs"] > 0
