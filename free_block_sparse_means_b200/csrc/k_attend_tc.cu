@@ -6,14 +6,18 @@
 // merged K/V groups routed to the query group, or [0, N) for probes).  Every
 // row's softmax is renormalised over exactly those keys (hard drop).
 //
-// One persistent CTA per SM, 8 warps, items taken round-robin:
-//   warp 0      TMA producer: Q tile once per item, K and V tiles of 128 keys
-//               into a two-stage ring (128-byte-swizzled boxes of 64 columns).
+// One persistent CTA per SM, 8 warps:
+//   warp 0      producer: takes the next item from the global cursor and
+//               publishes it in a 4-slot shared-memory ring for the other
+//               roles; TMA-loads the Q tile once per item and K and V tiles of
+//               128 keys into a three-stage ring (128-byte-swizzled boxes of 64
+//               columns).
 //   warp 1      owns TMEM (512 columns: S0, S1, O) and issues the MMAs from one
 //               thread: S = Q K^T (A and B K-major in shared memory) into the
 //               S buffer of the tile, and O += P V with P read from TMEM (the
 //               bf16 probabilities the softmax wrote over S) and V as an
-//               MN-major B operand.
+//               MN-major B operand.  A tile whose key range ends early is
+//               multiplied only up to its last 16-key block.
 //   warps 4..7  one thread per query row (= TMEM lane): scaled, masked row
 //               max, exp2, row sums, P back to TMEM; O is rescaled in TMEM only
 //               when the running max grows by more than 2^8 (the final
@@ -21,7 +25,8 @@
 //               epilogue O / l to global memory.
 // Every mbarrier wait is bounded in time; a wait that runs out sets an abort
 // flag that ends every role, the device error word records a timeout, copies
-// and MMAs in flight are drained, and TMEM is freed.
+// and MMAs in flight are drained, and TMEM is freed.  TMEM loads and stores
+// are warp-collective, so the softmax warps reconverge before each one.
 #include <cudaTypedefs.h>
 #include <stdlib.h>
 #include <string.h>
@@ -33,11 +38,13 @@ namespace spr {
 namespace {
 
 constexpr int TBM = 128, TBN = 128, TD = 128;
+constexpr int NST = 3;                         // K/V pipeline stages
+constexpr int NITQ = 4;                        // item ring slots
 constexpr uint32_t TILE_BYTES = TBN * TD * 2;  // one Q, K or V tile: 32 KB
 constexpr uint32_t BOX_BYTES = TBN * 64 * 2;   // one 64-column swizzled box: 16 KB
 constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, TMEM_COLS = 512;
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s
-constexpr size_t SMEM_BYTES = 1024 + 5 * TILE_BYTES + 256;
+constexpr size_t SMEM_BYTES = 1024 + (1 + 2 * NST) * TILE_BYTES + 512;
 
 struct TcArgs {
   const int4* items;
@@ -71,6 +78,7 @@ struct TileIter {
     t0 = run.x;
     valid = r < rend && run.x < run.y;
   }
+  __device__ int nvalid() const { return min(TBN, run.y - t0); }
   __device__ void next() {
     t0 += TBN;
     if (t0 >= run.y) {
@@ -95,31 +103,39 @@ __global__ void __launch_bounds__(256, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = base;
-  uint8_t* sK[2] = {base + TILE_BYTES, base + 2 * TILE_BYTES};
-  uint8_t* sV[2] = {base + 3 * TILE_BYTES, base + 4 * TILE_BYTES};
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + 5 * TILE_BYTES);
+  uint8_t* sKV = base + TILE_BYTES;  // stage s: K at sKV + 2s tiles, V right after
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (1 + 2 * NST) * TILE_BYTES);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;   // [2]
-  uint64_t* kv_empty = bars + 4;  // [2]
-  uint64_t* s_full = bars + 6;    // [2]
-  uint64_t* p_full = bars + 8;    // [2]
-  uint64_t* o_done = bars + 10;
-  uint64_t* o_free = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 14);
-  volatile int* abort_s = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* kv_full = bars + 2;         // [NST]
+  uint64_t* kv_empty = bars + 2 + NST;  // [NST]
+  uint64_t* s_full = bars + 2 + 2 * NST;   // [2]
+  uint64_t* p_full = bars + 4 + 2 * NST;   // [2]
+  uint64_t* o_done = bars + 6 + 2 * NST;
+  uint64_t* o_free = bars + 7 + 2 * NST;
+  uint64_t* drain = bars + 8 + 2 * NST;
+  uint64_t* it_full = bars + 9 + 2 * NST;           // [NITQ]
+  uint64_t* it_empty = bars + 9 + 2 * NST + NITQ;   // [NITQ]
+  int* it_ring = reinterpret_cast<int*>(bars + 9 + 2 * NST + 2 * NITQ);  // [NITQ]
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(it_ring + NITQ);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = a.hdr->n_items;
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
     tc::mbar_init(q_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NST; ++s) {
       tc::mbar_init(kv_full + s, 1);
       tc::mbar_init(kv_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       tc::mbar_init(s_full + s, 1);
       tc::mbar_init(p_full + s, 128);
+    }
+    for (int s = 0; s < NITQ; ++s) {
+      tc::mbar_init(it_full + s, 1);
+      tc::mbar_init(it_empty + s, 1 + 128);  // the MMA thread and every softmax thread
     }
     tc::mbar_init(o_done, 1);
     tc::mbar_init(o_free, 128);
@@ -145,16 +161,20 @@ __global__ void __launch_bounds__(256, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int kv = 0, itc = 0, q_loads = 0;
+      int kv = 0, q_loads = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++itc) {
+      for (int k = 0; ok; ++k) {
+        const int slot = k % NITQ;
+        if (k >= NITQ && !tc::mbar_wait(it_empty + slot, ((k / NITQ) - 1) & 1, abort_s, WAIT_NS))
+          break;
+        const int item = (int)atomicAdd(&a.hdr->work_next, 1u);
+        it_ring[slot] = item;
+        tc::mbar_arrive(it_full + slot);
+        if (item >= n_items) break;
         const int4 it = a.items[item];
         TileIter I;
         I.init(a, it);
-        if (itc > 0 && !tc::mbar_wait(q_empty, (itc - 1) & 1, abort_s, WAIT_NS)) {
-          ok = false;
-          break;
-        }
+        if (k > 0 && !tc::mbar_wait(q_empty, (k - 1) & 1, abort_s, WAIT_NS)) break;
         tc::mbar_expect_tx(q_full, TILE_BYTES);
         const CUtensorMap* qm = it.w >= 0 ? &tmQ : &tmQprobe;
         const int qrow = it.w >= 0 ? it.x * a.N + it.y : it.x * a.M + it.y;
@@ -162,46 +182,54 @@ __global__ void __launch_bounds__(256, 1)
         tc::tma_load_2d(sQ + BOX_BYTES, qm, 64, qrow, q_full);
         ++q_loads;
         for (; I.valid; I.next(), ++kv) {
-          const int s = kv & 1;
-          if (kv >= 2 && !tc::mbar_wait(kv_empty + s, ((kv >> 1) - 1) & 1, abort_s, WAIT_NS)) {
+          const int s = kv % NST;
+          if (kv >= NST &&
+              !tc::mbar_wait(kv_empty + s, ((kv / NST) - 1) & 1, abort_s, WAIT_NS)) {
             ok = false;
             break;
           }
+          uint8_t* kd = sKV + (size_t)(2 * s) * TILE_BYTES;
+          uint8_t* vd = kd + TILE_BYTES;
           tc::mbar_expect_tx(kv_full + s, 2 * TILE_BYTES);
           const int krow = it.x * a.N + I.t0;
-          tc::tma_load_2d(sK[s], &tmK, 0, krow, kv_full + s);
-          tc::tma_load_2d(sK[s] + BOX_BYTES, &tmK, 64, krow, kv_full + s);
-          tc::tma_load_2d(sV[s], &tmV, 0, krow, kv_full + s);
-          tc::tma_load_2d(sV[s] + BOX_BYTES, &tmV, 64, krow, kv_full + s);
+          tc::tma_load_2d(kd, &tmK, 0, krow, kv_full + s);
+          tc::tma_load_2d(kd + BOX_BYTES, &tmK, 64, krow, kv_full + s);
+          tc::tma_load_2d(vd, &tmV, 0, krow, kv_full + s);
+          tc::tma_load_2d(vd + BOX_BYTES, &tmV, 64, krow, kv_full + s);
         }
       }
       if (*abort_s) {  // let our copies in flight land before the block exits
-        for (int k = kv - 2; k < kv; ++k)
-          if (k >= 0) tc::mbar_wait_bounded(kv_full + (k & 1), (k >> 1) & 1, 100000000ull);
+        for (int k = kv - NST; k < kv; ++k)
+          if (k >= 0) tc::mbar_wait_bounded(kv_full + (k % NST), (k / NST) & 1, 100000000ull);
         if (q_loads > 0) tc::mbar_wait_bounded(q_full, (q_loads - 1) & 1, 100000000ull);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idS = tc::idesc_bf16(TBM, TBN, 0);
-      const uint32_t idPV = tc::idesc_bf16(TBM, TD, 1);
       const uint32_t q_addr = smem_u32(sQ);
-      int kv = 0, pg = 0, itc = 0;
+      int kv = 0, pg = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++itc) {
+      for (int k = 0; ok; ++k) {
+        const int slot = k % NITQ;
+        if (!tc::mbar_wait(it_full + slot, (k / NITQ) & 1, abort_s, WAIT_NS)) break;
+        const int item = it_ring[slot];
+        tc::mbar_arrive(it_empty + slot);
+        if (item >= n_items) break;
         const int4 it = a.items[item];
         TileIter Is, Ip;
         Is.init(a, it);
         Ip.init(a, it);
-        if (!tc::mbar_wait(q_full, itc & 1, abort_s, WAIT_NS)) break;
+        if (!tc::mbar_wait(q_full, k & 1, abort_s, WAIT_NS)) break;
         int kv_s = kv, sg = pg;
         auto issue_s = [&]() -> bool {
-          const int s = kv_s & 1;
-          if (!tc::mbar_wait(kv_full + s, (kv_s >> 1) & 1, abort_s, WAIT_NS)) return false;
+          const int s = kv_s % NST;
+          if (!tc::mbar_wait(kv_full + s, (kv_s / NST) & 1, abort_s, WAIT_NS)) return false;
           tc::tc_fence_after();
+          const int n16 = (Is.nvalid() + 15) & ~15;
+          const uint32_t idS = tc::idesc_bf16(TBM, n16, 0);
           const uint32_t d = tbase + ((sg & 1) ? S_COL1 : S_COL0);
-          const uint32_t k_addr = smem_u32(sK[s]);
+          const uint32_t k_addr = smem_u32(sKV + (size_t)(2 * s) * TILE_BYTES);
 #pragma unroll
           for (int ks = 0; ks < TD / 16; ++ks) {
             const uint32_t off = (ks >> 2) * BOX_BYTES + (ks & 3) * 32;
@@ -213,10 +241,11 @@ __global__ void __launch_bounds__(256, 1)
           ++sg;
           return true;
         };
-        for (int k = 0; k < 2 && Is.valid && ok; ++k) {
+        for (int j = 0; j < 2 && Is.valid && ok; ++j) {
           ok = issue_s();
           Is.next();
         }
+        const uint32_t idPV = tc::idesc_bf16(TBM, TD, 1);
         bool first = true;
         for (; Ip.valid && ok; Ip.next()) {
           const int b = pg & 1;
@@ -224,16 +253,16 @@ __global__ void __launch_bounds__(256, 1)
             ok = false;
             break;
           }
-          if (first && itc > 0 && !tc::mbar_wait(o_free, (itc - 1) & 1, abort_s, WAIT_NS)) {
+          if (first && k > 0 && !tc::mbar_wait(o_free, (k - 1) & 1, abort_s, WAIT_NS)) {
             ok = false;
             break;
           }
           tc::tc_fence_after();
-          const int s = kv & 1;
-          const uint32_t v_addr = smem_u32(sV[s]);
+          const int s = kv % NST;
+          const uint32_t v_addr = smem_u32(sKV + (size_t)(2 * s + 1) * TILE_BYTES);
           const uint32_t p_col = tbase + (b ? S_COL1 : S_COL0);
-#pragma unroll
-          for (int kk = 0; kk < TBN / 16; ++kk)
+          const int nk = (Ip.nvalid() + 15) >> 4;  // 16-key blocks holding valid keys
+          for (int kk = 0; kk < nk; ++kk)
             tc::mma_ts(tbase + O_COL, p_col + kk * 8,
                        tc::smem_desc_sw128(v_addr + kk * 2048, BOX_BYTES, 1024), idPV,
                        !(first && kk == 0));
@@ -255,20 +284,31 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int row = threadIdx.x - 128;                 // query row in the tile
+    const int row = threadIdx.x - 128;                          // query row in the tile
     const uint32_t lane_f = (uint32_t)((warp & 3) * 32) << 16;  // TMEM lane field
-    int pg = 0, pvseen = 0, itc = 0;
+    int pg = 0, pvseen = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++itc) {
+    for (int k = 0; ok; ++k) {
+      const int slot = k % NITQ;
+      const bool got_it = tc::mbar_wait(it_full + slot, (k / NITQ) & 1, abort_s, WAIT_NS);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got_it)) break;
+      const int item = it_ring[slot];
+      tc::mbar_arrive(it_empty + slot);
+      if (item >= n_items) break;
       const int4 it = a.items[item];
       TileIter I;
       I.init(a, it);
       float m = -INFINITY, l = 0.f;
       bool first = true;
       int ntiles = 0;
+      unsigned long long exec_pairs = 0;
       for (; I.valid; I.next(), ++pg, ++ntiles) {
         const int b = pg & 1;
         const uint32_t scol = tbase + lane_f + (b ? S_COL1 : S_COL0);
+        const int nvalid = I.nvalid();
+        exec_pairs += (unsigned long long)TBM * ((nvalid + 15) & ~15);
+        const int nch = (nvalid + 31) >> 5;  // 32-key chunks holding valid keys
         const bool got_s = tc::mbar_wait(s_full + b, (pg >> 1) & 1, abort_s, WAIT_NS);
         __syncwarp();  // TMEM loads and stores below are warp-collective
         if (!__all_sync(0xffffffffu, got_s)) {
@@ -278,9 +318,9 @@ __global__ void __launch_bounds__(256, 1)
         tc::tc_fence_after();
         uint32_t sr[TBN];
 #pragma unroll
-        for (int c = 0; c < TBN / 32; ++c) tc::tmem_ld32(scol + 32 * c, sr + 32 * c);
+        for (int c = 0; c < TBN / 32; ++c)
+          if (c < nch) tc::tmem_ld32(scol + 32 * c, sr + 32 * c);
         tc::tmem_wait_ld();
-        const int nvalid = min(TBN, I.run.y - I.t0);
         float mx = -INFINITY;
 #pragma unroll
         for (int c = 0; c < TBN; ++c) {
@@ -299,16 +339,18 @@ __global__ void __launch_bounds__(256, 1)
         float sum = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          uint32_t pr[32];
+          if (64 * h < nvalid) {  // uniform across the warp: one tile for all rows
+            uint32_t pr[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(__uint_as_float(sr[64 * h + 2 * c]) - m_use);
-            const float p1 = ex2(__uint_as_float(sr[64 * h + 2 * c + 1]) - m_use);
-            sum += p0 + p1;
-            pr[c] = pack_bf16(p0, p1);
+            for (int c = 0; c < 32; ++c) {
+              const float p0 = ex2(__uint_as_float(sr[64 * h + 2 * c]) - m_use);
+              const float p1 = ex2(__uint_as_float(sr[64 * h + 2 * c + 1]) - m_use);
+              sum += p0 + p1;
+              pr[c] = pack_bf16(p0, p1);
+            }
+            __syncwarp();
+            tc::tmem_st32(scol + 32 * h, pr);
           }
-          __syncwarp();
-          tc::tmem_st32(scol + 32 * h, pr);
         }
         if (!first) {  // O holds PV of the previous tile once it is done
           const bool got_o = tc::mbar_wait(o_done, pvseen & 1, abort_s, WAIT_NS);
@@ -377,8 +419,7 @@ __global__ void __launch_bounds__(256, 1)
       tc::tc_fence_before();
       tc::mbar_arrive(o_free);
       if (row == 0)
-        atomicAdd(reinterpret_cast<unsigned long long*>(&a.stats[it.x].tile_pairs),
-                  (unsigned long long)ntiles * TBN * TBM);
+        atomicAdd(reinterpret_cast<unsigned long long*>(&a.stats[it.x].tile_pairs), exec_pairs);
     }
   }
   tc::tc_fence_before();
