@@ -14,9 +14,10 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "lib", "libsparsepr.so")
 
-SPR_OK, SPR_EINVAL, SPR_EUNSUPPORTED, SPR_EWORKSPACE, SPR_ECUDA, SPR_EDEVICE = range(6)
+(SPR_OK, SPR_EINVAL, SPR_EUNSUPPORTED, SPR_EWORKSPACE, SPR_ECUDA, SPR_EDEVICE,
+ SPR_ESCRATCH) = range(7)
 STATUS_NAMES = {0: "SPR_OK", 1: "SPR_EINVAL", 2: "SPR_EUNSUPPORTED", 3: "SPR_EWORKSPACE",
-                4: "SPR_ECUDA", 5: "SPR_EDEVICE"}
+                4: "SPR_ECUDA", 5: "SPR_EDEVICE", 6: "SPR_ESCRATCH"}
 ROUTE_TAU, ROUTE_BUDGET = 0, 1
 
 VIEWS = {
@@ -57,7 +58,7 @@ class SprHeadStats(ctypes.Structure):
 EXPORTS = ["sparsepr_workspace_size", "sparsepr_check_params", "sparsepr_partition",
            "sparsepr_route", "sparsepr_attend", "sparsepr_reconstruct", "sparsepr_call",
            "sparsepr_get_stats", "sparsepr_workspace_view", "sparsepr_version",
-           "sparsepr_launch_count"]
+           "sparsepr_launch_count", "sparsepr_attend_routed_noalloc"]
 
 _lib = None
 
@@ -96,6 +97,10 @@ def load_library(path: str = LIB_PATH):
     lib.sparsepr_version.restype = ctypes.c_char_p
     lib.sparsepr_launch_count.argtypes = []
     lib.sparsepr_launch_count.restype = ctypes.c_int64
+    i32 = ctypes.c_int32
+    lib.sparsepr_attend_routed_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                                   i32, ctypes.c_float, vp, vp, vp]
+    lib.sparsepr_attend_routed_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -216,6 +221,22 @@ def workspace_tensor(prm, ws, which, dtype, shape) -> torch.Tensor:
     if n * esz > nb:
         raise ValueError(f"view {which}: {shape} exceeds {nb} bytes")
     return ws[off:off + n * esz].view(dtype).view(*shape)
+
+
+def sparsepr_attend_routed_noalloc(Qp, Kp, Vp, q_off, run_ptr, runs, Gk, O, status=None,
+                                   scale=0.0, stream=None):
+    """Routed attention without device allocation.
+
+    Qp, Kp, Vp: [BH, N, d] bf16 group-major; q_off, run_ptr: [BH, Gq + 1]
+    int32; runs: [BH, Gq * Gk, 2] int32 key ranges; O: [BH, N, d] fp32;
+    status: optional int32[4] device tensor receiving the device error word.
+    """
+    BH, N, d = Qp.shape
+    Gq = q_off.shape[1] - 1
+    _check("sparsepr_attend_routed_noalloc", load_library().sparsepr_attend_routed_noalloc(
+        Qp.data_ptr(), Kp.data_ptr(), Vp.data_ptr(), q_off.data_ptr(), run_ptr.data_ptr(),
+        runs.data_ptr(), BH, N, d, Gq, Gk, float(scale), O.data_ptr(),
+        status.data_ptr() if status is not None else None, _stream(stream)))
 
 
 def sparsepr_launch_count() -> int:

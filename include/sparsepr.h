@@ -49,7 +49,9 @@ typedef enum {
   SPR_EUNSUPPORTED = 2,  /* valid but not supported by these kernels (d, layout) */
   SPR_EWORKSPACE = 3,    /* workspace too small or misaligned */
   SPR_ECUDA = 4,         /* a CUDA runtime call failed (launch, copy) */
-  SPR_EDEVICE = 5        /* a kernel set the device error word */
+  SPR_EDEVICE = 5,       /* a kernel set the device error word */
+  SPR_ESCRATCH = 6       /* too large for the fixed scratch area of
+                            sparsepr_attend_routed_noalloc */
 } spr_status;
 
 enum { SPR_ROUTE_TAU = 0, SPR_ROUTE_BUDGET = 1 };
@@ -201,6 +203,64 @@ typedef enum {
 
 spr_status sparsepr_workspace_view(const spr_params* prm, int32_t which, size_t* offset,
                                    size_t* bytes);
+
+/*
+ * Routed attention with no device memory allocation.  The method has no
+ * counterpart to this entry point: it runs the stage-3 computation above
+ * (every row of query group i attends, softmax renormalised over the kept
+ * keys, to the key ranges routed to i [paperlayer §4 "Sparse Execution"])
+ * on group-major inputs the caller supplies, for callers that cannot
+ * allocate device memory where they run it (a launch sequence replayed
+ * with fixed addresses, a memory pool partitioned ahead of time, a thread
+ * that must not enter the allocator).  It enqueues kernels only: no
+ * cudaMalloc, cudaFree or allocating library call, ever.  Its own state (error
+ * word, work cursor, per-head counters, work list) lives in a fixed 4 MiB
+ * area of device memory inside the library image; nothing has to start at
+ * zero, since each call re-initialises that state before using it.
+ *
+ * Device pointers, caller-owned (bf16 = 16-bit bfloat, row-major):
+ *   Qp, Kp, Vp  [BH, N, d] bf16, contiguous, 16-byte aligned: queries, keys
+ *               and values of each head in group-major order (the rows of a
+ *               group adjacent; V rows follow their keys).
+ *   q_off       [BH, Gq + 1] int32: rows q_off[h][i] .. q_off[h][i+1] - 1 of
+ *               head h form query group i; 0 <= q_off[h][i] <= q_off[h][i+1]
+ *               <= N.  Rows outside every group are not written.
+ *   run_ptr     [BH, Gq + 1] int32: the key ranges of group i of head h are
+ *               entries run_ptr[h][i] .. run_ptr[h][i+1] - 1 of that head's
+ *               slice of `runs`, with 0 <= run_ptr[h][i] <= run_ptr[h][i+1]
+ *               <= Gq * Gk.
+ *   runs        [BH, Gq * Gk, 2] int32 (8-byte aligned): key range {x, y}
+ *               covers keys x .. y - 1, 0 <= x < y <= N.  Ranges of a group
+ *               should not overlap (an overlapping key counts twice).
+ *   O           [BH, N, d] fp32 (16-byte aligned): row r of group i receives
+ *               softmax(scale * q_r K_S^T) V_S over the union S of its ranges.
+ *               Rows of groups with no ranges are not written.
+ *   status      int32[4] or NULL: after the call's kernels, the device error
+ *               word and three info words (0 = no error; 1 = an index out of
+ *               range, info = {head, group, 0 q_off | 1 run_ptr | 2 a range};
+ *               2 = work list overflow; 4 = a bounded wait in the attention
+ *               kernel gave up).  On an index error nothing is computed.
+ * Sizes: BH heads (batch x heads) >= 1, N >= 1 with BH * N < 2^31, d in
+ * {64, 128}, 1 <= Gq, Gk <= 256.  scale <= 0 selects 1/sqrt(d).
+ *
+ * Limit: 256 + 80 * BH (rounded up to 256) + 16 * (BH * (ceil(N / 128) + Gq)
+ * + 1) bytes must fit in 4 MiB (e.g. 40 heads of 75,600 tokens with Gq = 256
+ * need 0.52 MiB); larger problems return SPR_ESCRATCH and enqueue nothing.
+ *
+ * The first call on each device looks up the scratch area's address and sets
+ * the attention kernel's shared-memory limit (runtime calls that may load the
+ * library's device code); make that first call before capturing a stream.
+ * All calls on one device share the one scratch area: two calls that may
+ * overlap on the GPU (different streams without ordering between them, or
+ * different host threads) race on it and both results are undefined.  Calls
+ * in one stream order are safe.  Argument errors return synchronously with
+ * nothing enqueued.
+ */
+spr_status sparsepr_attend_routed_noalloc(const void* Qp, const void* Kp, const void* Vp,
+                                          const int32_t* q_off, const int32_t* run_ptr,
+                                          const int32_t* runs, int32_t BH, int32_t N, int32_t d,
+                                          int32_t Gq, int32_t Gk, float scale, float* O,
+                                          int32_t* status, void* stream);
 
 /* Library version string (static storage). */
 const char* sparsepr_version(void);

@@ -121,3 +121,24 @@ def test_workspace_scales_with_problem(lib):
                                                       r=32, route_mode="budget"))
     assert big > 20 * small
     assert big < 8e9  # fits easily in 180 GB
+
+
+def test_noalloc_rejects_on_the_host(lib):
+    f = lib.sparsepr_attend_routed_noalloc
+    ok = dict(BH=2, N=4096, d=128, Gq=64, Gk=64)
+
+    def call(ptr=256, runs=256, O=256, status=None, **kw):
+        a = dict(ok, **kw)
+        return f(ptr, ptr, ptr, 256, 256, runs, a["BH"], a["N"], a["d"], a["Gq"], a["Gk"], 0.0, O,
+                 status, None)
+
+    assert call(ptr=None) == spr._binding.SPR_EINVAL
+    assert call(O=None) == spr._binding.SPR_EINVAL
+    assert call(Gq=0) == spr._binding.SPR_EINVAL
+    assert call(Gk=257) == spr._binding.SPR_EINVAL
+    assert call(d=96) == spr._binding.SPR_EUNSUPPORTED
+    assert call(ptr=264) == spr._binding.SPR_EUNSUPPORTED  # Q/K/V not 16-byte aligned
+    assert call(runs=260) == spr._binding.SPR_EUNSUPPORTED  # ranges not 8-byte aligned
+    # 256 + 80*BH (to 256) + 16*(BH*(ceil(N/128) + Gq) + 1) bytes must fit in 4 MiB
+    assert call(BH=64, N=1 << 20, Gq=256) == spr._binding.SPR_ESCRATCH
+    assert call(BH=40, N=75600, Gq=257) == spr._binding.SPR_EINVAL
