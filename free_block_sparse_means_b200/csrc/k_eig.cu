@@ -2,20 +2,22 @@
 // sampled-query response metric M_K [paperlayer App. B.1] and the weighted
 // probe-residual Gram matrix [paperlayer App. A.3].
 //
-// One block per matrix, everything in shared memory, fp32, following the
-// textbook route for a few eigenpairs of a dense symmetric matrix (Golub & Van
-// Loan, "Matrix Computations": Householder tridiagonalisation §8.3.1,
-// bisection on Sturm sequence counts §8.4.1, inverse iteration §7.6.1):
+// One block per matrix, fp32, following the textbook route for a few
+// eigenpairs of a dense symmetric matrix (Golub & Van Loan, "Matrix
+// Computations": Householder tridiagonalisation §8.3.1, bisection on Sturm
+// sequence counts §8.4.1, inverse iteration §7.6.1):
 //   1. A = Q T Q^T with T tridiagonal: n-2 Householder reflectors, each applied
-//      to the trailing block as a symmetric rank-2 update (3 barriers each;
-//      the matrix-vector product and the update go one warp per row).
+//      to the trailing block as a symmetric rank-2 update, with the matrix held
+//      in registers (two barriers per reflector).
 //   2. The K largest eigenvalues of T by multisection: a group of G lanes of
 //      one warp evaluates the Sturm count (number of eigenvalues below x, i.e.
 //      negative pivots of T - xI = L D L^T) at G points per step.
 //   3. Eigenvectors of T by inverse iteration on (T - lambda I) with partial
-//      pivoting, then orthonormalised in descending eigenvalue order by
-//      Cholesky QR (Y Y^T = L L^T, Y <- L^-1 Y).
-//   4. Back-transformation x = H_0 H_1 ... H_{n-3} y.
+//      pivoting (one thread per eigenvector, factors in shared memory), then
+//      orthonormalised in descending eigenvalue order by Cholesky QR
+//      (Y Y^T = L L^T, Y <- L^-1 Y).
+//   4. Back-transformation x = H_0 H_1 ... H_{n-3} y, each warp holding its
+//      vectors in registers.
 // Outputs: evals[m][k] (descending, k < K), evecs[m][row][k] (stride n), and
 // the trace of each matrix.
 #include <float.h>
@@ -25,6 +27,7 @@
 namespace spr {
 
 constexpr int EIG_THREADS = 512;
+constexpr int EIG_WARPS = EIG_THREADS / 32;
 
 template <int NN>
 __device__ int sturm_count(const float* a, const float* b2, float pivmin, float x) {
@@ -32,6 +35,7 @@ __device__ int sturm_count(const float* a, const float* b2, float pivmin, float 
   float q = a[0] - x;
   if (fabsf(q) < pivmin) q = -pivmin;
   c += q < 0.f;
+#pragma unroll 8
   for (int i = 1; i < NN; ++i) {
     q = (a[i] - x) - __fdividef(b2[i - 1], q);
     if (fabsf(q) < pivmin) q = -pivmin;
@@ -40,97 +44,248 @@ __device__ int sturm_count(const float* a, const float* b2, float pivmin, float 
   return c;
 }
 
+// Shared-memory plan (floats), all offsets multiples of 4.
 template <int NN>
-__global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K, float* evals,
+struct EigSmem {
+  static constexpr int LD = NN + 1;
+  static constexpr int TR = NN / 32;   // rows per thread block (tridiagonalisation)
+  static constexpr int TC = NN / 16;   // columns per thread block
+  static constexpr int VPAD = NN + NN / 2;  // a vector with 4 floats of padding after every 8
+  static constexpr int VH = 0;                           // NN x NN reflectors
+  static constexpr int TV = VH + NN * NN;                // ta, tb, tb2, tau, lam (NN each)
+  static constexpr int MISC = TV + 5 * NN;               // [8]
+  static constexpr int VS = MISC + 8;                    // [2][VPAD] reflector vectors
+  static constexpr int PS = VS + 2 * VPAD;               // [VPAD] p
+  static constexpr int PART = PS + VPAD;                 // [EIG_WARPS] partial p.v
+  static constexpr int Y = PART + EIG_WARPS;             // K x LD eigenvectors of T
+  static constexpr int INV = 5 * NN * 32 + NN * 8;       // inverse-iteration factors of 32 vectors
+  __host__ __device__ static int g_off(int K) { return Y + ((K * LD + 3) & ~3); }
+  __host__ __device__ static int total(int K) {
+    const int gm = K * (K + 1);
+    return g_off(K) + (gm > INV ? gm : INV);
+  }
+};
+
+template <int NN>
+__global__ void __launch_bounds__(EIG_THREADS, 1) k_eig_top(const float* Ain, int K, float* evals,
                                                         float* evecs, float* trace_out) {
-  constexpr int LD = NN + 1;
+  using S = EigSmem<NN>;
+  constexpr int LD = S::LD, TR = S::TR, TC = S::TC, VPAD = S::VPAD;
+  static_assert(TR % 2 == 0 && TC % 4 == 0 && 32 * TR == NN, "block shape");
+  auto vpad = [](int j) { return j + (j >> 3) * 4; };
   extern __shared__ __align__(16) float esm[];
-  float* A = esm;                // NN x LD; later the eigenvectors Y (K x LD)
-  float* Vh = A + NN * LD;       // NN x NN reflectors, row j = v_j (entries j+1..)
-  float* ta = Vh + NN * NN;      // diag of T
-  float* tb = ta + NN;           // off-diagonal of T (tb[i] couples i, i+1)
-  float* tb2 = tb + NN;          // tb^2
-  float* tau = tb2 + NN;         // reflector scales
-  float* lam = tau + NN;         // eigenvalues (K)
-  float* pw = lam + NN;          // p = tau A22 v
-  float* misc = pw + NN;         // [8], then the Cholesky-QR Gram matrix
+  float* Vh = esm + S::VH;  // row j = v_j (entries j+1..)
+  float* ta = esm + S::TV;  // diag of T
+  float* tb = ta + NN;      // off-diagonal of T (tb[i] couples i, i+1)
+  float* tb2 = tb + NN;     // tb^2
+  float* tau = tb2 + NN;    // reflector scales
+  float* lam = tau + NN;    // eigenvalues (K)
+  float* misc = esm + S::MISC;
+  float* vsb = esm + S::VS;
+  float* psb = esm + S::PS;
+  float* part = esm + S::PART;
+  float* Y = esm + S::Y;           // K x LD
+  float* Gr = esm + S::g_off(K);   // inverse-iteration factors, then the Cholesky-QR Gram
   const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* src = Ain + (size_t)m * NN * NN;
-  for (int e = tid; e < NN * NN; e += EIG_THREADS) {
-    const int i = e / NN, j = e % NN;
-    A[i * LD + j] = 0.5f * (src[i * NN + j] + src[j * NN + i]);
-  }
-  __syncthreads();
   if (warp == 0) {
     float t = 0.f;
-    for (int i = lane; i < NN; i += 32) t += A[i * LD + i];
+    for (int i = lane; i < NN; i += 32) t += src[i * NN + i];
     t = warp_sum(t);
     if (lane == 0 && trace_out) trace_out[m] = t;
   }
   // ---- 1. tridiagonalisation --------------------------------------------
-  for (int k = 0; k < NN - 2; ++k) {
-    const int r0 = k + 1, mlen = NN - r0;
+  // The matrix lives in registers: a warp holds 2R consecutive rows, its lane
+  // (rb, cb) the R x C block of rows row0.. and columns c0.. (16 column blocks
+  // of C).  Step k applies reflector H_k (defined by row k, equal to column k
+  // by symmetry) to the trailing rows and columns: p = t A v (row partials
+  // reduced over the 16 column-block lanes), K = t/2 p.v, w = p - K v, and
+  // A -= v w^T + w v^T, i.e. a_ij -= v_i p_j + (p_i - 2 K v_i) v_j.  Reduced
+  // rows and columns need no masking in the update: v and p are zero there.
+  // The warp owning row k+1 builds the next reflector right after its own
+  // update, so a step takes two barriers.  Vectors live in shared memory with
+  // 4 floats of padding after every 8, so that the lanes' 16-byte reads of
+  // one vector hit distinct banks.
+  {
+    const int rb = lane >> 4, cb = lane & 15;
+    const int row0 = warp * 2 * TR + rb * TR, c0 = cb * TC;
+    float a[TR][TC];
+#pragma unroll
+    for (int r = 0; r < TR; ++r)
+#pragma unroll
+      for (int c = 0; c < TC; ++c)
+        a[r][c] = 0.5f * (src[(row0 + r) * NN + c0 + c] + src[(c0 + c) * NN + row0 + r]);
+
+    // Row rk of this thread's block (rk in [0, TR); other values give row 0).
+    auto select_row = [&](int rk, float* rv) {
+#pragma unroll
+      for (int c = 0; c < TC; ++c) {
+        float x = a[0][c];
+#pragma unroll
+        for (int r = 1; r < TR; ++r) x = (rk == r) ? a[r][c] : x;
+        rv[c] = x;
+      }
+    };
+    // Reflector of step k from the current row k, given as rv by the 16 lanes
+    // of the row block that holds it (the whole warp runs this; the other row
+    // block's values are ignored).
+    auto prepare = [&](int k, float* vs, const float* rv) {
+      const int rk = k - row0;
+      float sig = 0.f, x0 = 0.f, dg = 0.f;
+#pragma unroll
+      for (int c = 0; c < TC; ++c) {
+        const int col = c0 + c;
+        sig = (col > k + 1) ? fmaf(rv[c], rv[c], sig) : sig;
+        x0 = (col == k + 1) ? rv[c] : x0;
+        dg = (col == k) ? rv[c] : dg;
+      }
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) {
+        sig += __shfl_xor_sync(0xffffffffu, sig, o);
+        x0 += __shfl_xor_sync(0xffffffffu, x0, o);
+        dg += __shfl_xor_sync(0xffffffffu, dg, o);
+      }
+      if (rk >= 0 && rk < TR) {
+        float t = 0.f, alpha = x0, v0 = 0.f;
+        if (sig > 0.f) {
+          const float nrm = sqrtf(fmaf(x0, x0, sig));
+          alpha = x0 >= 0.f ? -nrm : nrm;
+          v0 = x0 - alpha;
+          t = 2.f * __frcp_rn(fmaf(v0, v0, sig));
+        }
+#pragma unroll
+        for (int c = 0; c < TC; c += 4) {
+          float4 val;
+          float* pv4 = &val.x;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int col = c0 + c + u;
+            pv4[u] = (t == 0.f || col <= k) ? 0.f : (col == k + 1 ? v0 : rv[c + u]);
+          }
+          *reinterpret_cast<float4*>(vs + vpad(c0 + c)) = val;
+          *reinterpret_cast<float4*>(Vh + k * NN + c0 + c) = val;
+        }
+        if (cb == 0) {
+          tau[k] = t;
+          ta[k] = dg;
+          tb[k] = alpha;
+        }
+      }
+    };
+
     if (warp == 0) {
-      float sig = 0.f;
-      for (int i = r0 + 1 + lane; i < NN; i += 32) {
-        const float x = A[i * LD + k];
-        sig += x * x;
-      }
-      sig = warp_sum(sig);
-      const float x0 = A[r0 * LD + k];
-      float t = 0.f, alpha = x0, v0 = 0.f;
-      if (sig > 0.f) {
-        const float nrm = sqrtf(x0 * x0 + sig);
-        alpha = x0 >= 0.f ? -nrm : nrm;
-        v0 = x0 - alpha;
-        t = 2.f / (v0 * v0 + sig);
-      }
-      for (int i = r0 + lane; i < NN; i += 32)
-        Vh[k * NN + i] = (t == 0.f) ? 0.f : (i == r0 ? v0 : A[i * LD + k]);
-      if (lane == 0) {
-        tau[k] = t;
-        ta[k] = A[k * LD + k];
-        tb[k] = alpha;
-      }
+      float rv[TC];
+      select_row(-row0, rv);
+      prepare(0, vsb, rv);
     }
     __syncthreads();
-    const float t = tau[k];
-    if (t != 0.f) {
-      const float* v = Vh + k * NN;
-      // p = t A22 v, one thread per row; A22 is kept exactly symmetric, so the
-      // thread reads its column (consecutive threads, consecutive addresses)
-      if (tid >= r0 && tid < NN) {
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-        int j = r0;
-        for (; j + 3 < NN; j += 4) {
-          s0 += A[j * LD + tid] * v[j];
-          s1 += A[(j + 1) * LD + tid] * v[j + 1];
-          s2 += A[(j + 2) * LD + tid] * v[j + 2];
-          s3 += A[(j + 3) * LD + tid] * v[j + 3];
+    // lane -> the row whose full product it holds after the transposed reduction
+    const int rsum = (TR == 4) ? 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1) : ((lane >> 3) & 1);
+    const bool rwriter = (TR == 4) ? (lane & 3) == 0 : (lane & 7) == 0;
+    for (int k = 0; k < NN - 2; ++k) {
+      const float t = tau[k];
+      const bool owner = warp == (k + 1) / (2 * TR);
+      if (t == 0.f) {  // nothing to apply (uniform: every thread reads the same t)
+        if (owner) {
+          float rv[TC];
+          select_row(k + 1 - row0, rv);
+          prepare(k + 1, vsb + ((k + 1) & 1) * VPAD, rv);
         }
-        for (; j < NN; ++j) s0 += A[j * LD + tid] * v[j];
-        pw[tid] = t * ((s0 + s1) + (s2 + s3));
+        __syncthreads();
+        continue;
+      }
+      const float* vs = vsb + (k & 1) * VPAD;
+      // blocks whose rows or columns are all reduced skip the arithmetic
+      const bool work = row0 + TR - 1 > k && c0 + TC > k + 1;
+      float vc[TC], s[TR];
+#pragma unroll
+      for (int c = 0; c < TC; c += 4) {
+        const float4 v4 = *reinterpret_cast<const float4*>(vs + vpad(c0 + c));
+        vc[c] = v4.x;
+        vc[c + 1] = v4.y;
+        vc[c + 2] = v4.z;
+        vc[c + 3] = v4.w;
+      }
+#pragma unroll
+      for (int r = 0; r < TR; ++r) s[r] = 0.f;
+      if (work) {
+#pragma unroll
+        for (int r = 0; r < TR; ++r)
+#pragma unroll
+          for (int c = 0; c < TC; ++c) s[r] = fmaf(a[r][c], vc[c], s[r]);
+      }
+      // transposed reduction over the 16 column-block lanes: every lane ends
+      // with the full product of row row0 + rsum
+      float u;
+      if constexpr (TR == 4) {
+        const bool hi = lane & 8, mid = lane & 4;
+        const float r0 = __shfl_xor_sync(0xffffffffu, hi ? s[0] : s[2], 8);
+        const float r1 = __shfl_xor_sync(0xffffffffu, hi ? s[1] : s[3], 8);
+        const float t0 = (hi ? s[2] : s[0]) + r0, t1 = (hi ? s[3] : s[1]) + r1;
+        u = (mid ? t1 : t0) + __shfl_xor_sync(0xffffffffu, mid ? t0 : t1, 4);
+        u += __shfl_xor_sync(0xffffffffu, u, 2);
+        u += __shfl_xor_sync(0xffffffffu, u, 1);
+      } else {
+        const bool hi = lane & 8;
+        u = (hi ? s[1] : s[0]) + __shfl_xor_sync(0xffffffffu, hi ? s[0] : s[1], 8);
+        u += __shfl_xor_sync(0xffffffffu, u, 4);
+        u += __shfl_xor_sync(0xffffffffu, u, 2);
+        u += __shfl_xor_sync(0xffffffffu, u, 1);
+      }
+      {
+        const int rw = row0 + rsum;
+        const float prow = rw > k ? t * u : 0.f;
+        float pv = 0.f;
+        if (rwriter) {
+          psb[vpad(rw)] = prow;
+          pv = prow * vs[vpad(rw)];
+        }
+#pragma unroll
+        for (int o = (TR == 4 ? 4 : 8); o < 32; o <<= 1) pv += __shfl_xor_sync(0xffffffffu, pv, o);
+        if (lane == 0) part[warp] = pv;
       }
       __syncthreads();
-      float kk = 0.f;  // (t / 2) p.v, every warp for itself
-      for (int j = r0 + lane; j < NN; j += 32) kk += pw[j] * v[j];
-      kk = 0.5f * t * warp_sum(kk);
-      for (int i = r0 + warp; i < NN; i += EIG_THREADS / 32) {
-        const float vi = v[i], wi = pw[i] - kk * vi;
-        for (int j = r0 + lane; j < NN; j += 32) {
-          const float vj = v[j];
-          A[i * LD + j] -= vi * (pw[j] - kk * vj) + wi * vj;
+      float kk = 0.f;
+#pragma unroll
+      for (int w = 0; w < EIG_WARPS / 4; ++w) {
+        const float4 q4 = reinterpret_cast<const float4*>(part)[w];
+        kk += (q4.x + q4.y) + (q4.z + q4.w);
+      }
+      kk *= 0.5f * t;
+      float pc[TC], vi[TR], pi[TR];
+#pragma unroll
+      for (int c = 0; c < TC; c += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(psb + vpad(c0 + c));
+        pc[c] = p4.x;
+        pc[c + 1] = p4.y;
+        pc[c + 2] = p4.z;
+        pc[c + 3] = p4.w;
+      }
+#pragma unroll
+      for (int r = 0; r < TR; ++r) {
+        vi[r] = vs[vpad(row0 + r)];
+        pi[r] = psb[vpad(row0 + r)];
+      }
+      if (work) {
+#pragma unroll
+        for (int r = 0; r < TR; ++r) {
+          const float ci = fmaf(-2.f * kk, vi[r], pi[r]);
+#pragma unroll
+          for (int c = 0; c < TC; ++c) a[r][c] = fmaf(-vi[r], pc[c], fmaf(-ci, vc[c], a[r][c]));
         }
+      }
+      if (owner) {  // the next reflector from the updated row k+1
+        float rv[TC];
+        select_row(k + 1 - row0, rv);
+        prepare(k + 1, vsb + ((k + 1) & 1) * VPAD, rv);
       }
       __syncthreads();
     }
-  }
-  if (tid == 0) {
-    ta[NN - 2] = A[(NN - 2) * LD + NN - 2];
-    ta[NN - 1] = A[(NN - 1) * LD + NN - 1];
-    tb[NN - 2] = A[(NN - 1) * LD + NN - 2];
-    tau[NN - 2] = 0.f;
-    tb[NN - 1] = 0.f;
+    if (warp == (NN - 1) / (2 * TR)) {  // last diagonal entry
+      float rv[TC];
+      select_row(NN - 1 - row0, rv);
+      prepare(NN - 1, vsb, rv);
+    }
   }
   __syncthreads();
   for (int i = tid; i < NN; i += EIG_THREADS) tb2[i] = tb[i] * tb[i];
@@ -182,110 +337,189 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
     }
   }
   __syncthreads();
-  // ---- 3. inverse iteration (one thread per eigenvector) -----------------
-  float* Y = A;  // K x LD, reuses the reduced matrix storage
-  for (int e = tid; e < K; e += EIG_THREADS) {
-    const float l = lam[e];
-    float ud[NN], us[NN], uf[NN], ml[NN], y[NN];
-    bool pv[NN];
-    // factor T - l I with partial pivoting (rows i, i+1 at step i)
-    float g = ta[0] - l, h = tb[0];
-    for (int i = 0; i < NN - 1; ++i) {
-      const float sdn = tb[i], gn = ta[i + 1] - l, hn = (i + 1 < NN - 1) ? tb[i + 1] : 0.f;
-      if (fabsf(g) >= fabsf(sdn)) {
-        const float mult = (g != 0.f) ? __fdividef(sdn, g) : 0.f;
-        ud[i] = g;
-        us[i] = h;
-        uf[i] = 0.f;
-        ml[i] = mult;
-        pv[i] = false;
-        g = gn - mult * h;
-        h = hn;
-      } else {
-        const float mult = __fdividef(g, sdn);
-        ud[i] = sdn;
-        us[i] = gn;
-        uf[i] = hn;
-        ml[i] = mult;
-        pv[i] = true;
-        g = h - mult * gn;
-        h = -mult * hn;
-      }
-    }
-    ud[NN - 1] = g;
+  // ---- 3. inverse iteration (warp 0, one lane per eigenvector) ------------
+  // Factors of T - lambda I = P L U in shared memory, [i][lane] so that the
+  // lanes' accesses fall in distinct banks: U's diagonal (as its reciprocal),
+  // first and second superdiagonals, L's multipliers, the iterate, pivots.
+  if (warp == 0) {
+    float* rud = Gr;
+    float* us = rud + NN * 32;
+    float* uf = us + NN * 32;
+    float* ml = uf + NN * 32;
+    float* yv = ml + NN * 32;
+    uint8_t* pv = reinterpret_cast<uint8_t*>(yv + NN * 32);
     const float tiny = 1e-7f * misc[3];
-    for (int i = 0; i < NN; ++i)
-      if (fabsf(ud[i]) < tiny) ud[i] = ud[i] < 0.f ? -tiny : tiny;
-    for (int i = 0; i < NN; ++i) y[i] = 0.5f + (float)((i * 2654435761u + e * 40503u) % 1024u) / 1024.f;
-    for (int it = 0; it < 3; ++it) {
-      for (int i = 0; i < NN - 1; ++i) {  // forward: L^-1 P
-        if (pv[i]) {
-          const float t = y[i];
-          y[i] = y[i + 1];
-          y[i + 1] = t;
+    auto clamp_rcp = [&](float u) {
+      if (fabsf(u) < tiny) u = u < 0.f ? -tiny : tiny;
+      return 1.f / u;
+    };
+    for (int e0 = 0; e0 < K; e0 += 32) {
+      const int e = e0 + lane;
+      if (e < K) {
+        const float l = lam[e];
+        // factor with partial pivoting (rows i, i+1 at step i)
+        float g = ta[0] - l, h = tb[0];
+        for (int i = 0; i < NN - 1; ++i) {
+          const float sdn = tb[i], gn = ta[i + 1] - l, hn = (i + 1 < NN - 1) ? tb[i + 1] : 0.f;
+          const int o = i * 32 + lane;
+          if (fabsf(g) >= fabsf(sdn)) {
+            const float mult = (g != 0.f) ? __fdividef(sdn, g) : 0.f;
+            rud[o] = clamp_rcp(g);
+            us[o] = h;
+            uf[o] = 0.f;
+            ml[o] = mult;
+            pv[o] = 0;
+            g = gn - mult * h;
+            h = hn;
+          } else {
+            const float mult = __fdividef(g, sdn);
+            rud[o] = clamp_rcp(sdn);
+            us[o] = gn;
+            uf[o] = hn;
+            ml[o] = mult;
+            pv[o] = 1;
+            g = h - mult * gn;
+            h = -mult * hn;
+          }
         }
-        y[i + 1] -= ml[i] * y[i];
+        rud[(NN - 1) * 32 + lane] = clamp_rcp(g);
+        for (int i = 0; i < NN; ++i)
+          yv[i * 32 + lane] = 0.5f + (float)((i * 2654435761u + e * 40503u) % 1024u) / 1024.f;
+        for (int it = 0; it < 3; ++it) {
+          // forward: y <- L^-1 P y, the running entry carried in a register
+          float cur = yv[lane];
+#pragma unroll 4
+          for (int i = 0; i < NN - 1; ++i) {
+            float nxt = yv[(i + 1) * 32 + lane];
+            if (pv[i * 32 + lane]) {
+              const float t = cur;
+              cur = nxt;
+              nxt = t;
+            }
+            nxt -= ml[i * 32 + lane] * cur;
+            yv[i * 32 + lane] = cur;
+            cur = nxt;
+          }
+          // back: y <- U^-1 y, with y_{i+1}, y_{i+2} carried in registers
+          float y2 = cur * rud[(NN - 1) * 32 + lane];
+          yv[(NN - 1) * 32 + lane] = y2;
+          float y1 = (yv[(NN - 2) * 32 + lane] - us[(NN - 2) * 32 + lane] * y2) *
+                     rud[(NN - 2) * 32 + lane];
+          yv[(NN - 2) * 32 + lane] = y1;
+          float nrm = y2 * y2 + y1 * y1;
+#pragma unroll 4
+          for (int i = NN - 3; i >= 0; --i) {
+            const int o = i * 32 + lane;
+            const float yi = (yv[o] - us[o] * y1 - uf[o] * y2) * rud[o];
+            yv[o] = yi;
+            nrm += yi * yi;
+            y2 = y1;
+            y1 = yi;
+          }
+          const float inv = nrm > 0.f ? rsqrtf(nrm) : 0.f;
+          for (int i = 0; i < NN; ++i) yv[i * 32 + lane] *= inv;
+        }
+        for (int i = 0; i < NN; ++i) Y[e * LD + i] = yv[i * 32 + lane];
       }
-      y[NN - 1] = __fdividef(y[NN - 1], ud[NN - 1]);  // back: U^-1
-      y[NN - 2] = __fdividef(y[NN - 2] - us[NN - 2] * y[NN - 1], ud[NN - 2]);
-      for (int i = NN - 3; i >= 0; --i)
-        y[i] = __fdividef(y[i] - us[i] * y[i + 1] - uf[i] * y[i + 2], ud[i]);
-      float nrm = 0.f;
-      for (int i = 0; i < NN; ++i) nrm += y[i] * y[i];
-      const float inv = nrm > 0.f ? rsqrtf(nrm) : 0.f;
-      for (int i = 0; i < NN; ++i) y[i] *= inv;
+      __syncwarp();
     }
-    for (int i = 0; i < NN; ++i) Y[e * LD + i] = y[i];
   }
   __syncthreads();
   // Orthonormalise in descending eigenvalue order by Cholesky QR (the same
   // basis as Gram-Schmidt in that order): Gm = Y Y^T = L L^T, Y <- L^-1 Y.
-  float* Gm = misc + 8;  // K x (K + 1)
+  float* Gm = Gr;  // K x (K + 1), reuses the inverse-iteration storage
   const int GL = K + 1;
   for (int e = tid; e < K * K; e += EIG_THREADS) {
     const int a = e / K, b = e % K;
     if (b <= a) {
-      float s = 0.f;
-      for (int i = 0; i < NN; ++i) s += Y[a * LD + i] * Y[b * LD + i];
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < NN; i += 2) {
+        s0 = fmaf(Y[a * LD + i], Y[b * LD + i], s0);
+        s1 = fmaf(Y[a * LD + i + 1], Y[b * LD + i + 1], s1);
+      }
+      const float s = s0 + s1;
       Gm[a * GL + b] = s;
     }
   }
   __syncthreads();
-  if (warp == 0) {  // Cholesky of Gm, lanes over rows
-    for (int kq = 0; kq < K; ++kq) {
-      const float dkk = sqrtf(fmaxf(Gm[kq * GL + kq], 1e-30f));
-      __syncwarp();
-      for (int i = kq + 1 + lane; i < K; i += 32) Gm[i * GL + kq] /= dkk;
-      if (lane == 0) Gm[kq * GL + kq] = dkk;
-      __syncwarp();
-      for (int i = kq + 1 + lane; i < K; i += 32) {
-        const float lik = Gm[i * GL + kq];
-        for (int j = kq + 1; j <= i; ++j) Gm[i * GL + j] -= lik * Gm[j * GL + kq];
-      }
-      __syncwarp();
+  // Cholesky of Gm, one barrier per column: the trailing update uses the
+  // unscaled column (G_ij -= G_ik G_jk / G_kk), the scaling comes at the end.
+  for (int kq = 0; kq < K - 1; ++kq) {
+    const float rkk = 1.f / fmaxf(Gm[kq * GL + kq], 1e-30f);
+    const int nt = K - 1 - kq;  // trailing order
+    for (int e = tid; e < nt * (nt + 1) / 2; e += EIG_THREADS) {
+      int i = (int)((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);  // e -> (i, j), j <= i
+      while (i * (i + 1) / 2 > e) --i;
+      while ((i + 1) * (i + 2) / 2 <= e) ++i;
+      const int j = e - i * (i + 1) / 2;
+      const int gi = kq + 1 + i, gj = kq + 1 + j;
+      Gm[gi * GL + gj] -= Gm[gi * GL + kq] * Gm[gj * GL + kq] * rkk;
     }
+    __syncthreads();
+  }
+  for (int e = tid; e < K * K; e += EIG_THREADS) {
+    const int i = e / K, j = e % K;
+    if (j < i) Gm[i * GL + j] *= rsqrtf(fmaxf(Gm[j * GL + j], 1e-30f));
   }
   __syncthreads();
-  for (int i = tid; i < NN; i += EIG_THREADS) {  // forward substitution per column of Y
+  for (int i = tid; i < K; i += EIG_THREADS) Gm[i * GL + i] = sqrtf(fmaxf(Gm[i * GL + i], 1e-30f));
+  __syncthreads();
+  {  // Y <- L^-1 Y: TPC threads per column of Y split the sums, rows in order
+    constexpr int TPC = EIG_THREADS / NN;
+    const int col = tid / TPC, sub = tid % TPC;
     for (int a = 0; a < K; ++a) {
-      float s = Y[a * LD + i];
-      for (int b = 0; b < a; ++b) s -= Gm[a * GL + b] * Y[b * LD + i];
-      Y[a * LD + i] = s / Gm[a * GL + a];
+      float s = 0.f;
+      for (int b = sub; b < a; b += TPC) s = fmaf(Gm[a * GL + b], Y[b * LD + col], s);
+#pragma unroll
+      for (int o = 1; o < TPC; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (sub == 0) Y[a * LD + col] = (Y[a * LD + col] - s) / Gm[a * GL + a];
+      __syncwarp();
     }
   }
   __syncthreads();
-  // ---- 4. back-transformation, one warp per vector -----------------------
-  for (int kq = warp; kq < K; kq += EIG_THREADS / 32) {
-    float* y = Y + kq * LD;
-    for (int j = NN - 3; j >= 0; --j) {
-      const float t = tau[j];
-      if (t == 0.f) continue;
-      const float* v = Vh + j * NN;
-      float d = 0.f;
-      for (int i = j + 1 + lane; i < NN; i += 32) d += v[i] * y[i];
-      d = warp_sum(d) * t;
-      for (int i = j + 1 + lane; i < NN; i += 32) y[i] -= d * v[i];
-      __syncwarp();
+  // ---- 4. back-transformation: each warp takes two vectors at a time and
+  // keeps them in registers (lane holds rows lane + 32 m) ------------------
+  {
+    constexpr int RM = NN / 32;
+    for (int kq0 = warp; kq0 < K; kq0 += 2 * EIG_WARPS) {
+      const int kq1 = kq0 + EIG_WARPS;
+      const bool two = kq1 < K;
+      float y0[RM], y1[RM];
+#pragma unroll
+      for (int r = 0; r < RM; ++r) {
+        y0[r] = Y[kq0 * LD + lane + 32 * r];
+        y1[r] = two ? Y[kq1 * LD + lane + 32 * r] : 0.f;
+      }
+      for (int j = NN - 3; j >= 0; --j) {
+        const float t = tau[j];
+        if (t == 0.f) continue;
+        const float* v = Vh + j * NN;  // zero at rows <= j
+        float vr[RM], d0 = 0.f, d1 = 0.f;
+#pragma unroll
+        for (int r = 0; r < RM; ++r) {
+          vr[r] = v[lane + 32 * r];
+          d0 = fmaf(vr[r], y0[r], d0);
+          d1 = fmaf(vr[r], y1[r], d1);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          d0 += __shfl_xor_sync(0xffffffffu, d0, o);
+          d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+        }
+        d0 *= t;
+        d1 *= t;
+#pragma unroll
+        for (int r = 0; r < RM; ++r) {
+          y0[r] = fmaf(-d0, vr[r], y0[r]);
+          y1[r] = fmaf(-d1, vr[r], y1[r]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < RM; ++r) {
+        Y[kq0 * LD + lane + 32 * r] = y0[r];
+        if (two) Y[kq1 * LD + lane + 32 * r] = y1[r];
+      }
     }
   }
   __syncthreads();
@@ -299,8 +533,7 @@ __global__ void __launch_bounds__(EIG_THREADS) k_eig_top(const float* Ain, int K
 template <int NN>
 static cudaError_t eig_n(const float* A, int count, int K, float* ev, float* evec, float* trace,
                          cudaStream_t st) {
-  // A / Y, reflectors, T and scratch vectors, misc, Cholesky-QR Gram (K <= NN)
-  const size_t smem = (size_t)(NN * (NN + 1) + NN * NN + 6 * NN + 8 + NN * (NN + 1)) * 4;
+  const size_t smem = (size_t)EigSmem<NN>::total(K) * 4;
   cudaError_t e = cudaFuncSetAttribute(k_eig_top<NN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
