@@ -77,6 +77,8 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_RXBAR] = BH * 2 * d * 4;
   sz[B_PROJ] = BH * (M ? (M + 63) / 64 : 1) * d * (p->r > 0 ? p->r : 1) * 4;  // fit rhs partials
   sz[B_PART] = part_slots * 8;
+  // k-means partial sums: per chunk, one slot per (group, warp segment)
+  sz[B_CSUM] = BH * nchunk * (Gm + CSUM_SLOTS) * (d > P ? d : P) * 4;
   size_t off = 0;
   for (int i = 0; i < B_COUNT_; ++i) {
     L->off[i] = off;
@@ -153,6 +155,7 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.rxbar = AT(float*, B_RXBAR);
   P.proj = AT(float*, B_PROJ);
   P.part = AT(double*, B_PART);
+  P.csum = AT(float*, B_CSUM);
 #undef AT
   return P;
 }

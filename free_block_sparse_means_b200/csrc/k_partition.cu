@@ -159,20 +159,19 @@ __global__ void k_init_centk(const float* Z, int N, int G, int PP, const int32_t
 
 // ---------------------------------------------------------------------------
 // Key assignment in eigen-coordinates: argmin_g ||z - c_g||^2 (ties to the
-// lowest g).  One block per CHUNK rows; also the chunk's label histogram.
+// lowest g).  One block of ASG_THREADS threads per ASG_THREADS * RPT rows.
 // ---------------------------------------------------------------------------
+constexpr int ASG_THREADS = 128;
+
 template <int PP, int RPT>
-__global__ void __launch_bounds__(CHUNK / RPT) k_assign_z(const float* Z, int N, int G,
-                                                          const float* cent, int32_t* lab,
-                                                          int32_t* chunk_cnt, int nchunk) {
+__global__ void __launch_bounds__(ASG_THREADS) k_assign_z(const float* Z, int N, int G,
+                                                          const float* cent, int32_t* lab) {
   extern __shared__ __align__(16) float asm_[];
   float* C = asm_;
   float* cn = C + G * PP;
-  int* hist = reinterpret_cast<int*>(cn + G);
-  const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
-  constexpr int NT = CHUNK / RPT;
+  const int bh = blockIdx.y, tid = threadIdx.x;
+  constexpr int NT = ASG_THREADS;
   for (int e = tid; e < G * PP; e += NT) C[e] = cent[(size_t)bh * G * PP + e];
-  for (int g = tid; g < G; g += NT) hist[g] = 0;
   __syncthreads();
   for (int g = tid; g < G; g += NT) {
     float s = 0.f;
@@ -184,7 +183,7 @@ __global__ void __launch_bounds__(CHUNK / RPT) k_assign_z(const float* Z, int N,
   int n[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
-    n[r] = chunk * CHUNK + tid + r * NT;
+    n[r] = blockIdx.x * NT * RPT + tid + r * NT;
     const float4* src = reinterpret_cast<const float4*>(Z + ((size_t)bh * N + (n[r] < N ? n[r] : 0)) * PP);
 #pragma unroll
     for (int k = 0; k < PP / 4; ++k) {
@@ -227,12 +226,7 @@ __global__ void __launch_bounds__(CHUNK / RPT) k_assign_z(const float* Z, int N,
   }
 #pragma unroll
   for (int r = 0; r < RPT; ++r)
-    if (n[r] < N) {
-      lab[(size_t)bh * N + n[r]] = arg[r];
-      atomicAdd(&hist[arg[r]], 1);
-    }
-  __syncthreads();
-  for (int g = tid; g < G; g += NT) chunk_cnt[((size_t)bh * nchunk + chunk) * G + g] = hist[g];
+    if (n[r] < N) lab[(size_t)bh * N + n[r]] = arg[r];
 }
 
 // ---------------------------------------------------------------------------
@@ -405,6 +399,233 @@ __global__ void __launch_bounds__(256) k_segsum(SegArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// k-means update without a global permutation.  After an assignment pass,
+// each CHUNK-row chunk counts its labels (the histogram the final stable
+// scatter also uses), sorts its rows by label (stable: by row within a
+// label) and warp w sums the rows at sorted positions [32w, 32w + 32),
+// flushing one partial sum per group it meets into slot g + w of the chunk
+// (distinct: the groups met by warp w + 1 start where warp w's end).  The
+// reducer adds, for each group, the slots of every warp segment that holds
+// it, chunk by chunk in order, in fp64; the order of every sum is fixed, so
+// the update is deterministic.  Rows: SEG_Z rows of Z (fp32, DD wide) or
+// SEG_QSCALED rows (s / rms_n) q_n (bf16 q, DD = head dim).
+// ---------------------------------------------------------------------------
+struct ChunkSumArgs {
+  const float* Z;
+  TensorView Q;
+  const float* rms;
+  float scale;
+  const int32_t* lab;
+  int32_t* chunk_cnt;        // [BH][nchunk][G] label histogram of each chunk (out)
+  int N, G, nchunk;
+  int32_t* loff;             // [BH][nchunk][G] chunk-local group offsets (out)
+  float* part;               // [BH][nchunk][G + CSUM_SLOTS][DD] partial sums (out)
+  Header* hdr;
+};
+
+template <int MODE, int DD>
+__global__ void __launch_bounds__(CHUNK) k_chunk_sums(ChunkSumArgs a) {
+  constexpr int NV = (MODE == SEG_Z) ? (DD + 31) / 32 : DD / 32;  // values per lane
+  constexpr int UN = 8;  // rows in flight per warp (divides 32)
+  __shared__ int cnt[32][MAX_GROUPS];
+  __shared__ int loff[MAX_GROUPS];
+  __shared__ int srt[CHUNK];  // local row | label << 10, in sorted order
+  __shared__ int wsum[32];
+  const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int G = a.G;
+  const size_t cidx = (size_t)bh * a.nchunk + chunk;
+  const int n0 = chunk * CHUNK, rows = min(CHUNK, a.N - n0);
+  for (int e = tid; e < 32 * G; e += CHUNK) cnt[e / G][e % G] = 0;
+  if (tid < G) loff[tid] = 0;
+  srt[tid] = -1;  // an unfilled position (only after an index error) is skipped
+  __syncthreads();
+  int g = tid < rows ? a.lab[(size_t)bh * a.N + n0 + tid] : -1;
+  if (g >= G || g < -1) {
+    set_error(a.hdr, ERR_INDEX, 3, bh, n0 + tid);
+    g = -1;
+  }
+  if (g >= 0) atomicAdd(&loff[g], 1);  // the chunk's label histogram
+  __syncthreads();
+  {  // exclusive scan of the histogram over the groups
+    const int v = tid < G ? loff[tid] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      const int x = wsum[lane];
+      int xi = x;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, xi, o);
+        if (lane >= o) xi += t;
+      }
+      wsum[lane] = xi - x;
+    }
+    __syncthreads();
+    if (tid < G) {
+      const int lo = wsum[w] + incl - v;
+      loff[tid] = lo;
+      a.loff[cidx * G + tid] = lo;
+      a.chunk_cnt[cidx * G + tid] = v;
+    }
+  }
+  const unsigned mask = __match_any_sync(0xffffffffu, g);
+  const int rank_w = __popc(mask & ((1u << lane) - 1u));
+  if (g >= 0 && (__ffs(mask) - 1) == lane) cnt[w][g] = __popc(mask);
+  __syncthreads();
+  if (g >= 0) {
+    int before = 0;
+    for (int i = 0; i < w; ++i) before += cnt[i][g];
+    const int pos = loff[g] + before + rank_w;
+    if (pos < 0 || pos >= rows)
+      set_error(a.hdr, ERR_INDEX, 4, bh, pos);
+    else
+      srt[pos] = tid | (g << 10);
+  }
+  __syncthreads();
+  const int p0 = 32 * w, p1 = min(p0 + 32, rows);
+  if (p0 >= p1) return;
+  // lane i decodes sorted position p0 + i once; the warp then walks the 32
+  // positions in order with the row, label and scale broadcast by shuffles
+  const int e_l = p0 + lane < p1 ? srt[p0 + lane] : -1;
+  const int g_l = e_l >= 0 ? e_l >> 10 : -1;
+  const int row_l = n0 + (e_l >= 0 ? (e_l & 1023) : 0);
+  float f_l = 1.f;
+  if (MODE == SEG_QSCALED && e_l >= 0) f_l = a.scale / a.rms[(size_t)bh * a.N + row_l];
+  const float* zbase = a.Z + (size_t)bh * a.N * DD;
+  const bf16* qbase = MODE == SEG_QSCALED ? a.Q.row(bh, 0) : nullptr;
+  const int64_t qsn = a.Q.sn;
+  float* slot0 = a.part + cidx * (size_t)(G + CSUM_SLOTS) * DD;
+  float acc[NV];
+#pragma unroll
+  for (int q = 0; q < NV; ++q) acc[q] = 0.f;
+  int cur = __shfl_sync(0xffffffffu, g_l, 0);
+  auto flush = [&](int gg) {
+    if (gg < 0) return;
+    float* dst = slot0 + (size_t)(gg + w) * DD;
+    if (MODE == SEG_Z) {
+#pragma unroll
+      for (int q = 0; q < NV; ++q)
+        if (lane + 32 * q < DD) dst[lane + 32 * q] = acc[q];
+    } else {
+#pragma unroll
+      for (int q = 0; q < NV / 2; ++q)
+        reinterpret_cast<float2*>(dst)[lane + 32 * q] = make_float2(acc[2 * q], acc[2 * q + 1]);
+    }
+  };
+#pragma unroll 1
+  for (int u0 = 0; u0 < 32; u0 += UN) {
+    float v[UN][NV], fu[UN];
+    int gu[UN];
+#pragma unroll
+    for (int u = 0; u < UN; ++u) {
+      gu[u] = u0 + u < 32 ? __shfl_sync(0xffffffffu, g_l, u0 + u) : -1;
+      fu[u] = __shfl_sync(0xffffffffu, f_l, u0 + u);
+      const int row = __shfl_sync(0xffffffffu, row_l, u0 + u);
+#pragma unroll
+      for (int q = 0; q < NV; ++q) v[u][q] = 0.f;
+      if (gu[u] >= 0) {
+        if (MODE == SEG_Z) {
+          const float* src = zbase + (size_t)row * DD;
+#pragma unroll
+          for (int q = 0; q < NV; ++q)
+            if (lane + 32 * q < DD) v[u][q] = src[lane + 32 * q];
+        } else {
+          const __nv_bfloat162* src = reinterpret_cast<const __nv_bfloat162*>(qbase + row * qsn);
+#pragma unroll
+          for (int q = 0; q < NV / 2; ++q) {
+            const __nv_bfloat162 x = src[lane + 32 * q];
+            v[u][2 * q] = __low2float(x);
+            v[u][2 * q + 1] = __high2float(x);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UN; ++u) {
+      if (gu[u] < 0) continue;
+      if (gu[u] != cur) {
+        flush(cur);
+#pragma unroll
+        for (int q = 0; q < NV; ++q) acc[q] = 0.f;
+        cur = gu[u];
+      }
+#pragma unroll
+      for (int q = 0; q < NV; ++q) acc[q] = fmaf(fu[u], v[u][q], acc[q]);
+    }
+  }
+  flush(cur);
+}
+
+// Group means from the chunk partial sums.  Grid (G, BH), one thread per
+// coordinate; an empty group keeps its previous centroid.  The block first
+// lists the slots holding the group (chunk by chunk, warp segment by warp
+// segment), then every thread adds its coordinate over the list with four
+// interleaved fp64 accumulators (fixed assignment, so the order is fixed).
+template <int DD>
+__global__ void k_chunk_reduce(const float* part, const int32_t* chunk_cnt, const int32_t* loff,
+                               int G, int nchunk, float* out) {
+  extern __shared__ int cred[];  // [nchunk] counts, [nchunk] list starts, slot list
+  int* cc = cred;
+  int* cs = cred + nchunk;
+  int* list = cred + 2 * nchunk;
+  __shared__ int nlist;
+  __shared__ long long tot_s;
+  const int bh = blockIdx.y, g = blockIdx.x, i = threadIdx.x;
+  for (int c = i; c < nchunk; c += blockDim.x) {
+    const size_t idx = ((size_t)bh * nchunk + c) * G + g;
+    const int n = chunk_cnt[idx];
+    cc[c] = n;
+    cs[c] = n > 0 ? min((loff[idx] + n - 1) >> 5, CSUM_SLOTS - 1) - (loff[idx] >> 5) + 1 : 0;
+    list[c] = n > 0 ? loff[idx] >> 5 : 0;  // first warp segment, moved below
+  }
+  __syncthreads();
+  if (i == 0) {  // exclusive scan of the per-chunk slot counts, totals
+    int acc = 0;
+    long long tot = 0;
+    for (int c = 0; c < nchunk; ++c) {
+      const int k = cs[c];
+      cs[c] = acc;
+      acc += k;
+      tot += cc[c];
+    }
+    nlist = acc;
+    tot_s = tot;
+  }
+  __syncthreads();
+  // slot offsets (relative to the part buffer of this head), chunk-major
+  for (int c = i; c < nchunk; c += blockDim.x) cc[c] = cc[c] > 0 ? list[c] : -1;
+  __syncthreads();
+  int* slots = list + nchunk;
+  for (int c = i; c < nchunk; c += blockDim.x) {
+    if (cc[c] < 0) continue;
+    const int n = (c + 1 < nchunk ? cs[c + 1] : nlist) - cs[c];
+    for (int k = 0; k < n; ++k) slots[cs[c] + k] = c * (G + CSUM_SLOTS) + g + cc[c] + k;
+  }
+  __syncthreads();
+  if (i >= DD || tot_s == 0) return;
+  const float* base = part + (size_t)bh * nchunk * (G + CSUM_SLOTS) * DD + i;
+  const int n = nlist;
+  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+  int k = 0;
+  for (; k + 3 < n; k += 4) {
+    s0 += (double)base[(size_t)slots[k] * DD];
+    s1 += (double)base[(size_t)slots[k + 1] * DD];
+    s2 += (double)base[(size_t)slots[k + 2] * DD];
+    s3 += (double)base[(size_t)slots[k + 3] * DD];
+  }
+  if (k < n) s0 += (double)base[(size_t)slots[k] * DD];
+  if (k + 1 < n) s1 += (double)base[(size_t)slots[k + 1] * DD];
+  if (k + 2 < n) s2 += (double)base[(size_t)slots[k + 2] * DD];
+  out[((size_t)bh * G + g) * DD + i] = (float)(((s0 + s1) + (s2 + s3)) / (double)tot_s);
+}
+
 // Key objective with the final centroids: sum_n ||z_n - c_{lab_n}||^2 (fp64
 // partial per chunk).
 template <int PP>
@@ -524,11 +745,12 @@ __global__ void __launch_bounds__(256) k_amat(const float* Ct, int G, int D,
 //   assign: B rows = Bq_g = A a_g; score_g = (s / rms_n) q.Bq_g - beta_g;
 //           label = argmax (ties to the lowest g)  (query k-means assignment
 //           in factored form: u.m_g - ||m_g||^2 / 2 with m_g = Ctilde a_g)
-// One block per CHUNK rows (8 sub-tiles of 128), 8 warps x 16 rows.
+// One block per rows_per_cta rows (sub-tiles of 128), 8 warps x 16 rows.
 // ---------------------------------------------------------------------------
 struct RowGemmArgs {
   TensorView Q;
   int N, G, nchunk, split_rows;
+  int rows_per_cta;     // multiple of ATT_BM; CHUNK for the quadratic form
   const bf16* bsplit;   // [BH][2][split_rows][D]
   const float* beta;    // [BH][G]
   float scale;
@@ -536,7 +758,6 @@ struct RowGemmArgs {
   float* rms;
   float* un2;
   int32_t* lab;
-  int32_t* chunk_cnt;
   double* part;
   Header* hdr;
 };
@@ -550,8 +771,7 @@ __global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
   uint8_t* Blo = Bhi + NC * D * 2;
   uint8_t* Qs = Blo + NC * D * 2;
   float* betas = reinterpret_cast<float*>(Qs + ATT_BM * D * 2);
-  int* hist = reinterpret_cast<int*>(betas + MAX_GROUPS);
-  double* red = reinterpret_cast<double*>(hist + MAX_GROUPS);
+  double* red = reinterpret_cast<double*>(betas + 2 * MAX_GROUPS);
   const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
   const int nrows_b = QUAD ? D : a.G;
@@ -568,14 +788,11 @@ __global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
     *reinterpret_cast<uint4*>(Blo + swz<CH>(r, c)) = lo;
   }
   if (!QUAD)
-    for (int g = tid; g < MAX_GROUPS; g += 256) {
-      betas[g] = g < a.G ? a.beta[(size_t)bh * a.G + g] : 0.f;
-      hist[g] = 0;
-    }
+    for (int g = tid; g < MAX_GROUPS; g += 256) betas[g] = g < a.G ? a.beta[(size_t)bh * a.G + g] : 0.f;
   const float gk = QUAD ? (float)max(1, a.stats[bh].gk_nonempty) : 1.f;
   double un2acc = 0.0;
-  for (int sub = 0; sub < CHUNK / ATT_BM; ++sub) {
-    const int row0 = chunk * CHUNK + sub * ATT_BM;
+  for (int sub = 0; sub < a.rows_per_cta / ATT_BM; ++sub) {
+    const int row0 = chunk * a.rows_per_cta + sub * ATT_BM;
     if (row0 >= a.N) break;
     __syncthreads();  // previous tile consumed
     for (int e = tid; e < ATT_BM * CH; e += 256) {
@@ -682,14 +899,8 @@ __global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
         if (bhv > best_hi || (bhv == best_hi && ah < arg_hi)) { best_hi = bhv; arg_hi = ah; }
       }
       if (tig == 0) {
-        if (r_lo < a.N) {
-          a.lab[(size_t)bh * a.N + r_lo] = arg_lo;
-          atomicAdd(&hist[arg_lo], 1);
-        }
-        if (r_hi < a.N) {
-          a.lab[(size_t)bh * a.N + r_hi] = arg_hi;
-          atomicAdd(&hist[arg_hi], 1);
-        }
+        if (r_lo < a.N) a.lab[(size_t)bh * a.N + r_lo] = arg_lo;
+        if (r_hi < a.N) a.lab[(size_t)bh * a.N + r_hi] = arg_hi;
       }
     }
   }
@@ -703,9 +914,6 @@ __global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
       for (int i = 0; i < 8; ++i) s += red[i];
       a.part[((size_t)bh * 2 + 1) * (a.nchunk + 1) + chunk] = s;
     }
-  } else {
-    for (int g = tid; g < a.G; g += 256)
-      a.chunk_cnt[((size_t)bh * a.nchunk + chunk) * a.G + g] = hist[g];
   }
 }
 
@@ -769,32 +977,42 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
   spr_launch(k_init_centk, BH, 256, 0, st, P.Z, N, p.Gk, pp, P.initk, P.centk);
   // Key k-means
-  const size_t asmem = (size_t)p.Gk * pp * 4 + p.Gk * 4 + p.Gk * 4;
+  const size_t asmem = (size_t)p.Gk * pp * 4 + p.Gk * 4;
   for (int it = 0; it < p.iters; ++it) {
 #define ASG(PPV, RPT)                                                                      \
   do {                                                                                     \
     cudaFuncSetAttribute(k_assign_z<PPV, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                          (int)asmem);                                                      \
-    spr_launch(k_assign_z<PPV, RPT>, dim3(nchunk, BH), CHUNK / RPT, asmem, st,                     \
-        P.Z, N, p.Gk, P.centk, P.labk, P.chunk, nchunk);                                   \
+    const int rows_b = ASG_THREADS * (RPT);                                                \
+    spr_launch(k_assign_z<PPV, RPT>, dim3((N + rows_b - 1) / rows_b, BH), ASG_THREADS, asmem, \
+               st, P.Z, N, p.Gk, P.centk, P.labk);                                         \
   } while (0)
     if (pp == 8) ASG(8, 4); else if (pp == 16) ASG(16, 4); else if (pp == 32) ASG(32, 2); else ASG(64, 1);
 #undef ASG
-    spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gk, N, P.cbase, P.kvoff, P.counts);
-    spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labk, N, p.Gk, nchunk, P.cbase, P.kvoff,
-                                                 P.permk, P.hdr);
-    SegArgs sa{};
-    sa.Z = P.Z;
-    sa.perm = P.permk;
-    sa.off = P.kvoff;
-    sa.N = N;
-    sa.G = p.Gk;
-    sa.out = P.centk;
-    sa.keep_empty = 1;
-#define SEGZ(PPV) spr_launch(k_segsum<SEG_Z, PPV>, dim3(p.Gk, BH), 256, 0, st, sa)
-    if (pp == 8) SEGZ(8); else if (pp == 16) SEGZ(16); else if (pp == 32) SEGZ(32); else SEGZ(64);
-#undef SEGZ
+    ChunkSumArgs ca{};
+    ca.Z = P.Z;
+    ca.lab = P.labk;
+    ca.chunk_cnt = P.chunk;
+    ca.N = N;
+    ca.G = p.Gk;
+    ca.nchunk = nchunk;
+    ca.loff = P.cbase;
+    ca.part = P.csum;
+    ca.hdr = P.hdr;
+    const size_t rsm = (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int);
+#define KSUM(PPV)                                                                            \
+  do {                                                                                       \
+    spr_launch(k_chunk_sums<SEG_Z, PPV>, dim3(nchunk, BH), CHUNK, 0, st, ca);                \
+    spr_launch(k_chunk_reduce<PPV>, dim3(p.Gk, BH), ((PPV) + 31) / 32 * 32, rsm, st, P.csum, \
+               P.chunk, P.cbase, p.Gk, nchunk, P.centk);                                     \
+  } while (0)
+    if (pp == 8) KSUM(8); else if (pp == 16) KSUM(16); else if (pp == 32) KSUM(32); else KSUM(64);
+#undef KSUM
   }
+  // group-major key order of the final labels
+  spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gk, N, P.cbase, P.kvoff, P.counts);
+  spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labk, N, p.Gk, nchunk, P.cbase, P.kvoff,
+             P.permk, P.hdr);
 #define OBJZ(PPV) \
   spr_launch(k_obj_z<PPV>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.labk, nchunk, P.part)
   if (pp == 8) OBJZ(8); else if (pp == 16) OBJZ(16); else if (pp == 32) OBJZ(32); else OBJZ(64);
@@ -832,7 +1050,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   ra.rms = P.rms;
   ra.un2 = P.un2;
   ra.lab = P.labq;
-  ra.chunk_cnt = P.chunk;
+  ra.rows_per_cta = CHUNK;
   ra.part = P.part;
   ra.hdr = P.hdr;
   {
@@ -848,22 +1066,29 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   for (int it = 0; it < p.iters; ++it) {
     spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
                                           split_rows, nullptr);
-    spr_launch(k_rowgemm<D, false>, dim3(nchunk, BH), 256, smq, st, ra);
-    spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gq, N, P.cbase, P.qoff, P.counts);
-    spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labq, N, p.Gq, nchunk, P.cbase, P.qoff,
-                                                 P.permq, P.hdr);
-    SegArgs sa{};
-    sa.Q = Q;
-    sa.rms = P.rms;
-    sa.scale = scale;
-    sa.perm = P.permq;
-    sa.off = P.qoff;
-    sa.N = N;
-    sa.G = p.Gq;
-    sa.out = P.centq;
-    sa.keep_empty = 1;
-    spr_launch(k_segsum<SEG_QSCALED, D>, dim3(p.Gq, BH), 256, 0, st, sa);
+    RowGemmArgs rq = ra;
+    rq.rows_per_cta = 2 * ATT_BM;
+    spr_launch(k_rowgemm<D, false>, dim3((N + 2 * ATT_BM - 1) / (2 * ATT_BM), BH), 256, smq, st, rq);
+    ChunkSumArgs ca{};
+    ca.Q = Q;
+    ca.rms = P.rms;
+    ca.scale = scale;
+    ca.lab = P.labq;
+    ca.chunk_cnt = P.chunk;
+    ca.N = N;
+    ca.G = p.Gq;
+    ca.nchunk = nchunk;
+    ca.loff = P.cbase;
+    ca.part = P.csum;
+    ca.hdr = P.hdr;
+    spr_launch(k_chunk_sums<SEG_QSCALED, D>, dim3(nchunk, BH), CHUNK, 0, st, ca);
+    spr_launch(k_chunk_reduce<D>, dim3(p.Gq, BH), D, (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int), st, P.csum,
+               P.chunk, P.cbase, p.Gq, nchunk, P.centq);
   }
+  // group-major query order of the final labels
+  spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gq, N, P.cbase, P.qoff, P.counts);
+  spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labq, N, p.Gq, nchunk, P.cbase, P.qoff,
+             P.permq, P.hdr);
   // objective terms n_g a_g^T A a_g with the final centroids (into part's tail)
   spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
                                         split_rows, P.part + (size_t)BH * 2 * (nchunk + 1));
