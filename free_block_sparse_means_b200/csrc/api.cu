@@ -79,6 +79,10 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_PART] = part_slots * 8;
   // k-means partial sums: per chunk, one slot per (group, warp segment)
   sz[B_CSUM] = BH * nchunk * (Gm + CSUM_SLOTS) * (d > P ? d : P) * 4;
+  // probe rows gathered for the fit: sparse outputs X, residuals R, block means
+  sz[B_XP] = BH * (M ? M : 1) * d * 4;
+  sz[B_RP] = BH * (M ? M : 1) * d * 4;
+  sz[B_PMEAN] = BH * (M ? (M + 31) / 32 : 1) * 2 * d * 4;
   size_t off = 0;
   for (int i = 0; i < B_COUNT_; ++i) {
     L->off[i] = off;
@@ -156,6 +160,9 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.proj = AT(float*, B_PROJ);
   P.part = AT(double*, B_PART);
   P.csum = AT(float*, B_CSUM);
+  P.xp = AT(float*, B_XP);
+  P.rp = AT(float*, B_RP);
+  P.pmean = AT(float*, B_PMEAN);
 #undef AT
   return P;
 }

@@ -35,7 +35,7 @@ enum Buf : int {
   B_KP, B_VP, B_QP, B_CRAW, B_CT, B_AMAT, B_RMS, B_UN2, B_CENTQ, B_BQ16, B_BETA,
   B_QBAR, B_LOGIT, B_ENTRY, B_TOP, B_SEL, B_ROWPTR, B_COLIDX, B_RUNPTR, B_RUNS, B_PPOS,
   B_PIDX, B_PW, B_PSLOT, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
-  B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_CSUM, B_COUNT_
+  B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_CSUM, B_XP, B_RP, B_PMEAN, B_COUNT_
 };
 
 struct Layout {
@@ -64,7 +64,7 @@ struct Ptrs {
   spr_head_stats* stats;
   float *MK, *trace, *eval, *evec, *W, *Z, *centk, *Craw, *Ct, *Amat, *rms, *un2, *centq, *beta,
       *qbar, *logit, *entry, *pw, *osp, *odn, *fitU, *fitB, *fitBv, *gram, *axx, *rxbar,
-      *proj, *csum;
+      *proj, *csum, *xp, *rp, *pmean;
   double* part;
   int32_t *initk, *initq, *labk, *labq, *chunk, *cbase, *counts, *permk, *kvoff, *permq,
       *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx, *pslot;
