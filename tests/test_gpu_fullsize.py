@@ -1,0 +1,37 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times (every head of the call in one launch sequence), checked on
+sampled heads and, for the long sequences, on sampled rows.
+
+  mid      24 heads x 8192 tokens (the benchmark workload): three whole heads
+  hunyuan  24 heads x 118,800 tokens: two heads, 2048 sampled rows each
+  wan      40 heads x 75,600 tokens: one head, 2048 sampled rows
+The oracle runs driven by the GPU's cluster labels (see gpu_support).
+"""
+import numpy as np
+import pytest
+
+from gpu_support import check_head, run_gpu
+from synthetic import workload
+
+pytestmark = pytest.mark.gpu
+
+
+def test_mid_benchmark_launch_sampled_heads():
+    wl = workload("mid")
+    check = [0, 11, 23]
+    g = run_gpu(wl, check=check)
+    for bh in check:
+        check_head(g, wl, bh)
+    for st in g["stats"]:
+        assert 0.2 < st["rho_exec"] <= 0.25 + 1e-9, st["rho_exec"]
+
+
+@pytest.mark.parametrize("name,check", [("hunyuan", [0, 17]), ("wan", [29])])
+def test_long_sequences_sampled_rows(name, check):
+    wl = workload(name)
+    g = run_gpu(wl, check=check)
+    rows = np.sort(np.random.default_rng(7).choice(wl.N, 2048, replace=False))
+    for bh in check:
+        check_head(g, wl, bh, rows=rows)
+    for st in g["stats"]:
+        assert st["rho_exec"] <= 0.25 + 1e-9, st["rho_exec"]
