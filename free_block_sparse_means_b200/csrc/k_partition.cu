@@ -265,13 +265,13 @@ __global__ void __launch_bounds__(256) k_chunk_scan(const int32_t* chunk_cnt, in
 
 // Stable scatter: perm[off[g] + chunk base + rank among equal labels before
 // this row in the chunk] = row.
-__global__ void __launch_bounds__(1024) k_scatter(const int32_t* lab, int N, int G, int nchunk,
+__global__ void __launch_bounds__(CHUNK) k_scatter(const int32_t* lab, int N, int G, int nchunk,
                                                   const int32_t* cbase, const int32_t* off,
                                                   int32_t* perm, Header* hdr) {
   __shared__ int cnt[32][MAX_GROUPS];
   const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < 32 * G; e += 1024) cnt[e / G][e % G] = 0;
+  for (int e = tid; e < 32 * G; e += CHUNK) cnt[e / G][e % G] = 0;
   __syncthreads();
   const int n = chunk * CHUNK + tid;
   int g = n < N ? lab[(size_t)bh * N + n] : -1;
@@ -977,41 +977,29 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
   spr_launch(k_init_centk, BH, 256, 0, st, P.Z, N, p.Gk, pp, P.initk, P.centk);
   // Key k-means
-  const size_t asmem = (size_t)p.Gk * pp * 4 + p.Gk * 4;
   for (int it = 0; it < p.iters; ++it) {
-#define ASG(PPV, RPT)                                                                      \
-  do {                                                                                     \
-    cudaFuncSetAttribute(k_assign_z<PPV, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                         (int)asmem);                                                      \
-    const int rows_b = ASG_THREADS * (RPT);                                                \
-    spr_launch(k_assign_z<PPV, RPT>, dim3((N + rows_b - 1) / rows_b, BH), ASG_THREADS, asmem, \
-               st, P.Z, N, p.Gk, P.centk, P.labk);                                         \
-  } while (0)
-    if (pp == 8) ASG(8, 4); else if (pp == 16) ASG(16, 4); else if (pp == 32) ASG(32, 2); else ASG(64, 1);
-#undef ASG
-    ChunkSumArgs ca{};
-    ca.Z = P.Z;
-    ca.lab = P.labk;
-    ca.chunk_cnt = P.chunk;
-    ca.N = N;
-    ca.G = p.Gk;
-    ca.nchunk = nchunk;
-    ca.loff = P.cbase;
-    ca.part = P.csum;
-    ca.hdr = P.hdr;
+    KmArgs ka{};
+    ka.Z = P.Z;
+    ka.cent = P.centk;
+    ka.N = N;
+    ka.G = p.Gk;
+    ka.nchunk = nchunk;
+    ka.lab = P.labk;
+    ka.chunk_cnt = P.chunk;
+    ka.loff = P.cbase;
+    ka.part = P.csum;
+    ka.hdr = P.hdr;
+    if ((e = launch_kmeans_step(KM_KEY, pp, ka, nchunk, BH, st)) != cudaSuccess) return e;
     const size_t rsm = (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int);
-#define KSUM(PPV)                                                                            \
-  do {                                                                                       \
-    spr_launch(k_chunk_sums<SEG_Z, PPV>, dim3(nchunk, BH), CHUNK, 0, st, ca);                \
-    spr_launch(k_chunk_reduce<PPV>, dim3(p.Gk, BH), ((PPV) + 31) / 32 * 32, rsm, st, P.csum, \
-               P.chunk, P.cbase, p.Gk, nchunk, P.centk);                                     \
-  } while (0)
-    if (pp == 8) KSUM(8); else if (pp == 16) KSUM(16); else if (pp == 32) KSUM(32); else KSUM(64);
-#undef KSUM
+#define KRED(PPV)                                                                             \
+  spr_launch(k_chunk_reduce<PPV>, dim3(p.Gk, BH), ((PPV) + 31) / 32 * 32, rsm, st, P.csum, \
+             P.chunk, P.cbase, p.Gk, nchunk, P.centk)
+    if (pp == 8) KRED(8); else if (pp == 16) KRED(16); else if (pp == 32) KRED(32); else KRED(64);
+#undef KRED
   }
   // group-major key order of the final labels
   spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gk, N, P.cbase, P.kvoff, P.counts);
-  spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labk, N, p.Gk, nchunk, P.cbase, P.kvoff,
+  spr_launch(k_scatter, dim3(nchunk, BH), CHUNK, 0, st, P.labk, N, p.Gk, nchunk, P.cbase, P.kvoff,
              P.permk, P.hdr);
 #define OBJZ(PPV) \
   spr_launch(k_obj_z<PPV>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.labk, nchunk, P.part)
@@ -1066,28 +1054,28 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   for (int it = 0; it < p.iters; ++it) {
     spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
                                           split_rows, nullptr);
-    RowGemmArgs rq = ra;
-    rq.rows_per_cta = 2 * ATT_BM;
-    spr_launch(k_rowgemm<D, false>, dim3((N + 2 * ATT_BM - 1) / (2 * ATT_BM), BH), 256, smq, st, rq);
-    ChunkSumArgs ca{};
-    ca.Q = Q;
-    ca.rms = P.rms;
-    ca.scale = scale;
-    ca.lab = P.labq;
-    ca.chunk_cnt = P.chunk;
-    ca.N = N;
-    ca.G = p.Gq;
-    ca.nchunk = nchunk;
-    ca.loff = P.cbase;
-    ca.part = P.csum;
-    ca.hdr = P.hdr;
-    spr_launch(k_chunk_sums<SEG_QSCALED, D>, dim3(nchunk, BH), CHUNK, 0, st, ca);
+    KmArgs qa{};
+    qa.Q = Q;
+    qa.rms = P.rms;
+    qa.scale = scale;
+    qa.bsplit = P.bq16;
+    qa.split_rows = split_rows;
+    qa.beta = P.beta;
+    qa.N = N;
+    qa.G = p.Gq;
+    qa.nchunk = nchunk;
+    qa.lab = P.labq;
+    qa.chunk_cnt = P.chunk;
+    qa.loff = P.cbase;
+    qa.part = P.csum;
+    qa.hdr = P.hdr;
+    if ((e = launch_kmeans_step(KM_QUERY, D, qa, nchunk, BH, st)) != cudaSuccess) return e;
     spr_launch(k_chunk_reduce<D>, dim3(p.Gq, BH), D, (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int), st, P.csum,
                P.chunk, P.cbase, p.Gq, nchunk, P.centq);
   }
   // group-major query order of the final labels
   spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gq, N, P.cbase, P.qoff, P.counts);
-  spr_launch(k_scatter, dim3(nchunk, BH), 1024, 0, st, P.labq, N, p.Gq, nchunk, P.cbase, P.qoff,
+  spr_launch(k_scatter, dim3(nchunk, BH), CHUNK, 0, st, P.labq, N, p.Gq, nchunk, P.cbase, P.qoff,
              P.permq, P.hdr);
   // objective terms n_g a_g^T A a_g with the final centroids (into part's tail)
   spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,

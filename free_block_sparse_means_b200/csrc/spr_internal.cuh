@@ -12,7 +12,7 @@ namespace spr {
 
 typedef __nv_bfloat16 bf16;
 
-constexpr int CHUNK = 1024;        // rows per histogram chunk (k-means, permutation)
+constexpr int CHUNK = 512;         // rows per histogram chunk (k-means, permutation)
 constexpr int MAX_GROUPS = 256;    // Gk, Gq upper bound
 constexpr int MAX_P = 64;          // eigen-coordinate upper bound
 constexpr int MAX_PROBES = 4096;   // M upper bound
@@ -105,6 +105,29 @@ cudaError_t launch_reconstruct(const spr_params& p, const Layout& L, const Ptrs&
 cudaError_t launch_eig(const float* A, int count, int n, int K, float* evals, float* evecs,
                        float* trace, cudaStream_t st);
 int num_sms();
+
+// One fused Lloyd iteration (assignment, chunk histogram and sort, segmented
+// partial sums) of the query (KM_QUERY, width = d) or key (KM_KEY, width =
+// padded eigen-coordinate count) k-means; grid (nchunk, BH).
+enum { KM_QUERY = 0, KM_KEY = 1 };
+struct KmArgs {
+  TensorView Q;           // query rows
+  const float* Z;         // key rows [BH][N][width]
+  const float* rms;       // query row RMS; the update rows are (scale / rms) q
+  float scale;
+  const bf16* bsplit;     // query: [BH][2][split_rows][d] bf16 hi, lo of Bq_g
+  int split_rows;
+  const float* beta;      // query: [BH][G]
+  const float* cent;      // key: [BH][G][width] centroids
+  int N, G, nchunk;
+  int32_t* lab;           // [BH][N] labels (out)
+  int32_t* chunk_cnt;     // [BH][nchunk][G] chunk label histograms (out)
+  int32_t* loff;          // [BH][nchunk][G] chunk-local group offsets (out)
+  float* part;            // [BH][nchunk][G + CSUM_SLOTS][width] partial sums (out)
+  Header* hdr;
+};
+cudaError_t launch_kmeans_step(int mode, int width, const KmArgs& a, int nchunk, int BH,
+                               cudaStream_t st);
 
 // Every kernel launch of the library goes through spr_launch, which counts it
 // (sparsepr_launch_count reports the total).
