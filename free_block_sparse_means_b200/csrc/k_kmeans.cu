@@ -1,7 +1,9 @@
 // One Lloyd iteration of the partition's two k-means [paperlayer App. B.1,
 // B.2] on a chunk of CHUNK rows, fused into one kernel:
-//   1. assignment on the tensor cores (mma.sync m16n8k16 bf16, fp32
-//      accumulation), tiles of 128 rows double-buffered in shared memory;
+//   1. assignment on the tensor cores (tcgen05.mma kind::f16, bf16 operands
+//      in K-major 128-byte-swizzled shared memory, fp32 accumulator of 128
+//      rows x NC groups in TMEM), tiles of 128 rows double-buffered with
+//      cp.async; one thread per row reads its scores back for the argmax;
 //        query rows: score_g = (s / rms_n) q . Bq_g - beta_g, q exact in bf16,
 //                    Bq_g split into bf16 hi + lo (two products);
 //        key rows:   score_g = 2 z . c_g - ||c_g||^2, z and c_g both split
@@ -17,53 +19,107 @@
 #include <float.h>
 
 #include "spr_internal.cuh"
+#include "tc_sm100.cuh"
 
 namespace spr {
 
 constexpr int KM_THREADS = 256;
-constexpr int KM_TILE = 128;  // rows per sub-tile: 8 warps x 16
+constexpr int KM_TILE = 128;                 // rows per sub-tile (the UMMA M)
+constexpr uint32_t KM_BOX = KM_TILE * 128;   // one 64-column SW128 box of a tile: 16 KB
+constexpr uint64_t KM_WAIT_NS = 2000000000ull;
 
-__host__ __device__ constexpr int km_rs(int DK) { return DK * 2 + 16; }  // padded bf16 row (bytes)
+// Shared-memory plan (bytes from a 1024-aligned base):
+//   Bh, Bl     centroid operand, K-major SW128, nbox boxes of NC rows x 128 B
+//   A region   QUERY: two tiles of nbox boxes; KEY: two raw fp32 tiles, then
+//              the hi / lo bf16 tiles (one box each); reused afterwards by
+//              the sort arrays and the segment staging
+//   betas[MAX_GROUPS], labs[CHUNK], mbarrier, TMEM base, abort flag
+struct KmPlan {
+  int nbox, NC;
+  size_t b_off, a_off, a_size, tail_off, total;
+};
+__host__ __device__ inline KmPlan km_plan(int mode, int DK, int SW, int G) {
+  KmPlan p;
+  p.nbox = DK > 64 ? DK / 64 : 1;
+  p.NC = ((G + 31) / 32) * 32;
+  const size_t sb = (size_t)p.nbox * p.NC * 128;
+  p.b_off = 0;
+  p.a_off = 2 * sb;
+  const size_t tiles = mode == KM_KEY ? 2 * (size_t)KM_TILE * SW * 4 + 2 * (size_t)KM_BOX
+                                      : 2 * (size_t)p.nbox * KM_BOX;
+  const size_t rb = mode == KM_KEY ? (size_t)SW * 4 : (size_t)SW * 2;
+  const size_t stg = (size_t)(KM_THREADS / 32) * (mode == KM_KEY ? 32 : 16) * rb;
+  const size_t sortb = (32 * (size_t)G + CHUNK + MAX_GROUPS + 32) * 4 + stg;
+  p.a_size = ((tiles > sortb ? tiles : sortb) + 1023) & ~(size_t)1023;
+  p.tail_off = p.a_off + p.a_size;
+  p.total = p.tail_off + (MAX_GROUPS + CHUNK) * 4 + 64;
+  return p;
+}
+
+// 16-byte chunk c (K-major: K elements 8c .. 8c + 7) of row r in a tile or
+// operand of nbox 64-column SW128 boxes of `rows` rows.
+__device__ __forceinline__ uint32_t sw_off(int r, int c, int rows) {
+  return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint4 split8(const float* v, bool lo) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bf16 h0 = __float2bfloat16_rn(v[2 * i]), h1 = __float2bfloat16_rn(v[2 * i + 1]);
+    w[i] = lo ? pack_bf16(v[2 * i] - __bfloat162float(h0), v[2 * i + 1] - __bfloat162float(h1))
+              : pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 template <int MODE, int DK, int SW>
-__global__ void __launch_bounds__(KM_THREADS) k_kmeans_step(KmArgs a) {
-  constexpr int RS = km_rs(DK);
-  constexpr int NA = (MODE == KM_KEY) ? 2 : 1;  // A tiles: hi (and lo)
-  constexpr int KS = DK / 16;                    // k-steps
-  extern __shared__ __align__(128) uint8_t km[];
-  const int G = a.G, NC = ((G + 31) / 32) * 32;
-  uint8_t* Bh = km;
-  uint8_t* Bl = Bh + NC * RS;
-  float* betas = reinterpret_cast<float*>(Bl + NC * RS);
+__global__ void __launch_bounds__(KM_THREADS, 1) k_kmeans_step(KmArgs a) {
+  constexpr int KS = DK / 16;  // UMMA k-steps
+  constexpr int NCH = DK / 8;  // 16-byte chunks per A / B row
+  extern __shared__ uint8_t km_raw[];
+  uint8_t* km = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(km_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const int G = a.G;
+  const KmPlan pl = km_plan(MODE, DK, SW, G);
+  const int NC = pl.NC;
+  uint8_t* Bh = km + pl.b_off;
+  uint8_t* Bl = Bh + (size_t)pl.nbox * NC * 128;
+  uint8_t* Ab = km + pl.a_off;
+  float* betas = reinterpret_cast<float*>(km + pl.tail_off);
   int* labs = reinterpret_cast<int*>(betas + MAX_GROUPS);
-  uint8_t* Ab = reinterpret_cast<uint8_t*>(labs + CHUNK);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(labs + CHUNK);
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(mbar + 1);
+  volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_s + 1);
   const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
+  const int warp = tid >> 5, lane = tid & 31;
   const int N = a.N, n0 = chunk * CHUNK, rows = min(CHUNK, N - n0);
+  const uint32_t tcols = NC <= 32 ? 32 : NC <= 64 ? 64 : NC <= 128 ? 128 : 256;
 
-  // ---- centroid operand -------------------------------------------------
+  // ---- centroid operand (K-major SW128, bf16 hi and lo) -------------------
   if (MODE == KM_QUERY) {
     const bf16* bsrc = a.bsplit + (size_t)bh * 2 * a.split_rows * DK;
-    for (int e = tid; e < NC * (DK / 8); e += KM_THREADS) {
-      const int r = e / (DK / 8), c = e % (DK / 8);
+    for (int e = tid; e < NC * NCH; e += KM_THREADS) {
+      const int r = e / NCH, c = e % NCH;
       uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
       if (r < G) {
         hi = reinterpret_cast<const uint4*>(bsrc + (size_t)r * DK)[c];
         lo = reinterpret_cast<const uint4*>(bsrc + ((size_t)a.split_rows + r) * DK)[c];
       }
-      *reinterpret_cast<uint4*>(Bh + r * RS + c * 16) = hi;
-      *reinterpret_cast<uint4*>(Bl + r * RS + c * 16) = lo;
+      *reinterpret_cast<uint4*>(Bh + sw_off(r, c, NC)) = hi;
+      *reinterpret_cast<uint4*>(Bl + sw_off(r, c, NC)) = lo;
     }
     for (int g = tid; g < MAX_GROUPS; g += KM_THREADS)
       betas[g] = g < G ? a.beta[(size_t)bh * G + g] : 0.f;
   } else {
     const float* cs = a.cent + (size_t)bh * G * SW;
-    for (int e = tid; e < NC * DK; e += KM_THREADS) {
-      const int r = e / DK, c = e % DK;
-      const float v = (r < G && c < SW) ? cs[r * SW + c] : 0.f;
-      const bf16 hi = __float2bfloat16_rn(v);
-      reinterpret_cast<bf16*>(Bh + r * RS)[c] = hi;
-      reinterpret_cast<bf16*>(Bl + r * RS)[c] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    for (int e = tid; e < NC * NCH; e += KM_THREADS) {
+      const int r = e / NCH, c = e % NCH;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = (r < G && 8 * c + i < SW) ? cs[r * SW + 8 * c + i] : 0.f;
+      *reinterpret_cast<uint4*>(Bh + sw_off(r, c, NC)) = split8(v, false);
+      *reinterpret_cast<uint4*>(Bl + sw_off(r, c, NC)) = split8(v, true);
     }
     for (int g = tid; g < MAX_GROUPS; g += KM_THREADS) {
       float s = 0.f;
@@ -72,20 +128,34 @@ __global__ void __launch_bounds__(KM_THREADS) k_kmeans_step(KmArgs a) {
       betas[g] = s;
     }
   }
+  if (tid == 0) {
+    tc::mbar_init(mbar, 1);
+    *abort_s = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tmem_s, tcols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_proxy_async_smem();
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = *tmem_s;
 
-  // ---- assignment -------------------------------------------------------
-  // QUERY: A tiles [2][KM_TILE][RS] loaded with cp.async.
+  // ---- assignment on the tensor cores ------------------------------------
+  // QUERY: A tiles [2][nbox boxes] loaded with cp.async into the SW128 layout.
   // KEY:   raw fp32 tiles [2][KM_TILE][SW] with cp.async, converted into the
-  //        hi / lo bf16 tiles Ah, Al [KM_TILE][RS] before each use.
+  //        hi / lo bf16 tiles (one box each) before each use.
   uint8_t* raw = Ab;
-  uint8_t* Akey = Ab + (MODE == KM_KEY ? 2 * KM_TILE * SW * 4 : 0);
+  uint8_t* Akey = Ab + (MODE == KM_KEY ? 2 * (size_t)KM_TILE * SW * 4 : 0);
   auto load_tile = [&](int sub, int buf) {
     const int r0 = n0 + sub * KM_TILE;
     if (MODE == KM_QUERY) {
-      uint8_t* dst = Ab + (size_t)buf * KM_TILE * RS;
-      for (int e = tid; e < KM_TILE * (DK / 8); e += KM_THREADS) {
-        const int r = e / (DK / 8), c = e % (DK / 8), n = r0 + r;
-        cp_async16(dst + r * RS + c * 16, a.Q.row(bh, n < N ? n : 0) + c * 8, n < N ? 16 : 0);
+      uint8_t* dst = Ab + (size_t)buf * pl.nbox * KM_BOX;
+      for (int e = tid; e < KM_TILE * NCH; e += KM_THREADS) {
+        const int r = e / NCH, c = e % NCH, n = r0 + r;
+        cp_async16(dst + sw_off(r, c, KM_TILE), a.Q.row(bh, n < N ? n : 0) + c * 8, n < N ? 16 : 0);
       }
     } else {
       uint8_t* dst = raw + (size_t)buf * KM_TILE * SW * 4;
@@ -97,7 +167,10 @@ __global__ void __launch_bounds__(KM_THREADS) k_kmeans_step(KmArgs a) {
     }
     cp_async_commit();
   };
+  const uint32_t idesc = tc::idesc_bf16(KM_TILE, NC, 0);
+  const uint32_t bh_addr = smem_u32(Bh), bl_addr = smem_u32(Bl);
   const int nsub = (rows + KM_TILE - 1) / KM_TILE;
+  uint32_t phase = 0;
   load_tile(0, 0);
   for (int sub = 0; sub < nsub; ++sub) {
     if (sub + 1 < nsub) {
@@ -106,107 +179,87 @@ __global__ void __launch_bounds__(KM_THREADS) k_kmeans_step(KmArgs a) {
     } else {
       cp_async_wait<0>();
     }
-    __syncthreads();
-    const uint8_t* Ah;
-    const uint8_t* Al = nullptr;
+    uint32_t ah_addr, al_addr = 0;
     if (MODE == KM_QUERY) {
-      Ah = Ab + (size_t)(sub & 1) * KM_TILE * RS;
+      ah_addr = smem_u32(Ab + (size_t)(sub & 1) * pl.nbox * KM_BOX);
     } else {
+      __syncthreads();  // raw tile complete
       const float* src = reinterpret_cast<const float*>(raw + (size_t)(sub & 1) * KM_TILE * SW * 4);
-      uint8_t* h = Akey;
-      uint8_t* l = Akey + KM_TILE * RS;
-      for (int e = tid; e < KM_TILE * (DK / 4); e += KM_THREADS) {
-        const int r = e / (DK / 4), c4 = e % (DK / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (4 * c4 < SW) v = reinterpret_cast<const float4*>(src + r * SW)[c4];
-        const bf16 hx = __float2bfloat16_rn(v.x), hy = __float2bfloat16_rn(v.y);
-        const bf16 hz = __float2bfloat16_rn(v.z), hw = __float2bfloat16_rn(v.w);
-        uint2 ph, pl;
-        ph.x = pack_bf16(__bfloat162float(hx), __bfloat162float(hy));
-        ph.y = pack_bf16(__bfloat162float(hz), __bfloat162float(hw));
-        pl.x = pack_bf16(v.x - __bfloat162float(hx), v.y - __bfloat162float(hy));
-        pl.y = pack_bf16(v.z - __bfloat162float(hz), v.w - __bfloat162float(hw));
-        *reinterpret_cast<uint2*>(h + r * RS + c4 * 8) = ph;
-        *reinterpret_cast<uint2*>(l + r * RS + c4 * 8) = pl;
+      for (int e = tid; e < KM_TILE * NCH; e += KM_THREADS) {
+        const int r = e / NCH, c = e % NCH;
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 8 * c + i < SW ? src[r * SW + 8 * c + i] : 0.f;
+        *reinterpret_cast<uint4*>(Akey + sw_off(r, c, KM_TILE)) = split8(v, false);
+        *reinterpret_cast<uint4*>(Akey + KM_BOX + sw_off(r, c, KM_TILE)) = split8(v, true);
       }
-      __syncthreads();
-      Ah = h;
-      Al = l;
+      ah_addr = smem_u32(Akey);
+      al_addr = smem_u32(Akey + KM_BOX);
     }
-    uint32_t af[KS][4], al[NA == 2 ? KS : 1][4];
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int c = ks * 2 + (lane >> 4);
-      ldsm_x4(af[ks][0], af[ks][1], af[ks][2], af[ks][3], Ah + r * RS + c * 16);
-      if (NA == 2)
-        ldsm_x4(al[ks][0], al[ks][1], al[ks][2], al[ks][3], Al + r * RS + c * 16);
-    }
-    const int lr_lo = sub * KM_TILE + warp * 16 + gid, lr_hi = lr_lo + 8;  // chunk-local rows
-    const int r_lo = n0 + lr_lo, r_hi = n0 + lr_hi;
-    float alpha_lo = 2.f, alpha_hi = 2.f;
-    if (MODE == KM_QUERY) {
-      alpha_lo = r_lo < N ? a.scale / a.rms[(size_t)bh * N + r_lo] : 0.f;
-      alpha_hi = r_hi < N ? a.scale / a.rms[(size_t)bh * N + r_hi] : 0.f;
-    }
-    float best_lo = -FLT_MAX, best_hi = -FLT_MAX;
-    int arg_lo = 0, arg_hi = 0;
-    for (int nc = 0; nc < NC; nc += 32) {
-      float acc[4][4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+    tc::fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {  // D = A Bh^T + A Bl^T (+ Al Bh^T), fp32 in TMEM
+      tc::tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
+        const uint32_t ao = (ks >> 2) * KM_BOX + (ks & 3) * 32;
+        const uint32_t bo = (ks >> 2) * NC * 128 + (ks & 3) * 32;
+        tc::mma_ss(tbase, tc::smem_desc_sw128(ah_addr + ao, 16, 1024),
+                   tc::smem_desc_sw128(bh_addr + bo, 16, 1024), idesc, ks > 0);
+        tc::mma_ss(tbase, tc::smem_desc_sw128(ah_addr + ao, 16, 1024),
+                   tc::smem_desc_sw128(bl_addr + bo, 16, 1024), idesc, 1);
+        if (MODE == KM_KEY)
+          tc::mma_ss(tbase, tc::smem_desc_sw128(al_addr + ao, 16, 1024),
+                     tc::smem_desc_sw128(bh_addr + bo, 16, 1024), idesc, 1);
+      }
+      tc::mma_commit(mbar);
+    }
+    if (warp < 4) {  // one tile row per thread: scores from TMEM, argmax
+      bool ok = tc::mbar_wait(mbar, phase, abort_s, KM_WAIT_NS);
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, ok);
+      tc::tc_fence_after();
+      const int lr = sub * KM_TILE + warp * 32 + lane, n = n0 + lr;
+      int arg = -1;
+      if (ok) {
+        float alpha = 2.f;
+        if (MODE == KM_QUERY) alpha = n < N ? a.scale / a.rms[(size_t)bh * N + n] : 0.f;
+        float best = -FLT_MAX;
+        arg = 0;
+        for (int c0 = 0; c0 < NC; c0 += 32) {
+          uint32_t v[32];
+          __syncwarp();
+          tc::tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + c0, v);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {  // two n-tile pairs of 16 columns
-          const int brow = nc + pr * 16 + (lane & 7) + (lane >> 4) * 8;
-          const int bc = ks * 2 + ((lane >> 3) & 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(b0, b1, b2, b3, Bh + brow * RS + bc * 16);
-          mma16816(acc[pr * 2], af[ks], b0, b1);
-          mma16816(acc[pr * 2 + 1], af[ks], b2, b3);
-          if (NA == 2) {
-            mma16816(acc[pr * 2], al[ks], b0, b1);
-            mma16816(acc[pr * 2 + 1], al[ks], b2, b3);
+          for (int j = 0; j < 32; ++j) {
+            const int g = c0 + j;
+            const float sc = alpha * __uint_as_float(v[j]) - betas[g];
+            if (g < G && sc > best) {
+              best = sc;
+              arg = g;
+            }
           }
-          ldsm_x4(b0, b1, b2, b3, Bl + brow * RS + bc * 16);
-          mma16816(acc[pr * 2], af[ks], b0, b1);
-          mma16816(acc[pr * 2 + 1], af[ks], b2, b3);
         }
       }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const int col = nc + t * 8 + 2 * tig;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int g = col + e;
-          if (g < G) {
-            const float sl = alpha_lo * acc[t][e] - betas[g];
-            const float sh = alpha_hi * acc[t][2 + e] - betas[g];
-            if (sl > best_lo) { best_lo = sl; arg_lo = g; }
-            if (sh > best_hi) { best_hi = sh; arg_hi = g; }
-          }
-        }
-      }
+      labs[lr] = n < N ? arg : -1;
+      if (n < N && arg >= 0) a.lab[(size_t)bh * N + n] = arg;
     }
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      const float bl = __shfl_xor_sync(0xffffffffu, best_lo, o);
-      const int al_ = __shfl_xor_sync(0xffffffffu, arg_lo, o);
-      if (bl > best_lo || (bl == best_lo && al_ < arg_lo)) { best_lo = bl; arg_lo = al_; }
-      const float bhv = __shfl_xor_sync(0xffffffffu, best_hi, o);
-      const int ah = __shfl_xor_sync(0xffffffffu, arg_hi, o);
-      if (bhv > best_hi || (bhv == best_hi && ah < arg_hi)) { best_hi = bhv; arg_hi = ah; }
+    phase ^= 1;
+    tc::tc_fence_before();
+    __syncthreads();  // TMEM read and tile buffers free
+  }
+  if (*abort_s) {
+    if (tid == 0) {
+      set_error(a.hdr, ERR_TIMEOUT, 7, bh, chunk);
+      tc::mbar_wait_bounded(mbar, phase ^ 1, KM_WAIT_NS);  // the last commit, if still pending
     }
-    if (tig == 0) {
-      labs[lr_lo] = r_lo < N ? arg_lo : -1;
-      labs[lr_hi] = r_hi < N ? arg_hi : -1;
-      if (r_lo < N) a.lab[(size_t)bh * N + r_lo] = arg_lo;
-      if (r_hi < N) a.lab[(size_t)bh * N + r_hi] = arg_hi;
-    }
-    __syncthreads();  // tile buffers free for the next load
+    __syncthreads();
+  }
+  tc::tc_fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    tc::tmem_dealloc(tbase, tcols);
   }
 
   // ---- histogram, scan, stable chunk-local sort (A region reused) --------
@@ -370,15 +423,7 @@ __global__ void __launch_bounds__(KM_THREADS) k_kmeans_step(KmArgs a) {
 }
 
 size_t kmeans_step_smem(int mode, int DK, int SW, int G) {
-  const size_t NC = (size_t)((G + 31) / 32) * 32;
-  const size_t rs = (size_t)km_rs(DK);
-  const size_t b = 2 * NC * rs + MAX_GROUPS * 4 + CHUNK * 4;
-  const size_t tiles = mode == KM_KEY ? 2 * (size_t)KM_TILE * SW * 4 + 2 * (size_t)KM_TILE * rs
-                                      : 2 * (size_t)KM_TILE * rs;
-  const size_t rb = mode == KM_KEY ? (size_t)SW * 4 : (size_t)SW * 2;
-  const size_t stg = (size_t)(KM_THREADS / 32) * (mode == KM_KEY ? 32 : 16) * rb;
-  const size_t sortb = (32 * (size_t)G + CHUNK + MAX_GROUPS + 32) * 4 + stg;
-  return b + (tiles > sortb ? tiles : sortb);
+  return km_plan(mode, DK, SW, G).total + 1024;  // + alignment slack
 }
 
 template <int MODE, int DK, int SW>
