@@ -321,13 +321,22 @@ __global__ void __launch_bounds__(256, 1)
         for (int c = 0; c < TBN / 32; ++c)
           if (c < nch) tc::tmem_ld32(scol + 32 * c, sr + 32 * c);
         tc::tmem_wait_ld();
-        float mx = -INFINITY;
+        // row max of the raw scores (the scale is positive), in eight
+        // independent chains; keys past the tile's valid count (partial
+        // tiles only) are masked to -inf
+        if (nvalid < TBN) {
 #pragma unroll
-        for (int c = 0; c < TBN; ++c) {
-          const float x = c < nvalid ? __uint_as_float(sr[c]) * a.scale_log2 : -INFINITY;
-          sr[c] = f2u(x);
-          mx = fmaxf(mx, x);
+          for (int c = 0; c < TBN; ++c)
+            if (c >= nvalid) sr[c] = f2u(-INFINITY);
         }
+        float mx8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(sr[q]);
+#pragma unroll
+        for (int c = 8; c < TBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                         a.scale_log2;
         const float mn = fmaxf(m, mx);
         float m_use = m;
         bool rescale = false;
@@ -336,22 +345,24 @@ __global__ void __launch_bounds__(256, 1)
           rescale = !first;
         }
         const float corr = rescale ? ex2(m - m_use) : 1.f;
-        float sum = 0.f;
+        const float neg = -m_use;
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (64 * h < nvalid) {  // uniform across the warp: one tile for all rows
             uint32_t pr[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const float p0 = ex2(__uint_as_float(sr[64 * h + 2 * c]) - m_use);
-              const float p1 = ex2(__uint_as_float(sr[64 * h + 2 * c + 1]) - m_use);
-              sum += p0 + p1;
+              const float p0 = ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c]), a.scale_log2, neg));
+              const float p1 = ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c + 1]), a.scale_log2, neg));
+              sum4[c & 3] += p0 + p1;
               pr[c] = pack_bf16(p0, p1);
             }
             __syncwarp();
             tc::tmem_st32(scol + 32 * h, pr);
           }
         }
+        const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         if (!first) {  // O holds PV of the previous tile once it is done
           const bool got_o = tc::mbar_wait(o_done, pvseen & 1, abort_s, WAIT_NS);
           __syncwarp();
