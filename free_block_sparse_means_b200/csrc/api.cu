@@ -79,6 +79,7 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_PART] = part_slots * 8;
   // k-means partial sums: per chunk, one slot per (group, warp segment)
   sz[B_CSUM] = BH * nchunk * (Gm + CSUM_SLOTS) * (d > P ? d : P) * 4;
+  if (sz[B_CSUM] < BH * Gm * 8 * d * 4) sz[B_CSUM] = BH * Gm * 8 * d * 4;  // group-mean slices
   // probe rows gathered for the fit: sparse outputs X, residuals R, block means
   sz[B_XP] = BH * (M ? M : 1) * d * 4;
   sz[B_RP] = BH * (M ? M : 1) * d * 4;

@@ -401,21 +401,44 @@ __global__ void __launch_bounds__(EIG_THREADS, 1) k_eig_top(const float* Ain, in
             cur = nxt;
           }
           // back: y <- U^-1 y, with y_{i+1}, y_{i+2} carried in registers
+          // Near-singular pivots make the solution grow step by step; when an
+          // entry passes 1e15 the whole system (solved entries and the
+          // right-hand side still to be used) is scaled by 1e-15 -- the
+          // direction is all that matters -- so y^2 sums stay finite.
+          auto shrink = [&]() {
+            for (int j = 0; j < NN; ++j) yv[j * 32 + lane] *= 1e-15f;
+          };
+          yv[(NN - 1) * 32 + lane] = cur;
           float y2 = cur * rud[(NN - 1) * 32 + lane];
+          if (fabsf(y2) > 1e15f) {
+            shrink();
+            y2 *= 1e-15f;
+          }
           yv[(NN - 1) * 32 + lane] = y2;
           float y1 = (yv[(NN - 2) * 32 + lane] - us[(NN - 2) * 32 + lane] * y2) *
                      rud[(NN - 2) * 32 + lane];
+          if (fabsf(y1) > 1e15f) {
+            shrink();
+            y1 *= 1e-15f;
+            y2 *= 1e-15f;
+          }
           yv[(NN - 2) * 32 + lane] = y1;
-          float nrm = y2 * y2 + y1 * y1;
 #pragma unroll 4
           for (int i = NN - 3; i >= 0; --i) {
             const int o = i * 32 + lane;
-            const float yi = (yv[o] - us[o] * y1 - uf[o] * y2) * rud[o];
+            float yi = (yv[o] - us[o] * y1 - uf[o] * y2) * rud[o];
+            if (fabsf(yi) > 1e15f) {
+              shrink();
+              yi *= 1e-15f;
+              y1 *= 1e-15f;
+              y2 *= 1e-15f;
+            }
             yv[o] = yi;
-            nrm += yi * yi;
             y2 = y1;
             y1 = yi;
           }
+          float nrm = 0.f;
+          for (int i = 0; i < NN; ++i) nrm += yv[i * 32 + lane] * yv[i * 32 + lane];
           const float inv = nrm > 0.f ? rsqrtf(nrm) : 0.f;
           for (int i = 0; i < NN; ++i) yv[i * 32 + lane] *= inv;
         }
@@ -524,9 +547,9 @@ __global__ void __launch_bounds__(EIG_THREADS, 1) k_eig_top(const float* Ain, in
   }
   __syncthreads();
   for (int e = tid; e < K; e += EIG_THREADS) evals[(size_t)m * NN + e] = lam[e];
-  for (int e = tid; e < NN * K; e += EIG_THREADS) {
-    const int row = e / K, kq = e % K;
-    evecs[(size_t)m * NN * NN + row * NN + kq] = Y[kq * LD + row];
+  for (int e = tid; e < NN * NN; e += EIG_THREADS) {  // columns past K are zero
+    const int row = e / NN, kq = e % NN;
+    evecs[(size_t)m * NN * NN + e] = kq < K ? Y[kq * LD + row] : 0.f;
   }
 }
 

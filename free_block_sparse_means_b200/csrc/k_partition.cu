@@ -18,13 +18,14 @@ int padded_p(int p) { return p <= 8 ? 8 : p <= 16 ? 16 : p <= 32 ? 32 : 64; }
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) k_metric(TensorView Q, int N, int Ms, float* MK) {
+  constexpr int SB = 128;  // sampled rows staged per step
   const int bh = blockIdx.x;
   const int ti = blockIdx.y / (D / 32), tj = blockIdx.y % (D / 32);
-  __shared__ float As[32][33], Bs[32][33];
+  __shared__ float As[SB][33], Bs[SB][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s0 = 0; s0 < Ms; s0 += 32) {
-    for (int e = threadIdx.x; e < 32 * 32; e += 256) {
+  for (int s0 = 0; s0 < Ms; s0 += SB) {
+    for (int e = threadIdx.x; e < SB * 32; e += 256) {
       const int rr = e >> 5, c = e & 31, s = s0 + rr;
       float a = 0.f, b = 0.f;
       if (s < Ms) {
@@ -38,7 +39,7 @@ __global__ void __launch_bounds__(256) k_metric(TensorView Q, int N, int Ms, flo
     }
     __syncthreads();
 #pragma unroll 8
-    for (int rr = 0; rr < 32; ++rr) {
+    for (int rr = 0; rr < SB; ++rr) {
       const float bv = Bs[rr][tx];
 #pragma unroll
       for (int k = 0; k < 4; ++k) acc[k] += As[rr][ty * 4 + k] * bv;
@@ -49,7 +50,6 @@ __global__ void __launch_bounds__(256) k_metric(TensorView Q, int N, int Ms, flo
   for (int k = 0; k < 4; ++k)
     MK[((size_t)bh * D + ti * 32 + ty * 4 + k) * D + tj * 32 + tx] = acc[k] / (float)Ms;
 }
-
 
 // W[:, k] = u_k sqrt(lambda_k / sum_j lambda_j) for k < p; zero for p <= k < pp.
 // The eigenvalue sum of the positive semidefinite M_K is its trace.
@@ -63,42 +63,6 @@ __global__ void k_keyweights(const float* evals, const float* evecs, const float
     if (k < p && tot > 0.f)
       w = evecs[((size_t)bh * D + i) * D + k] * sqrtf(fmaxf(evals[(size_t)bh * D + k], 0.f) / tot);
     W[(size_t)bh * D * pp + e] = w;
-  }
-}
-
-// z_n = W^T k_n  (key-response coordinates).
-template <int D, int PP>
-__global__ void __launch_bounds__(256) k_project(TensorView K, int N, const float* W, float* Z) {
-  __shared__ __align__(16) float Ws[D * PP];
-  const int bh = blockIdx.y;
-  for (int e = threadIdx.x; e < D * PP; e += 256) Ws[e] = W[(size_t)bh * D * PP + e];
-  __syncthreads();
-  for (int n = blockIdx.x * 256 + threadIdx.x; n < N; n += gridDim.x * 256) {
-    const uint4* srow = reinterpret_cast<const uint4*>(K.row(bh, n));
-    float acc[PP];
-#pragma unroll
-    for (int k = 0; k < PP; ++k) acc[k] = 0.f;
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 raw = srow[c];
-      const bf16* v = reinterpret_cast<const bf16*>(&raw);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float x = bf2f(v[e]);
-        const float4* w = reinterpret_cast<const float4*>(&Ws[(c * 8 + e) * PP]);
-#pragma unroll
-        for (int k = 0; k < PP / 4; ++k) {
-          const float4 ww = w[k];
-          acc[4 * k] += x * ww.x;
-          acc[4 * k + 1] += x * ww.y;
-          acc[4 * k + 2] += x * ww.z;
-          acc[4 * k + 3] += x * ww.w;
-        }
-      }
-    }
-    float4* dst = reinterpret_cast<float4*>(Z + ((size_t)bh * N + n) * PP);
-#pragma unroll
-    for (int k = 0; k < PP / 4; ++k)
-      dst[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
   }
 }
 
@@ -158,77 +122,6 @@ __global__ void k_init_centk(const float* Z, int N, int G, int PP, const int32_t
 }
 
 // ---------------------------------------------------------------------------
-// Key assignment in eigen-coordinates: argmin_g ||z - c_g||^2 (ties to the
-// lowest g).  One block of ASG_THREADS threads per ASG_THREADS * RPT rows.
-// ---------------------------------------------------------------------------
-constexpr int ASG_THREADS = 128;
-
-template <int PP, int RPT>
-__global__ void __launch_bounds__(ASG_THREADS) k_assign_z(const float* Z, int N, int G,
-                                                          const float* cent, int32_t* lab) {
-  extern __shared__ __align__(16) float asm_[];
-  float* C = asm_;
-  float* cn = C + G * PP;
-  const int bh = blockIdx.y, tid = threadIdx.x;
-  constexpr int NT = ASG_THREADS;
-  for (int e = tid; e < G * PP; e += NT) C[e] = cent[(size_t)bh * G * PP + e];
-  __syncthreads();
-  for (int g = tid; g < G; g += NT) {
-    float s = 0.f;
-    for (int k = 0; k < PP; ++k) s += C[g * PP + k] * C[g * PP + k];
-    cn[g] = s;
-  }
-  __syncthreads();
-  float z[RPT][PP];
-  int n[RPT];
-#pragma unroll
-  for (int r = 0; r < RPT; ++r) {
-    n[r] = blockIdx.x * NT * RPT + tid + r * NT;
-    const float4* src = reinterpret_cast<const float4*>(Z + ((size_t)bh * N + (n[r] < N ? n[r] : 0)) * PP);
-#pragma unroll
-    for (int k = 0; k < PP / 4; ++k) {
-      const float4 v = src[k];
-      z[r][4 * k] = v.x;
-      z[r][4 * k + 1] = v.y;
-      z[r][4 * k + 2] = v.z;
-      z[r][4 * k + 3] = v.w;
-    }
-  }
-  float best[RPT];
-  int arg[RPT];
-#pragma unroll
-  for (int r = 0; r < RPT; ++r) {
-    best[r] = FLT_MAX;
-    arg[r] = 0;
-  }
-  for (int g = 0; g < G; ++g) {
-    const float4* c4 = reinterpret_cast<const float4*>(C + g * PP);
-    float dot[RPT];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) dot[r] = 0.f;
-#pragma unroll
-    for (int k = 0; k < PP / 4; ++k) {
-      const float4 c = c4[k];
-#pragma unroll
-      for (int r = 0; r < RPT; ++r)
-        dot[r] += z[r][4 * k] * c.x + z[r][4 * k + 1] * c.y + z[r][4 * k + 2] * c.z +
-                  z[r][4 * k + 3] * c.w;
-    }
-    const float cg = cn[g];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const float sc = cg - 2.f * dot[r];
-      if (sc < best[r]) {
-        best[r] = sc;
-        arg[r] = g;
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < RPT; ++r)
-    if (n[r] < N) lab[(size_t)bh * N + n[r]] = arg[r];
-}
-
 // ---------------------------------------------------------------------------
 // Per (bh, g): base of each chunk within the group (exclusive scan over
 // chunks), group sizes, and group offsets (exclusive scan over g).
@@ -295,274 +188,6 @@ __global__ void __launch_bounds__(CHUNK) k_scatter(const int32_t* lab, int N, in
   }
 }
 
-// ---------------------------------------------------------------------------
-// Segmented sums over the members of each group (fixed order, fp64
-// accumulation, deterministic).  Modes:
-//   SEG_Z       rows of Z (fp32, PP wide) at perm[i]          -> k-means update
-//   SEG_QSCALED rows (s / rms_n) q_n at n = perm[i]           -> k-means update
-//   SEG_BF16    rows i of a contiguous permuted bf16 buffer     -> means
-// keep_empty: an empty group keeps out's previous row, else it is zeroed.
-// ---------------------------------------------------------------------------
-enum { SEG_Z = 0, SEG_QSCALED = 1, SEG_BF16 = 2 };
-
-struct SegArgs {
-  const float* Z;
-  TensorView Q;
-  const float* rms;
-  float scale;
-  const bf16* Xp;
-  const int32_t* perm;
-  const int32_t* off;
-  int N, G;
-  float* out;
-  int keep_empty;
-};
-
-template <int MODE, int DD>
-__device__ __forceinline__ void seg_row(const SegArgs& a, int bh, int i, int lane, float* v) {
-  constexpr int NV = (MODE == SEG_Z) ? (DD + 31) / 32 : DD / 32;
-  if (MODE == SEG_Z) {
-    const int row = a.perm[(size_t)bh * a.N + i];
-    const float* src = a.Z + ((size_t)bh * a.N + row) * DD;
-#pragma unroll
-    for (int q = 0; q < NV; ++q) v[q] = (lane + 32 * q < DD) ? src[lane + 32 * q] : 0.f;
-  } else {
-    const bf16* src;
-    float sc = 1.f;
-    if (MODE == SEG_QSCALED) {
-      const int row = a.perm[(size_t)bh * a.N + i];
-      src = a.Q.row(bh, row);
-      sc = a.scale / a.rms[(size_t)bh * a.N + row];
-    } else {
-      src = a.Xp + ((size_t)bh * a.N + i) * DD;
-    }
-#pragma unroll
-    for (int q = 0; q < NV / 2; ++q) {
-      const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(src)[lane + 32 * q];
-      v[2 * q] = sc * __low2float(x);
-      v[2 * q + 1] = sc * __high2float(x);
-    }
-  }
-}
-
-// 8 warps; warp w sums rows start + w + 8 t in ascending t, with four rows'
-// loads in flight, then the warps' partial sums are added in warp order.
-template <int MODE, int DD>
-__global__ void __launch_bounds__(256) k_segsum(SegArgs a) {
-  constexpr int NV = (MODE == SEG_Z) ? (DD + 31) / 32 : DD / 32;  // values per lane
-  constexpr int NW = 8, UN = 4;
-  __shared__ double red[NW][DD];
-  const int bh = blockIdx.y, g = blockIdx.x, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int start = a.off[(size_t)bh * (a.G + 1) + g], end = a.off[(size_t)bh * (a.G + 1) + g + 1];
-  double acc[NV];
-#pragma unroll
-  for (int q = 0; q < NV; ++q) acc[q] = 0.0;
-  for (int i0 = start + w; i0 < end; i0 += NW * UN) {
-    float v[UN][NV];
-#pragma unroll
-    for (int u = 0; u < UN; ++u) {
-      const int i = i0 + u * NW;
-      if (i < end) {
-        seg_row<MODE, DD>(a, bh, i, lane, v[u]);
-      } else {
-#pragma unroll
-        for (int q = 0; q < NV; ++q) v[u][q] = 0.f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < UN; ++u)
-#pragma unroll
-      for (int q = 0; q < NV; ++q) acc[q] += (double)v[u][q];
-  }
-  if (MODE == SEG_Z) {
-#pragma unroll
-    for (int q = 0; q < NV; ++q)
-      if (lane + 32 * q < DD) red[w][lane + 32 * q] = acc[q];
-  } else {
-#pragma unroll
-    for (int q = 0; q < NV / 2; ++q) {
-      red[w][2 * (lane + 32 * q)] = acc[2 * q];
-      red[w][2 * (lane + 32 * q) + 1] = acc[2 * q + 1];
-    }
-  }
-  __syncthreads();
-  const int cnt = end - start;
-  for (int k = threadIdx.x; k < DD; k += NW * 32) {
-    double s = 0.0;
-#pragma unroll
-    for (int q = 0; q < NW; ++q) s += red[q][k];
-    float* o = a.out + ((size_t)bh * a.G + g) * DD + k;
-    if (cnt > 0)
-      *o = (float)(s / cnt);
-    else if (!a.keep_empty)
-      *o = 0.f;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// k-means update without a global permutation.  After an assignment pass,
-// each CHUNK-row chunk counts its labels (the histogram the final stable
-// scatter also uses), sorts its rows by label (stable: by row within a
-// label) and warp w sums the rows at sorted positions [32w, 32w + 32),
-// flushing one partial sum per group it meets into slot g + w of the chunk
-// (distinct: the groups met by warp w + 1 start where warp w's end).  The
-// reducer adds, for each group, the slots of every warp segment that holds
-// it, chunk by chunk in order, in fp64; the order of every sum is fixed, so
-// the update is deterministic.  Rows: SEG_Z rows of Z (fp32, DD wide) or
-// SEG_QSCALED rows (s / rms_n) q_n (bf16 q, DD = head dim).
-// ---------------------------------------------------------------------------
-struct ChunkSumArgs {
-  const float* Z;
-  TensorView Q;
-  const float* rms;
-  float scale;
-  const int32_t* lab;
-  int32_t* chunk_cnt;        // [BH][nchunk][G] label histogram of each chunk (out)
-  int N, G, nchunk;
-  int32_t* loff;             // [BH][nchunk][G] chunk-local group offsets (out)
-  float* part;               // [BH][nchunk][G + CSUM_SLOTS][DD] partial sums (out)
-  Header* hdr;
-};
-
-template <int MODE, int DD>
-__global__ void __launch_bounds__(CHUNK) k_chunk_sums(ChunkSumArgs a) {
-  constexpr int NV = (MODE == SEG_Z) ? (DD + 31) / 32 : DD / 32;  // values per lane
-  constexpr int UN = 8;  // rows in flight per warp (divides 32)
-  __shared__ int cnt[32][MAX_GROUPS];
-  __shared__ int loff[MAX_GROUPS];
-  __shared__ int srt[CHUNK];  // local row | label << 10, in sorted order
-  __shared__ int wsum[32];
-  const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const int G = a.G;
-  const size_t cidx = (size_t)bh * a.nchunk + chunk;
-  const int n0 = chunk * CHUNK, rows = min(CHUNK, a.N - n0);
-  for (int e = tid; e < 32 * G; e += CHUNK) cnt[e / G][e % G] = 0;
-  if (tid < G) loff[tid] = 0;
-  srt[tid] = -1;  // an unfilled position (only after an index error) is skipped
-  __syncthreads();
-  int g = tid < rows ? a.lab[(size_t)bh * a.N + n0 + tid] : -1;
-  if (g >= G || g < -1) {
-    set_error(a.hdr, ERR_INDEX, 3, bh, n0 + tid);
-    g = -1;
-  }
-  if (g >= 0) atomicAdd(&loff[g], 1);  // the chunk's label histogram
-  __syncthreads();
-  {  // exclusive scan of the histogram over the groups
-    const int v = tid < G ? loff[tid] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    if (lane == 31) wsum[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-      const int x = wsum[lane];
-      int xi = x;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, xi, o);
-        if (lane >= o) xi += t;
-      }
-      wsum[lane] = xi - x;
-    }
-    __syncthreads();
-    if (tid < G) {
-      const int lo = wsum[w] + incl - v;
-      loff[tid] = lo;
-      a.loff[cidx * G + tid] = lo;
-      a.chunk_cnt[cidx * G + tid] = v;
-    }
-  }
-  const unsigned mask = __match_any_sync(0xffffffffu, g);
-  const int rank_w = __popc(mask & ((1u << lane) - 1u));
-  if (g >= 0 && (__ffs(mask) - 1) == lane) cnt[w][g] = __popc(mask);
-  __syncthreads();
-  if (g >= 0) {
-    int before = 0;
-    for (int i = 0; i < w; ++i) before += cnt[i][g];
-    const int pos = loff[g] + before + rank_w;
-    if (pos < 0 || pos >= rows)
-      set_error(a.hdr, ERR_INDEX, 4, bh, pos);
-    else
-      srt[pos] = tid | (g << 10);
-  }
-  __syncthreads();
-  const int p0 = 32 * w, p1 = min(p0 + 32, rows);
-  if (p0 >= p1) return;
-  // lane i decodes sorted position p0 + i once; the warp then walks the 32
-  // positions in order with the row, label and scale broadcast by shuffles
-  const int e_l = p0 + lane < p1 ? srt[p0 + lane] : -1;
-  const int g_l = e_l >= 0 ? e_l >> 10 : -1;
-  const int row_l = n0 + (e_l >= 0 ? (e_l & 1023) : 0);
-  float f_l = 1.f;
-  if (MODE == SEG_QSCALED && e_l >= 0) f_l = a.scale / a.rms[(size_t)bh * a.N + row_l];
-  const float* zbase = a.Z + (size_t)bh * a.N * DD;
-  const bf16* qbase = MODE == SEG_QSCALED ? a.Q.row(bh, 0) : nullptr;
-  const int64_t qsn = a.Q.sn;
-  float* slot0 = a.part + cidx * (size_t)(G + CSUM_SLOTS) * DD;
-  float acc[NV];
-#pragma unroll
-  for (int q = 0; q < NV; ++q) acc[q] = 0.f;
-  int cur = __shfl_sync(0xffffffffu, g_l, 0);
-  auto flush = [&](int gg) {
-    if (gg < 0) return;
-    float* dst = slot0 + (size_t)(gg + w) * DD;
-    if (MODE == SEG_Z) {
-#pragma unroll
-      for (int q = 0; q < NV; ++q)
-        if (lane + 32 * q < DD) dst[lane + 32 * q] = acc[q];
-    } else {
-#pragma unroll
-      for (int q = 0; q < NV / 2; ++q)
-        reinterpret_cast<float2*>(dst)[lane + 32 * q] = make_float2(acc[2 * q], acc[2 * q + 1]);
-    }
-  };
-#pragma unroll 1
-  for (int u0 = 0; u0 < 32; u0 += UN) {
-    float v[UN][NV], fu[UN];
-    int gu[UN];
-#pragma unroll
-    for (int u = 0; u < UN; ++u) {
-      gu[u] = u0 + u < 32 ? __shfl_sync(0xffffffffu, g_l, u0 + u) : -1;
-      fu[u] = __shfl_sync(0xffffffffu, f_l, u0 + u);
-      const int row = __shfl_sync(0xffffffffu, row_l, u0 + u);
-#pragma unroll
-      for (int q = 0; q < NV; ++q) v[u][q] = 0.f;
-      if (gu[u] >= 0) {
-        if (MODE == SEG_Z) {
-          const float* src = zbase + (size_t)row * DD;
-#pragma unroll
-          for (int q = 0; q < NV; ++q)
-            if (lane + 32 * q < DD) v[u][q] = src[lane + 32 * q];
-        } else {
-          const __nv_bfloat162* src = reinterpret_cast<const __nv_bfloat162*>(qbase + row * qsn);
-#pragma unroll
-          for (int q = 0; q < NV / 2; ++q) {
-            const __nv_bfloat162 x = src[lane + 32 * q];
-            v[u][2 * q] = __low2float(x);
-            v[u][2 * q + 1] = __high2float(x);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < UN; ++u) {
-      if (gu[u] < 0) continue;
-      if (gu[u] != cur) {
-        flush(cur);
-#pragma unroll
-        for (int q = 0; q < NV; ++q) acc[q] = 0.f;
-        cur = gu[u];
-      }
-#pragma unroll
-      for (int q = 0; q < NV; ++q) acc[q] = fmaf(fu[u], v[u][q], acc[q]);
-    }
-  }
-  flush(cur);
-}
-
 // Group means from the chunk partial sums.  Grid (G, BH), one thread per
 // coordinate; an empty group keeps its previous centroid.  The block first
 // lists the slots holding the group (chunk by chunk, warp segment by warp
@@ -624,6 +249,68 @@ __global__ void k_chunk_reduce(const float* part, const int32_t* chunk_cnt, cons
   if (k + 1 < n) s1 += (double)base[(size_t)slots[k + 1] * DD];
   if (k + 2 < n) s2 += (double)base[(size_t)slots[k + 2] * DD];
   out[((size_t)bh * G + g) * DD + i] = (float)(((s0 + s1) + (s2 + s3)) / (double)tot_s);
+}
+
+// Means of the contiguous group-major bf16 rows of each group, balanced over
+// groups of very different sizes: each group's range is cut into GM_SLICES
+// equal slices, one block per (group, slice) sums its rows (fixed order,
+// fp64), and k_gmean_fin adds the slices in order.  Empty groups get zero.
+constexpr int GM_SLICES = 8;
+
+template <int D>
+__global__ void __launch_bounds__(256) k_gmean_part(const bf16* Xp, const int32_t* off, int N, int G,
+                                                    float* part) {
+  constexpr int NV = D / 32;  // values per lane (bf16 pairs: NV / 2)
+  __shared__ double red[8][D];
+  const int g = blockIdx.x, bh = blockIdx.y, sl = blockIdx.z;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o0 = off[(size_t)bh * (G + 1) + g], cnt = off[(size_t)bh * (G + 1) + g + 1] - o0;
+  const int lo = o0 + (int)((int64_t)cnt * sl / GM_SLICES);
+  const int hi = o0 + (int)((int64_t)cnt * (sl + 1) / GM_SLICES);
+  double acc[NV];
+#pragma unroll
+  for (int q = 0; q < NV; ++q) acc[q] = 0.0;
+  for (int i0 = lo + w; i0 < hi; i0 += 8 * 4) {
+    float v[4][NV];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + 8 * u;
+#pragma unroll
+      for (int q = 0; q < NV / 2; ++q) {
+        float2 x = make_float2(0.f, 0.f);
+        if (i < hi)
+          x = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Xp + ((size_t)bh * N + i) * D)[lane + 32 * q]);
+        v[u][2 * q] = x.x;
+        v[u][2 * q + 1] = x.y;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int q = 0; q < NV; ++q) acc[q] += (double)v[u][q];
+  }
+#pragma unroll
+  for (int q = 0; q < NV / 2; ++q) {
+    red[w][2 * (lane + 32 * q)] = acc[2 * q];
+    red[w][2 * (lane + 32 * q) + 1] = acc[2 * q + 1];
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < D; k += 256) {
+    double t = 0.0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += red[q][k];
+    part[(((size_t)bh * G + g) * GM_SLICES + sl) * D + k] = (float)t;
+  }
+}
+
+template <int D>
+__global__ void k_gmean_fin(const float* part, const int32_t* off, int G, float* out) {
+  const int g = blockIdx.x, bh = blockIdx.y, k = threadIdx.x;
+  const int cnt = off[(size_t)bh * (G + 1) + g + 1] - off[(size_t)bh * (G + 1) + g];
+  double t = 0.0;
+#pragma unroll
+  for (int sl = 0; sl < GM_SLICES; ++sl) t += (double)part[(((size_t)bh * G + g) * GM_SLICES + sl) * D + k];
+  out[((size_t)bh * G + g) * D + k] = cnt > 0 ? (float)(t / cnt) : 0.f;
 }
 
 // Key objective with the final centroids: sum_n ||z_n - c_{lab_n}||^2 (fp64
@@ -970,10 +657,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   spr_launch(k_metric<D>, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, Q, N, p.Ms, P.MK);
   if ((e = launch_eig(P.MK, BH, D, p.p, P.eval, P.evec, P.trace, st)) != cudaSuccess) return e;
   spr_launch(k_keyweights, BH, 256, 0, st, P.eval, P.evec, P.trace, D, p.p, pp, P.W);
-  const int pgrid = min((N + 255) / 256, max(1, 4 * sms / BH + 1));
-#define PROJ(PPV) spr_launch(k_project<D, PPV>, dim3(pgrid, BH), 256, 0, st, K, N, P.W, P.Z)
-  if (pp == 8) PROJ(8); else if (pp == 16) PROJ(16); else if (pp == 32) PROJ(32); else PROJ(64);
-#undef PROJ
+  if ((e = launch_project(K, N, D, pp, BH, P.W, P.Z, P.hdr, st)) != cudaSuccess) return e;
   spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
   spr_launch(k_init_centk, BH, 256, 0, st, P.Z, N, p.Gk, pp, P.initk, P.centk);
   // Key k-means
@@ -1009,16 +693,8 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   const int ggrid = sms * 8;
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
-  {
-    SegArgs sa{};
-    sa.Xp = P.Kp;
-    sa.off = P.kvoff;
-    sa.N = N;
-    sa.G = p.Gk;
-    sa.out = P.Craw;
-    sa.keep_empty = 0;
-    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gk, BH), 256, 0, st, sa);
-  }
+  spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.csum);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.csum, P.kvoff, p.Gk, P.Craw);
   // P.counts holds |K_j| now; keep a copy of key counts in kv_off differences.
   spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
   const int split_rows = p.Gq > D ? p.Gq : D;
@@ -1048,9 +724,6 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   }
   // Query k-means in the head dimension
   spr_launch(k_init_centq, BH, 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale, P.centq);
-  const int ncq = ((p.Gq + 31) / 32) * 32;
-  const size_t smq = (size_t)2 * ncq * D * 2 + ATT_BM * D * 2 + MAX_GROUPS * 8 + 64;
-  cudaFuncSetAttribute(k_rowgemm<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq);
   for (int it = 0; it < p.iters; ++it) {
     spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
                                           split_rows, nullptr);
@@ -1082,16 +755,8 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
                                         split_rows, P.part + (size_t)BH * 2 * (nchunk + 1));
   // Group-major queries and raw query means
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, Q, P.permq, N, BH, P.Qp);
-  {
-    SegArgs sa{};
-    sa.Xp = P.Qp;
-    sa.off = P.qoff;
-    sa.N = N;
-    sa.G = p.Gq;
-    sa.out = P.qbar;
-    sa.keep_empty = 0;
-    spr_launch(k_segsum<SEG_BF16, D>, dim3(p.Gq, BH), 256, 0, st, sa);
-  }
+  spr_launch(k_gmean_part<D>, dim3(p.Gq, BH, GM_SLICES), 256, 0, st, P.Qp, P.qoff, N, p.Gq, P.csum);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gq, BH), D, 0, st, P.csum, P.qoff, p.Gq, P.qbar);
   return cudaGetLastError();
 }
 

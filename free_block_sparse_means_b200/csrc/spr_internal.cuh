@@ -128,6 +128,9 @@ struct KmArgs {
 };
 cudaError_t launch_kmeans_step(int mode, int width, const KmArgs& a, int nchunk, int BH,
                                cudaStream_t st);
+// Key-response coordinates Z = K W (tensor cores); W is [BH][d][pp] fp32.
+cudaError_t launch_project(const TensorView& K, int N, int D, int PP, int BH, const float* W,
+                           float* Z, Header* hdr, cudaStream_t st);
 
 // Every kernel launch of the library goes through spr_launch, which counts it
 // (sparsepr_launch_count reports the total).
