@@ -24,18 +24,33 @@ __global__ void __launch_bounds__(256) k_metric(TensorView Q, int N, int Ms, flo
   __shared__ float As[SB][33], Bs[SB][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // a stage: 128 sampled rows x 32 columns of each operand, as 16-byte
+  // pieces (4 per row and operand), every load issued before any is used
+  constexpr int NL = SB * 4 * 2 / 256;
   for (int s0 = 0; s0 < Ms; s0 += SB) {
-    for (int e = threadIdx.x; e < SB * 32; e += 256) {
-      const int rr = e >> 5, c = e & 31, s = s0 + rr;
-      float a = 0.f, b = 0.f;
+    uint4 v[NL];
+#pragma unroll
+    for (int q = 0; q < NL; ++q) {
+      const int e = q * 256 + threadIdx.x;
+      const int mat = e / (SB * 4), rr = (e % (SB * 4)) >> 2, c = e & 3, s = s0 + rr;
+      v[q] = make_uint4(0, 0, 0, 0);
       if (s < Ms) {
         const int row = (int)(((int64_t)s * N) / Ms);
-        const bf16* q = Q.row(bh, row);
-        a = bf2f(q[ti * 32 + c]);
-        b = bf2f(q[tj * 32 + c]);
+        v[q] = *reinterpret_cast<const uint4*>(Q.row(bh, row) + (mat ? tj : ti) * 32 + c * 8);
       }
-      As[rr][c] = a;
-      Bs[rr][c] = b;
+    }
+#pragma unroll
+    for (int q = 0; q < NL; ++q) {
+      const int e = q * 256 + threadIdx.x;
+      const int mat = e / (SB * 4), rr = (e % (SB * 4)) >> 2, c = e & 3;
+      float* dst = (mat ? &Bs[rr][0] : &As[rr][0]) + c * 8;
+      const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+        dst[2 * k] = f.x;
+        dst[2 * k + 1] = f.y;
+      }
     }
     __syncthreads();
 #pragma unroll 8

@@ -513,7 +513,9 @@ static cudaError_t reconstruct_d(const spr_params& p, const Layout& L, const Ptr
   const int RA = (R + 1) & ~1;
   const size_t sm = (size_t)(2 * D * RA + D * APPLY_XT + 4 * RA * APPLY_XT) * 4;
   cudaFuncSetAttribute(k_apply<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  const int bph = max(1, min((N + APPLY_TR - 1) / APPLY_TR, (num_sms() * 4 + BH - 1) / BH));
+  // one wave: four 256-thread blocks fit on an SM (63 registers, 44 KB of
+  // shared memory at d = 128), so at most 4 x SMs blocks in all
+  const int bph = max(1, min((N + APPLY_TR - 1) / APPLY_TR, num_sms() * 4 / BH));
   spr_launch(k_apply<D>, dim3(bph, BH), 256, sm, st, P.osp, P.odn, P.pslot, P.permq, P.fitB,
              P.fitU, P.fitBv, P.stats, RA, N, M, p.H, p.o_strides[0], p.o_strides[1],
              p.o_strides[2], O, M > 0, P.hdr);

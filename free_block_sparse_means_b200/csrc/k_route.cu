@@ -176,9 +176,29 @@ __global__ void __launch_bounds__(1024) k_route_budget(const float* tail, const 
   const int ncell = Gq * Gk;
   const float* R = tail + (size_t)bh * ncell;
   auto bits = [](float r) -> long long { return r < 0.f ? -1ll : (long long)__float_as_uint(r); };
+  // the first RB_CACHE cells of every thread stay in registers (bit pattern,
+  // pair count) for the whole search; more cells are read again each round
+  constexpr int RB_CACHE = 8;
+  int cb[RB_CACHE];
+  long long cw[RB_CACHE];
+#pragma unroll
+  for (int q = 0; q < RB_CACHE; ++q) {
+    const int t = tid + q * 1024;
+    cb[q] = -1;
+    cw[q] = 0;
+    if (t < ncell) {
+      const int i = t / Gk, j = t - i * Gk;
+      if (nqs[i] > 0 && nks[j] > 0) {
+        cb[q] = (int)bits(R[t]);
+        cw[q] = (long long)nqs[i] * nks[j];
+      }
+    }
+  }
   auto cost = [&](long long T) {
     long long c = 0;
-    for (int t = tid; t < ncell; t += 1024) {
+#pragma unroll
+    for (int q = 0; q < RB_CACHE; ++q) c += (long long)cb[q] >= T ? cw[q] : 0ll;
+    for (int t = tid + RB_CACHE * 1024; t < ncell; t += 1024) {
       const int i = t / Gk, j = t - i * Gk;
       if (nqs[i] > 0 && nks[j] > 0 && bits(R[t]) >= T) c += (long long)nqs[i] * nks[j];
     }
