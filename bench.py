@@ -170,7 +170,8 @@ def oracle_head_seconds(wl, bh):
     """Seconds the fp64 oracle takes for one whole head (independent mode)."""
     from oracle import Params, sparsepr_head
     prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
-                 tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index)
+                 tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index,
+                 partition=wl.partition)
     Q, K, V = voronoi_qkv(wl, heads=[bh])
     q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
     t0 = time.perf_counter()
@@ -197,7 +198,8 @@ def config_of(wl, world):
             "Ms": wl.Ms, "p": wl.p, "Gk": wl.Gk, "Gq": wl.Gq, "iters": wl.iters,
             "routing": (f"budget rho_target={wl.rho_target}" if wl.route_mode == "budget"
                         else f"tau={wl.tau}"),
-            "M": wl.M, "r": wl.r, "lambda": wl.lam, "parallelism": f"heads x{world} (weak)",
+            "M": wl.M, "r": wl.r, "lambda": wl.lam, "partition": wl.partition,
+            "parallelism": f"heads x{world} (weak)",
             "l2": "flushed (256 MiB write) before every timed call"}
 
 
@@ -225,22 +227,28 @@ def run_reference(args, wl):
     return 0
 
 
-def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=256, seed=0):
+def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=1024, seed=0):
     """Attention-reconstruction error against dense attention on sampled rows
-    (the same rows in every head): relative L2 over the sample of the
-    hard-drop output (routed cells only) and of the SparsePR output.  The
-    dense reference rows are computed here in fp32 (measurement only)."""
+    (the same rows in every head), as measurement only (dense rows in fp32,
+    the fit below in fp64, both with torch outside the timed region):
+      - relative L2 over the sample of the hard-drop output (routed cells
+        only) and of the SparsePR output;
+      - the O3 split of the hard-drop residual R = dense - hard drop: its
+        least-squares affine fit on [hard-drop output, 1] per head and the
+        remainder; reported as the affine-explainable fraction sum ||P||^2 /
+        sum ||R||^2 and the orthogonal energy sum ||R - P||^2 relative to the
+        dense output's energy (estimated on the sampled rows)."""
     BH, N, d = wl.BH, wl.N, wl.d
     dev = Q.device
     g = torch.Generator().manual_seed(seed)
-    rows = torch.randint(0, N, (min(rows_per_head, N),), generator=g).to(dev)
+    rows = torch.randperm(N, generator=g)[: min(rows_per_head, N)].to(dev)
     perm_q = spr.workspace_tensor(prm, ws, "perm_q", torch.int32, (BH, N)).long()
     inv = torch.empty_like(perm_q)
     inv.scatter_(1, perm_q, torch.arange(N, device=dev).expand(BH, N).contiguous())
     osp = spr.workspace_tensor(prm, ws, "o_sparse", torch.float32, (BH, N, d))
     q, k, v, o = (t.reshape(BH, N, d) for t in (Q, K, V, O))
     scale = 1.0 / d ** 0.5
-    num_hd = num_sp = den = 0.0
+    num_hd = num_sp = den = e_res = e_aff = e_orth = 0.0
     for bh in range(BH):
         s = (q[bh, rows].float() @ k[bh].float().T) * scale
         dense = torch.softmax(s, dim=-1) @ v[bh].float()
@@ -249,8 +257,16 @@ def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=256, seed=0):
         num_hd += float(((hd - dense) ** 2).sum())
         num_sp += float(((sp - dense) ** 2).sum())
         den += float((dense ** 2).sum())
+        R = (dense - hd).double()
+        F = torch.cat([hd.double(), torch.ones(hd.shape[0], 1, dtype=torch.float64, device=dev)], 1)
+        P = F @ torch.linalg.lstsq(F.cpu(), R.cpu()).solution.to(dev)
+        e_res += float((R * R).sum())
+        e_aff += float((P * P).sum())
+        e_orth += float(((R - P) ** 2).sum())
     return {"rows_sampled_per_head": int(rows.numel()), "dense": 0.0,
-            "hard_drop": (num_hd / den) ** 0.5, "sparsepr": (num_sp / den) ** 0.5}
+            "hard_drop": (num_hd / den) ** 0.5, "sparsepr": (num_sp / den) ** 0.5,
+            "o3_affine_fraction": e_aff / e_res if e_res > 0 else 0.0,
+            "o3_orthogonal_energy_rel": e_orth / den}
 
 
 def run_ours(args, wl):
@@ -273,7 +289,8 @@ def run_ours(args, wl):
     O = torch.empty_like(Q)
     prm = spr.make_params(Q, K, V, O, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
                           seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
-                          rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam)
+                          rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
+                          partition=wl.partition)
     ws = spr.alloc_workspace(prm, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -393,10 +410,13 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--partition", default="response", choices=["response", "semantic"],
+                    help="semantic: the raw-row k-means comparator instead of the method's "
+                         "response-coupled partition")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    wl = workload(args.workload)
+    wl = workload(args.workload, partition=args.partition)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

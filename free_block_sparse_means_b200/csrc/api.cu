@@ -50,8 +50,8 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_RMS] = BH * N * 4;
   sz[B_UN2] = BH * N * 4;
   sz[B_CENTQ] = BH * Gq * d * 4;
-  sz[B_BQ16] = BH * 2 * (Gq > d ? Gq : d) * d * 2;
-  sz[B_BETA] = BH * Gq * 4;
+  sz[B_BQ16] = BH * 2 * (Gm > d ? Gm : d) * d * 2;  // semantic mode: key groups too
+  sz[B_BETA] = BH * Gm * 4;
   sz[B_QBAR] = BH * Gq * d * 4;
   sz[B_LOGIT] = BH * Gq * Gk * 4;
   sz[B_ENTRY] = BH * Gq * Gk * 4;
@@ -214,6 +214,8 @@ spr_status sparsepr_check_params(const spr_params* p) {
   if (p->r < 0 || p->r > p->d) return SPR_EINVAL;
   if (!(p->lambda >= 0.0) || !isfinite(p->lambda)) return SPR_EINVAL;
   if (!isfinite(p->scale)) return SPR_EINVAL;
+  if (p->partition != SPR_PARTITION_RESPONSE && p->partition != SPR_PARTITION_SEMANTIC)
+    return SPR_EINVAL;
   return SPR_OK;
 }
 

@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(256) k_gather_rows(TensorView src, const int32
        e += (int64_t)gridDim.x * 256) {
     const int64_t rowi = e / LANES;
     const int c = (int)(e % LANES);
-    const int bh = (int)(rowi / N), i = (int)(rowi % N);
+    const int bh = (int)(rowi / N);
     const int n = perm[rowi];
     reinterpret_cast<uint4*>(dst)[e] = reinterpret_cast<const uint4*>(src.row(bh, n))[c];
   }
@@ -658,6 +658,123 @@ __global__ void k_qprep(const float* A, const float* centq, int G, int D, const 
 }
 
 // ---------------------------------------------------------------------------
+// Semantic partition (the comparator of [paperlayer §2 "Token Partitioning";
+// §3.1 O3]): k-means on the raw key rows and, independently, on the raw query
+// rows.  It runs through the query k-means kernels with A = I (so Bq_g = c_g
+// and beta_g = ||c_g||^2 / 2) and every row's factor scale / rms = 1 (rms set
+// to the scale): the score x . c_g - ||c_g||^2 / 2 ranks groups by distance.
+// ---------------------------------------------------------------------------
+__global__ void k_semantic_setup(float* A, float* rms, int D, int N, float scale) {
+  const int bh = blockIdx.y;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < D * D + N; e += gridDim.x * blockDim.x) {
+    if (e < D * D)
+      A[(size_t)bh * D * D + e] = (e / D == e % D) ? 1.f : 0.f;
+    else
+      rms[(size_t)bh * N + (e - D * D)] = scale;
+  }
+}
+
+// Raw-row k-means objective sum_n ||x_n - c_{lab_n}||^2, fp64 partial per
+// chunk into part[bh][which][chunk] (which = 0 keys, 1 queries).
+template <int D>
+__global__ void __launch_bounds__(256) k_obj_rows(TensorView X, int N, int G, const float* cent,
+                                                  const int32_t* lab, int nchunk, int which,
+                                                  double* part) {
+  __shared__ double red[8];
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  double acc = 0.0;
+  for (int n = chunk * CHUNK + threadIdx.x; n < min(N, (chunk + 1) * CHUNK); n += 256) {
+    const int g = lab[(size_t)bh * N + n];
+    const bf16* x = X.row(bh, n);
+    const float* c = cent + ((size_t)bh * G + g) * D;
+    float s = 0.f;
+    for (int k = 0; k < D; ++k) {
+      const float t = bf2f(x[k]) - c[k];
+      s = fmaf(t, t, s);
+    }
+    acc += s;
+  }
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < 8; ++i) s += red[i];
+    part[((size_t)bh * 2 + which) * (nchunk + 1) + chunk] = s;
+  }
+}
+
+template <int D>
+static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, const Ptrs& P,
+                                        const TensorView& Q, const TensorView& K,
+                                        const TensorView& V, cudaStream_t st) {
+  const int BH = L.BH, N = p.N, nchunk = L.nchunk;
+  const float scale = p.scale > 0.f ? p.scale : 1.f / sqrtf((float)D);
+  const int Gm = p.Gk > p.Gq ? p.Gk : p.Gq;
+  const int split_rows = Gm > D ? Gm : D;
+  const int ggrid = num_sms() * 8;
+  cudaError_t e;
+  spr_launch(k_semantic_setup, dim3(64, BH), 256, 0, st, P.Amat, P.rms, D, N, scale);
+  spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
+  auto lloyd = [&](const TensorView& X, int G, const int32_t* init, float* cent,
+                   int32_t* lab) -> cudaError_t {
+    spr_launch(k_init_centq, BH, 256, 0, st, X, N, G, D, init, P.rms, scale, cent);
+    for (int it = 0; it < p.iters; ++it) {
+      spr_launch(k_qprep, dim3(BH, G), D, 0, st, P.Amat, cent, G, D, P.counts, P.beta, P.bq16,
+                 split_rows, nullptr);
+      KmArgs a{};
+      a.Q = X;
+      a.rms = P.rms;
+      a.scale = scale;
+      a.bsplit = P.bq16;
+      a.split_rows = split_rows;
+      a.beta = P.beta;
+      a.N = N;
+      a.G = G;
+      a.nchunk = nchunk;
+      a.lab = lab;
+      a.chunk_cnt = P.chunk;
+      a.loff = P.cbase;
+      a.part = P.csum;
+      a.hdr = P.hdr;
+      const cudaError_t e2 = launch_kmeans_step(KM_QUERY, D, a, nchunk, BH, st);
+      if (e2 != cudaSuccess) return e2;
+      spr_launch(k_chunk_reduce<D>, dim3(G, BH), D, (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int), st,
+                 P.csum, P.chunk, P.cbase, G, nchunk, cent);
+    }
+    return cudaSuccess;
+  };
+  // K/V groups from the raw keys; the k-means centroids live in Craw until
+  // the group means of the permuted keys replace them
+  if ((e = lloyd(K, p.Gk, P.initk, P.Craw, P.labk)) != cudaSuccess) return e;
+  spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gk, N, P.cbase, P.kvoff, P.counts);
+  spr_launch(k_scatter, dim3(nchunk, BH), CHUNK, 0, st, P.labk, N, p.Gk, nchunk, P.cbase, P.kvoff,
+             P.permk, P.hdr);
+  spr_launch(k_obj_rows<D>, dim3(nchunk, BH), 256, 0, st, K, N, p.Gk, P.Craw, P.labk, nchunk, 0,
+             P.part);
+  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
+  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
+  spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.csum);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.csum, P.kvoff, p.Gk, P.Craw);
+  spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
+  // query groups from the raw queries
+  if ((e = lloyd(Q, p.Gq, P.initq, P.centq, P.labq)) != cudaSuccess) return e;
+  spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gq, N, P.cbase, P.qoff, P.counts);
+  spr_launch(k_scatter, dim3(nchunk, BH), CHUNK, 0, st, P.labq, N, p.Gq, nchunk, P.cbase, P.qoff,
+             P.permq, P.hdr);
+  spr_launch(k_obj_rows<D>, dim3(nchunk, BH), 256, 0, st, Q, N, p.Gq, P.centq, P.labq, nchunk, 1,
+             P.part);
+  // the objective is direct here: no n_g a_g^T A a_g term to subtract
+  if (cudaMemsetAsync(P.part + (size_t)BH * 2 * (nchunk + 1), 0, (size_t)BH * p.Gq * sizeof(double),
+                      st) != cudaSuccess)
+    return cudaGetLastError();
+  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, Q, P.permq, N, BH, P.Qp);
+  spr_launch(k_gmean_part<D>, dim3(p.Gq, BH, GM_SLICES), 256, 0, st, P.Qp, P.qoff, N, p.Gq, P.csum);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gq, BH), D, 0, st, P.csum, P.qoff, p.Gq, P.qbar);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Host orchestration of stage 1.
 // ---------------------------------------------------------------------------
 template <int D>
@@ -778,6 +895,10 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
 cudaError_t launch_partition(const spr_params& p, const Layout& L, const Ptrs& P,
                              const TensorView& Q, const TensorView& K, const TensorView& V,
                              cudaStream_t st) {
+  if (p.partition == SPR_PARTITION_SEMANTIC) {
+    if (p.d == 64) return partition_semantic_d<64>(p, L, P, Q, K, V, st);
+    return partition_semantic_d<128>(p, L, P, Q, K, V, st);
+  }
   if (p.d == 64) return partition_d<64>(p, L, P, Q, K, V, st);
   return partition_d<128>(p, L, P, Q, K, V, st);
 }

@@ -57,6 +57,17 @@ typedef enum {
 enum { SPR_ROUTE_TAU = 0, SPR_ROUTE_BUDGET = 1 };
 
 /*
+ * Partition construction.  SPR_PARTITION_RESPONSE is the method's
+ * Response-Coupled Partitioning.  SPR_PARTITION_SEMANTIC is the comparator the
+ * pages measure it against [paperlayer §2 "Token Partitioning"; §3.1 O3, a
+ * matched comparison]: the same fixed-iteration k-means run on the raw key
+ * rows and, independently, on the raw query rows (Euclidean, same initial
+ * rows, iterations and tie rule), with routing, renormalized hard drop, probes
+ * and reconstruction unchanged.
+ */
+enum { SPR_PARTITION_RESPONSE = 0, SPR_PARTITION_SEMANTIC = 1 };
+
+/*
  * Parameters of one call.  Shapes: B batches, H heads, N tokens (N_q = N_k =
  * N, full-sequence attention [paperlayer §2]), head dim d in {64, 128}.
  *
@@ -83,6 +94,8 @@ typedef struct {
   int32_t M;          /* probe rows per head, 0..min(N, 4096); 0 = hard drop only */
   int32_t r;          /* residual subspace rank, 0..d */
   double lambda;      /* ridge strength (>= 0), weights normalised to sum 1 */
+  int32_t partition;  /* SPR_PARTITION_RESPONSE (0, default) or _SEMANTIC;
+                         semantic mode ignores Ms and p */
 } spr_params;
 
 /* Per-(batch, head) results, copied out by sparsepr_get_stats. */

@@ -51,6 +51,15 @@ Readings (the pages leave these steps open; the plainest reading is taken):
      term is restricted to U_r: the intercept keeps the full weighted mean
      residual; probe rows keep their exact dense value.
   R8 rho_exec counts routed cells and, separately, the M*N_k probe pairs.
+  R11 semantic partition (the comparator of [paperlayer §2 "Token
+     Partitioning"; §3.1 O3]): the R3 k-means run on the raw key rows and,
+     independently, on the raw query rows, with the same initial rows,
+     iteration count and tie rule; routing, hard drop, probes and the fit are
+     unchanged (the pages' matched comparison).
+  R12 O3 decomposition: the residual is dense minus hard-drop output over the
+     rows given; its affine part is the least-squares fit of the residual on
+     [sparse output, 1] (every output column jointly), the orthogonal part the
+     remainder.
 """
 from __future__ import annotations
 
@@ -65,7 +74,7 @@ __all__ = [
     "kv_centroids", "query_response_coords", "group_major_permutation",
     "route_logits", "route_masses", "route_select", "route_to_csr",
     "select_probes", "hard_drop_attention", "fit_residual", "apply_correction",
-    "rho_exec", "sparsepr_head", "sparsepr_call",
+    "rho_exec", "sparsepr_head", "sparsepr_call", "affine_residual_decomposition",
 ]
 
 MASK64 = (1 << 64) - 1
@@ -91,6 +100,7 @@ class Params:
     seed: int = 0
     scale: float | None = None  # default 1/sqrt(d)
     weight_power: float = 0.5
+    partition: str = "response"  # "response" | "semantic" (reading R11)
 
 
 # ---------------------------------------------------------------------------
@@ -494,31 +504,50 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
     N, d = Q.shape
     s = prm.scale if prm.scale is not None else 1.0 / np.sqrt(d)
     out = {"scale": s}
-    # Key-response coordinates and paired K/V groups
-    qs_idx = sample_query_indices(N, prm.Ms)
-    MK = response_metric(Q[qs_idx])
-    W, lamk = key_response_weights(MK, prm.p, prm.weight_power)
-    Z = K @ W
-    out.update(MK=MK, W=W, eig_MK=lamk, Z=Z)
-    if lab_k is None:
-        init_k = kmeans_init_indices(K.shape[0], prm.Gk, prm.seed, bh, 0)
-        lab_k, _, _, hist_k = kmeans(Z, prm.Gk, prm.iters, init_k)
-        out["kmeans_k_hist"] = hist_k
-    lab_k = np.asarray(lab_k, np.int64)
-    Cz = group_means(Z, lab_k, prm.Gk)
-    ne_k = np.bincount(lab_k, minlength=prm.Gk) > 0
-    out["obj_k"] = kmeans_objective(Z, lab_k, np.where(ne_k[:, None], Cz, 0.0))
-    C, counts_k = kv_centroids(K, lab_k, prm.Gk)
-    # Query-response coordinates and query groups
-    Uq, rms, Ct = query_response_coords(Q, C, counts_k, s)
-    if lab_q is None:
-        init_q = kmeans_init_indices(N, prm.Gq, prm.seed, bh, 1)
-        lab_q, _, _, hist_q = kmeans(Uq, prm.Gq, prm.iters, init_q)
-        out["kmeans_q_hist"] = hist_q
-    lab_q = np.asarray(lab_q, np.int64)
-    Cu = group_means(Uq, lab_q, prm.Gq)
-    ne_q = np.bincount(lab_q, minlength=prm.Gq) > 0
-    out["obj_q"] = kmeans_objective(Uq, lab_q, np.where(ne_q[:, None], Cu, 0.0))
+    if prm.partition == "semantic":
+        # Semantic comparator (reading R11): k-means on the raw rows
+        if lab_k is None:
+            init_k = kmeans_init_indices(K.shape[0], prm.Gk, prm.seed, bh, 0)
+            lab_k, _, _, hist_k = kmeans(K, prm.Gk, prm.iters, init_k)
+            out["kmeans_k_hist"] = hist_k
+        lab_k = np.asarray(lab_k, np.int64)
+        C, counts_k = kv_centroids(K, lab_k, prm.Gk)
+        out["obj_k"] = kmeans_objective(K, lab_k, np.where((counts_k > 0)[:, None], C, 0.0))
+        if lab_q is None:
+            init_q = kmeans_init_indices(N, prm.Gq, prm.seed, bh, 1)
+            lab_q, _, _, hist_q = kmeans(Q, prm.Gq, prm.iters, init_q)
+            out["kmeans_q_hist"] = hist_q
+        lab_q = np.asarray(lab_q, np.int64)
+        Cu = group_means(Q, lab_q, prm.Gq)
+        ne_q = np.bincount(lab_q, minlength=prm.Gq) > 0
+        out["obj_q"] = kmeans_objective(Q, lab_q, np.where(ne_q[:, None], Cu, 0.0))
+        rms, Ct = None, None
+    else:
+        # Key-response coordinates and paired K/V groups
+        qs_idx = sample_query_indices(N, prm.Ms)
+        MK = response_metric(Q[qs_idx])
+        W, lamk = key_response_weights(MK, prm.p, prm.weight_power)
+        Z = K @ W
+        out.update(MK=MK, W=W, eig_MK=lamk, Z=Z)
+        if lab_k is None:
+            init_k = kmeans_init_indices(K.shape[0], prm.Gk, prm.seed, bh, 0)
+            lab_k, _, _, hist_k = kmeans(Z, prm.Gk, prm.iters, init_k)
+            out["kmeans_k_hist"] = hist_k
+        lab_k = np.asarray(lab_k, np.int64)
+        Cz = group_means(Z, lab_k, prm.Gk)
+        ne_k = np.bincount(lab_k, minlength=prm.Gk) > 0
+        out["obj_k"] = kmeans_objective(Z, lab_k, np.where(ne_k[:, None], Cz, 0.0))
+        C, counts_k = kv_centroids(K, lab_k, prm.Gk)
+        # Query-response coordinates and query groups
+        Uq, rms, Ct = query_response_coords(Q, C, counts_k, s)
+        if lab_q is None:
+            init_q = kmeans_init_indices(N, prm.Gq, prm.seed, bh, 1)
+            lab_q, _, _, hist_q = kmeans(Uq, prm.Gq, prm.iters, init_q)
+            out["kmeans_q_hist"] = hist_q
+        lab_q = np.asarray(lab_q, np.int64)
+        Cu = group_means(Uq, lab_q, prm.Gq)
+        ne_q = np.bincount(lab_q, minlength=prm.Gq) > 0
+        out["obj_q"] = kmeans_objective(Uq, lab_q, np.where(ne_q[:, None], Cu, 0.0))
     out.update(lab_k=lab_k, lab_q=lab_q, C=C, counts_k=counts_k, rms=rms, Ctilde=Ct,
                Cu=Cu)
     # Group-major layouts
@@ -565,6 +594,27 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
     if want_dense:
         out["O_dense"] = dense_attention(Q[want], K, V, s)
     return out
+
+
+def affine_residual_decomposition(O_sparse, O_dense):
+    """O3 diagnostic [paperlayer §3.1 O3]; reading R12.
+
+    R = O_dense - O_sparse.  Its affine part P is the least-squares fit of R
+    on the features [O_sparse, 1] (one coefficient matrix for all output
+    columns), the orthogonal part E = R - P.  Returns a dict with the
+    residual, affine and orthogonal energies (squared Frobenius norms) and the
+    affine-explainable fraction ||P||^2 / ||R||^2.  It needs the full dense
+    residual, so it is a diagnostic of a partition, not part of execution.
+    """
+    X = np.asarray(O_sparse, np.float64)
+    R = np.asarray(O_dense, np.float64) - X
+    F = np.concatenate([X, np.ones((X.shape[0], 1))], axis=1)
+    beta, *_ = np.linalg.lstsq(F, R, rcond=None)
+    P = F @ beta
+    E = R - P
+    er, ep, eo = float((R * R).sum()), float((P * P).sum()), float((E * E).sum())
+    return {"residual_energy": er, "affine_energy": ep, "orthogonal_energy": eo,
+            "affine_fraction": ep / er if er > 0 else 0.0}
 
 
 def sparsepr_call(Q, K, V, prm: Params, **kw):

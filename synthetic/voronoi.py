@@ -45,6 +45,7 @@ class Workload:
     r: int
     lam: float
     center_scale: float = 2.0
+    partition: str = "response"  # or "semantic" (the comparator)
 
     @property
     def N(self) -> int:

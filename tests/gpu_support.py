@@ -33,20 +33,25 @@ def oracle_params(wl, **kw) -> Params:
     return Params(**d)
 
 
-def run_gpu(wl, N=None, heads=None, inputs=None, check=None):
+def run_gpu(wl, N=None, heads=None, inputs=None, check=None, partition=None):
     """Run sparsepr_call on cuda:0; return a dict of CPU numpy results (for
-    every head, or only for the head indices in `check`)."""
+    every head, or only for the head indices in `check`).  The partition
+    construction is the workload's unless given."""
+    partition = partition or wl.partition
     Q, K, V = inputs if inputs is not None else voronoi_qkv(wl, heads=heads, N=N)
     Qd, Kd, Vd = (t.cuda() for t in (Q, K, V))
     Od = torch.empty_like(Qd)
     prm = spr.make_params(Qd, Kd, Vd, Od, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
                           seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
-                          rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam)
+                          rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
+                          partition=partition)
     ws = spr.alloc_workspace(prm)
     spr.sparsepr_call(prm, Qd, Kd, Vd, Od, ws)
     stats, err = spr.sparsepr_get_stats(prm, ws)
     assert err == 0
-    return collect(prm, ws, Q, K, V, Od, stats, check)
+    g = collect(prm, ws, Q, K, V, Od, stats, check)
+    g["partition"] = partition
+    return g
 
 
 def collect(prm, ws, Q, K, V, Od, stats, check=None):
@@ -126,7 +131,7 @@ def fragile_cells(orc, wl, gpu_thr, live):
 
 def check_head(g, wl, bh, rows=None, report=None):
     """Driven-mode oracle for one head and every comparison of the contract."""
-    prm = oracle_params(wl)
+    prm = oracle_params(wl, partition=g.get("partition", "response"))
     q, k, v = (g[n][bh].double().numpy() for n in ("Q", "K", "V"))
     lab_k, lab_q = g["lab_k"][bh].astype(np.int64), g["lab_q"][bh].astype(np.int64)
     orc = sparsepr_head(q, k, v, prm, bh=bh, lab_k=lab_k, lab_q=lab_q, rows=rows)
