@@ -292,10 +292,16 @@ def run_ours(args, wl):
                           rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
                           partition=wl.partition)
     ws = spr.alloc_workspace(prm, device=dev)
+    prm_seeded = prm
+    if args.warm_iters > 0:  # every call after the first starts from the previous centroids
+        prm = spr.make_params(Q, K, V, O, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq,
+                              iters=args.warm_iters, seed=wl.index, route_mode=wl.route_mode,
+                              tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
+                              partition=wl.partition, init="warm")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def call_staged(ev=None):
+    def call_staged(ev=None, prm=prm):
         if ev is not None:
             ev[0].record(stream)
         spr.sparsepr_partition(prm, Q, K, V, ws, stream)
@@ -311,9 +317,9 @@ def run_ours(args, wl):
         if ev is not None:
             ev[4].record(stream)
 
-    for _ in range(args.warmup):
+    for w in range(args.warmup):
         flush.zero_()
-        call_staged()
+        call_staged(prm=prm_seeded if w == 0 else prm)
     torch.cuda.synchronize(dev)
     stats, err = spr.sparsepr_get_stats(prm, ws, stream)
     if err:
@@ -379,7 +385,11 @@ def run_ours(args, wl):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_call, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 (fp32 accumulate)", "data": "synthetic",
-            "config": config_of(wl, world), "ms_per_call": ms_per_call,
+            "config": dict(config_of(wl, world), **(
+                {"iters": args.warm_iters,
+                 "kmeans_start": "warm (previous call's centroids; first warm-up call seeded)"}
+                if args.warm_iters > 0 else {"kmeans_start": "seeded"})),
+            "ms_per_call": ms_per_call,
             "exec_pair_tflops": exec_tflops * world, "rho_exec": rho,
             "stage_ms": {"partition": stage_max[0], "route": stage_max[1], "attend": stage_max[2],
                          "reconstruct": stage_max[3]},
@@ -410,6 +420,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--warm-iters", type=int, default=0,
+                    help="T > 0: the first warm-up call is seeded, every later call starts its "
+                         "k-means from the previous call's centroids and runs T iterations")
     ap.add_argument("--partition", default="response", choices=["response", "semantic"],
                     help="semantic: the raw-row k-means comparator instead of the method's "
                          "response-coupled partition")

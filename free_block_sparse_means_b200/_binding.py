@@ -20,6 +20,7 @@ STATUS_NAMES = {0: "SPR_OK", 1: "SPR_EINVAL", 2: "SPR_EUNSUPPORTED", 3: "SPR_EWO
                 4: "SPR_ECUDA", 5: "SPR_EDEVICE", 6: "SPR_ESCRATCH"}
 ROUTE_TAU, ROUTE_BUDGET = 0, 1
 PARTITION_RESPONSE, PARTITION_SEMANTIC = 0, 1
+INIT_SEEDED, INIT_WARM = 0, 1
 
 VIEWS = {
     "lab_k": 0, "lab_q": 1, "perm_k": 2, "perm_q": 3, "kv_off": 4, "q_off": 5, "row_ptr": 6,
@@ -42,7 +43,7 @@ class SprParams(ctypes.Structure):
         ("tau", ctypes.c_double), ("rho_target", ctypes.c_double),
         ("M", ctypes.c_int32), ("r", ctypes.c_int32),
         ("lambda_", ctypes.c_double),
-        ("partition", ctypes.c_int32),
+        ("partition", ctypes.c_int32), ("init", ctypes.c_int32),
     ]
 
 
@@ -126,7 +127,7 @@ def _strides(t: torch.Tensor):
 
 def make_params(Q, K=None, V=None, O=None, *, Ms, p, Gk, Gq, iters=10, seed=0, route_mode="tau",
                 tau=0.9, rho_target=0.25, M=64, r=8, lam=1e-3, scale=0.0,
-                partition="response") -> SprParams:
+                partition="response", init="seeded") -> SprParams:
     """spr_params for tensors shaped [B, H, N, d] (strides taken from them)."""
     B, H, N, d = Q.shape
     prm = SprParams()
@@ -143,6 +144,9 @@ def make_params(Q, K=None, V=None, O=None, *, Ms, p, Gk, Gq, iters=10, seed=0, r
     if partition not in ("response", "semantic"):
         raise ValueError(f"partition must be 'response' or 'semantic', not {partition!r}")
     prm.partition = PARTITION_RESPONSE if partition == "response" else PARTITION_SEMANTIC
+    if init not in ("seeded", "warm"):
+        raise ValueError(f"init must be 'seeded' or 'warm', not {init!r}")
+    prm.init = INIT_SEEDED if init == "seeded" else INIT_WARM
     return prm
 
 

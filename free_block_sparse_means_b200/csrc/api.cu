@@ -216,6 +216,7 @@ spr_status sparsepr_check_params(const spr_params* p) {
   if (!isfinite(p->scale)) return SPR_EINVAL;
   if (p->partition != SPR_PARTITION_RESPONSE && p->partition != SPR_PARTITION_SEMANTIC)
     return SPR_EINVAL;
+  if (p->init != SPR_INIT_SEEDED && p->init != SPR_INIT_WARM) return SPR_EINVAL;
   return SPR_OK;
 }
 

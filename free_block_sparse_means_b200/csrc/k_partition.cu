@@ -136,6 +136,21 @@ __global__ void k_init_centk(const float* Z, int N, int G, int PP, const int32_t
   }
 }
 
+// Warm start of the key k-means [paperlayer App. C.1]: the previous call's
+// raw-key group means in this call's key-response coordinates,
+// c_g = W^T Craw_g (z = W^T k is linear; zero columns of W give zeros).
+__global__ void k_warm_centk(const float* Craw, const float* W, int G, int D, int PP, float* cent) {
+  const int bh = blockIdx.x;
+  for (int e = threadIdx.x; e < G * PP; e += blockDim.x) {
+    const int g = e / PP, k = e % PP;
+    const float* c = Craw + ((size_t)bh * G + g) * D;
+    const float* w = W + (size_t)bh * D * PP + k;
+    float s = 0.f;
+    for (int i = 0; i < D; ++i) s = fmaf(c[i], w[(size_t)i * PP], s);
+    cent[(size_t)bh * G * PP + e] = s;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // ---------------------------------------------------------------------------
 // Per (bh, g): base of each chunk within the group (exclusive scan over
@@ -718,7 +733,8 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
   spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
   auto lloyd = [&](const TensorView& X, int G, const int32_t* init, float* cent,
                    int32_t* lab) -> cudaError_t {
-    spr_launch(k_init_centq, BH, 256, 0, st, X, N, G, D, init, P.rms, scale, cent);
+    if (p.init != SPR_INIT_WARM)  // warm: cent holds the previous call's raw-row centroids
+      spr_launch(k_init_centq, BH, 256, 0, st, X, N, G, D, init, P.rms, scale, cent);
     for (int it = 0; it < p.iters; ++it) {
       spr_launch(k_qprep, dim3(BH, G), D, 0, st, P.Amat, cent, G, D, P.counts, P.beta, P.bq16,
                  split_rows, nullptr);
@@ -791,7 +807,10 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   spr_launch(k_keyweights, BH, 256, 0, st, P.eval, P.evec, P.trace, D, p.p, pp, P.W);
   if ((e = launch_project(K, N, D, pp, BH, P.W, P.Z, P.hdr, st)) != cudaSuccess) return e;
   spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
-  spr_launch(k_init_centk, BH, 256, 0, st, P.Z, N, p.Gk, pp, P.initk, P.centk);
+  if (p.init == SPR_INIT_WARM)  // the previous call's centroids, mapped (Craw still holds them)
+    spr_launch(k_warm_centk, BH, 256, 0, st, P.Craw, P.W, p.Gk, D, pp, P.centk);
+  else
+    spr_launch(k_init_centk, BH, 256, 0, st, P.Z, N, p.Gk, pp, P.initk, P.centk);
   // Key k-means
   for (int it = 0; it < p.iters; ++it) {
     KmArgs ka{};
@@ -855,7 +874,8 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
     spr_launch(k_rowgemm<D, true>, dim3(nchunk, BH), 256, sm, st, ra);
   }
   // Query k-means in the head dimension
-  spr_launch(k_init_centq, BH, 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale, P.centq);
+  if (p.init != SPR_INIT_WARM)  // warm: centq keeps the previous call's head-dim centroids
+    spr_launch(k_init_centq, BH, 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale, P.centq);
   for (int it = 0; it < p.iters; ++it) {
     spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
                                           split_rows, nullptr);

@@ -68,6 +68,20 @@ enum { SPR_ROUTE_TAU = 0, SPR_ROUTE_BUDGET = 1 };
 enum { SPR_PARTITION_RESPONSE = 0, SPR_PARTITION_SEMANTIC = 1 };
 
 /*
+ * k-means start [paperlayer App. C.1 names a warm-started GPU k-means].
+ * SPR_INIT_SEEDED: G distinct rows from the splitmix64 partial shuffle of
+ * `seed`.  SPR_INIT_WARM: the centroids the previous call left in the same
+ * workspace: its raw-key group means (zero for an empty group) mapped into
+ * this call's key-response coordinates by W (z = W^T k is linear), and its
+ * query centroids kept in head-dimension form a_g = mean of (s / rms) q
+ * (semantic mode: the raw-row centroids of both sides).  A warm call needs a
+ * workspace whose last completed call had the same B, H, N, d, Gk, Gq, p and
+ * partition; otherwise its starting centroids are whatever the workspace
+ * holds (the call still completes; only the clustering is affected).
+ */
+enum { SPR_INIT_SEEDED = 0, SPR_INIT_WARM = 1 };
+
+/*
  * Parameters of one call.  Shapes: B batches, H heads, N tokens (N_q = N_k =
  * N, full-sequence attention [paperlayer §2]), head dim d in {64, 128}.
  *
@@ -96,6 +110,7 @@ typedef struct {
   double lambda;      /* ridge strength (>= 0), weights normalised to sum 1 */
   int32_t partition;  /* SPR_PARTITION_RESPONSE (0, default) or _SEMANTIC;
                          semantic mode ignores Ms and p */
+  int32_t init;       /* SPR_INIT_SEEDED (0, default) or SPR_INIT_WARM */
 } spr_params;
 
 /* Per-(batch, head) results, copied out by sparsepr_get_stats. */

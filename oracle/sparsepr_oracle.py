@@ -60,6 +60,13 @@ Readings (the pages leave these steps open; the plainest reading is taken):
      rows given; its affine part is the least-squares fit of the residual on
      [sparse output, 1] (every output column jointly), the orthogonal part the
      remainder.
+  R13 warm start (the pages name a warm-started GPU k-means [paperlayer App.
+     C.1] and nothing more): a call's two k-means start from the previous
+     call's centroids instead of seeded rows: the previous raw-key group
+     means (zero for an empty group) mapped into this call's key-response
+     coordinates (z = W^T k is linear, so means map by W), and the previous
+     query centroids kept in head-dimension form a_g = mean of (s / rms) q,
+     whose query-response coordinates are Ctilde a_g.
 """
 from __future__ import annotations
 
@@ -194,23 +201,39 @@ def _sqdist(X, C):
     return (X * X).sum(1)[:, None] - 2.0 * (X @ C.T) + (C * C).sum(1)[None, :]
 
 
-def kmeans(X, G, iters, init_idx):
+def kmeans(X, G, iters, init_idx=None, init_centroids=None, payload=None, payload_init=None):
     """Lloyd's k-means with a fixed iteration count (reading R3).
 
     Each iteration assigns every row to its nearest centroid (ties to the lower
     index; numpy's argmin returns the first minimum) and then replaces each
     centroid by the mean of its rows; an empty cluster keeps its centroid.
-    Returns (labels, centroids, objective, objective_per_iteration).
+    The start is the rows ``init_idx`` (seeded) or ``init_centroids`` (a warm
+    start, reading R13).  ``payload`` rows, if given, get the same update
+    (group means under the same labels, empty groups keep theirs, starting
+    from ``payload_init``): the centroids in another representation of the
+    rows.  Returns (labels, centroids, objective, objective_per_iteration),
+    plus the payload centroids when a payload is given.
     """
     X = np.asarray(X, np.float64)
-    C = X[np.asarray(init_idx)].copy()
+    if init_centroids is not None:
+        C = np.array(init_centroids, np.float64)
+    else:
+        C = X[np.asarray(init_idx)].copy()
+    Pc = None
+    if payload is not None:
+        payload = np.asarray(payload, np.float64)
+        Pc = (np.array(payload_init, np.float64) if payload_init is not None
+              else payload[np.asarray(init_idx)].copy())
     lab = np.zeros(X.shape[0], np.int64)
     hist = []
     for _ in range(iters):
         lab = np.argmin(_sqdist(X, C), axis=1)
         C = group_means(X, lab, G, fallback=C)
+        if payload is not None:
+            Pc = group_means(payload, lab, G, fallback=Pc)
         hist.append(kmeans_objective(X, lab, C))
-    return lab, C, (hist[-1] if hist else kmeans_objective(X, lab, C)), hist
+    res = (lab, C, (hist[-1] if hist else kmeans_objective(X, lab, C)), hist)
+    return res + (Pc,) if payload is not None else res
 
 
 def kmeans_objective(X, lab, C):
@@ -489,13 +512,15 @@ def rho_exec(counts_q, counts_k, row_ptr, col_idx, M):
 # Whole call
 # ---------------------------------------------------------------------------
 def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
-                  rows=None, want_dense=False):
+                  rows=None, want_dense=False, warm=None):
     """One (batch, head) SparsePR call, fp64, following the pages' order.
 
     Driven mode: ``lab_k`` / ``lab_q`` (and optionally ``csr``) replace the
     oracle's own clustering (routing) so that everything downstream is
     recomputed from given assignments.  ``rows`` limits the routed attention
     and the output to those original rows (probe rows are always computed).
+    ``warm`` (reading R13) is the ``warm_state`` a previous call returned:
+    both k-means then start from its centroids instead of seeded rows.
     Returns a dict of every intermediate.
     """
     Q = np.asarray(Q, np.float64)
@@ -506,16 +531,19 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
     out = {"scale": s}
     if prm.partition == "semantic":
         # Semantic comparator (reading R11): k-means on the raw rows
+        a_q = None
         if lab_k is None:
             init_k = kmeans_init_indices(K.shape[0], prm.Gk, prm.seed, bh, 0)
-            lab_k, _, _, hist_k = kmeans(K, prm.Gk, prm.iters, init_k)
+            lab_k, _, _, hist_k = kmeans(K, prm.Gk, prm.iters, init_k,
+                                         init_centroids=None if warm is None else warm["C_raw"])
             out["kmeans_k_hist"] = hist_k
         lab_k = np.asarray(lab_k, np.int64)
         C, counts_k = kv_centroids(K, lab_k, prm.Gk)
         out["obj_k"] = kmeans_objective(K, lab_k, np.where((counts_k > 0)[:, None], C, 0.0))
         if lab_q is None:
             init_q = kmeans_init_indices(N, prm.Gq, prm.seed, bh, 1)
-            lab_q, _, _, hist_q = kmeans(Q, prm.Gq, prm.iters, init_q)
+            lab_q, a_q, _, hist_q = kmeans(Q, prm.Gq, prm.iters, init_q,
+                                           init_centroids=None if warm is None else warm["a_q"])
             out["kmeans_q_hist"] = hist_q
         lab_q = np.asarray(lab_q, np.int64)
         Cu = group_means(Q, lab_q, prm.Gq)
@@ -529,9 +557,14 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
         W, lamk = key_response_weights(MK, prm.p, prm.weight_power)
         Z = K @ W
         out.update(MK=MK, W=W, eig_MK=lamk, Z=Z)
+        a_q = None
         if lab_k is None:
             init_k = kmeans_init_indices(K.shape[0], prm.Gk, prm.seed, bh, 0)
-            lab_k, _, _, hist_k = kmeans(Z, prm.Gk, prm.iters, init_k)
+            # warm start: the previous raw-key means in today's coordinates
+            # (z = W^T k is linear, so a group mean maps by W as well)
+            lab_k, _, _, hist_k = kmeans(
+                Z, prm.Gk, prm.iters, init_k,
+                init_centroids=None if warm is None else np.asarray(warm["C_raw"]) @ W)
             out["kmeans_k_hist"] = hist_k
         lab_k = np.asarray(lab_k, np.int64)
         Cz = group_means(Z, lab_k, prm.Gk)
@@ -542,7 +575,14 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
         Uq, rms, Ct = query_response_coords(Q, C, counts_k, s)
         if lab_q is None:
             init_q = kmeans_init_indices(N, prm.Gq, prm.seed, bh, 1)
-            lab_q, _, _, hist_q = kmeans(Uq, prm.Gq, prm.iters, init_q)
+            # the centroids are carried along in head-dimension form as the
+            # means of (s / rms) q (u = s Ctilde q / rms, so m = Ctilde a):
+            # that form is what survives to the next call's coordinates
+            Qf = (s / rms)[:, None] * Q
+            a0 = None if warm is None else np.asarray(warm["a_q"])
+            lab_q, _, _, hist_q, a_q = kmeans(
+                Uq, prm.Gq, prm.iters, init_q,
+                init_centroids=None if a0 is None else a0 @ Ct.T, payload=Qf, payload_init=a0)
             out["kmeans_q_hist"] = hist_q
         lab_q = np.asarray(lab_q, np.int64)
         Cu = group_means(Uq, lab_q, prm.Gq)
@@ -550,6 +590,10 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
         out["obj_q"] = kmeans_objective(Uq, lab_q, np.where(ne_q[:, None], Cu, 0.0))
     out.update(lab_k=lab_k, lab_q=lab_q, C=C, counts_k=counts_k, rms=rms, Ctilde=Ct,
                Cu=Cu)
+    # what a warm-started next call starts from (reading R13): raw-key group
+    # means (zero for an empty group) and the query centroids in head-dim form
+    out["warm_state"] = {"C_raw": np.where((counts_k > 0)[:, None], np.nan_to_num(C), 0.0),
+                         "a_q": a_q}
     # Group-major layouts
     perm_k, kv_off = group_major_permutation(lab_k, prm.Gk)
     perm_q, q_off = group_major_permutation(lab_q, prm.Gq)
