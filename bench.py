@@ -171,7 +171,7 @@ def oracle_head_seconds(wl, bh):
     from oracle import Params, sparsepr_head
     prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
                  tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index,
-                 partition=wl.partition)
+                 partition=wl.partition, weights=wl.weights)
     Q, K, V = voronoi_qkv(wl, heads=[bh])
     q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
     t0 = time.perf_counter()
@@ -199,6 +199,7 @@ def config_of(wl, world):
             "routing": (f"budget rho_target={wl.rho_target}" if wl.route_mode == "budget"
                         else f"tau={wl.tau}"),
             "M": wl.M, "r": wl.r, "lambda": wl.lam, "partition": wl.partition,
+            "probe_weights": wl.weights,
             "parallelism": f"heads x{world} (weak)",
             "l2": "flushed (256 MiB write) before every timed call"}
 
@@ -290,14 +291,14 @@ def run_ours(args, wl):
     prm = spr.make_params(Q, K, V, O, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
                           seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
                           rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
-                          partition=wl.partition)
+                          partition=wl.partition, weights=wl.weights)
     ws = spr.alloc_workspace(prm, device=dev)
     prm_seeded = prm
     if args.warm_iters > 0:  # every call after the first starts from the previous centroids
         prm = spr.make_params(Q, K, V, O, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq,
                               iters=args.warm_iters, seed=wl.index, route_mode=wl.route_mode,
                               tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
-                              partition=wl.partition, init="warm")
+                              partition=wl.partition, weights=wl.weights, init="warm")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -423,13 +424,19 @@ def main(argv=None):
     ap.add_argument("--warm-iters", type=int, default=0,
                     help="T > 0: the first warm-up call is seeded, every later call starts its "
                          "k-means from the previous call's centroids and runs T iterations")
+    ap.add_argument("--weights", default="coverage", choices=["coverage", "uniform"],
+                    help="uniform: the unweighted estimator of the ablation")
+    ap.add_argument("--rank", type=int, default=0,
+                    help="r of the residual fit (0: the workload's; d: no subspace restriction)")
     ap.add_argument("--partition", default="response", choices=["response", "semantic"],
                     help="semantic: the raw-row k-means comparator instead of the method's "
                          "response-coupled partition")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    wl = workload(args.workload, partition=args.partition)
+    wl = workload(args.workload, partition=args.partition, weights=args.weights)
+    if args.rank > 0:
+        wl = wl.replace(r=args.rank)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

@@ -21,6 +21,7 @@ STATUS_NAMES = {0: "SPR_OK", 1: "SPR_EINVAL", 2: "SPR_EUNSUPPORTED", 3: "SPR_EWO
 ROUTE_TAU, ROUTE_BUDGET = 0, 1
 PARTITION_RESPONSE, PARTITION_SEMANTIC = 0, 1
 INIT_SEEDED, INIT_WARM = 0, 1
+WEIGHTS_COVERAGE, WEIGHTS_UNIFORM = 0, 1
 
 VIEWS = {
     "lab_k": 0, "lab_q": 1, "perm_k": 2, "perm_q": 3, "kv_off": 4, "q_off": 5, "row_ptr": 6,
@@ -43,7 +44,7 @@ class SprParams(ctypes.Structure):
         ("tau", ctypes.c_double), ("rho_target", ctypes.c_double),
         ("M", ctypes.c_int32), ("r", ctypes.c_int32),
         ("lambda_", ctypes.c_double),
-        ("partition", ctypes.c_int32), ("init", ctypes.c_int32),
+        ("partition", ctypes.c_int32), ("init", ctypes.c_int32), ("weights", ctypes.c_int32),
     ]
 
 
@@ -127,7 +128,7 @@ def _strides(t: torch.Tensor):
 
 def make_params(Q, K=None, V=None, O=None, *, Ms, p, Gk, Gq, iters=10, seed=0, route_mode="tau",
                 tau=0.9, rho_target=0.25, M=64, r=8, lam=1e-3, scale=0.0,
-                partition="response", init="seeded") -> SprParams:
+                partition="response", init="seeded", weights="coverage") -> SprParams:
     """spr_params for tensors shaped [B, H, N, d] (strides taken from them)."""
     B, H, N, d = Q.shape
     prm = SprParams()
@@ -147,6 +148,9 @@ def make_params(Q, K=None, V=None, O=None, *, Ms, p, Gk, Gq, iters=10, seed=0, r
     if init not in ("seeded", "warm"):
         raise ValueError(f"init must be 'seeded' or 'warm', not {init!r}")
     prm.init = INIT_SEEDED if init == "seeded" else INIT_WARM
+    if weights not in ("coverage", "uniform"):
+        raise ValueError(f"weights must be 'coverage' or 'uniform', not {weights!r}")
+    prm.weights = WEIGHTS_COVERAGE if weights == "coverage" else WEIGHTS_UNIFORM
     return prm
 
 

@@ -217,6 +217,7 @@ spr_status sparsepr_check_params(const spr_params* p) {
   if (p->partition != SPR_PARTITION_RESPONSE && p->partition != SPR_PARTITION_SEMANTIC)
     return SPR_EINVAL;
   if (p->init != SPR_INIT_SEEDED && p->init != SPR_INIT_WARM) return SPR_EINVAL;
+  if (p->weights != SPR_WEIGHTS_COVERAGE && p->weights != SPR_WEIGHTS_UNIFORM) return SPR_EINVAL;
   return SPR_OK;
 }
 

@@ -297,12 +297,14 @@ __global__ void __launch_bounds__(256) k_route_csr(const uint8_t* sel, const int
   }
 }
 
-// Stratified probes with coverage weights (reading R6).  Grid BH, block 256.
+// Stratified probes with coverage weights (reading R6), or every probe
+// weighing 1 / (probes selected) when `uniform`.  Grid BH, block 256.
 // pslot[bh][pos] receives the probe slot of each probed permuted position (the
 // caller fills it with -1 first).
 __global__ void __launch_bounds__(256) k_probes(const int32_t* qoff, const int32_t* permq, int Gq,
-                                                int N, int M, int32_t* ppos, int32_t* pidx,
-                                                float* pw, int32_t* pslot, spr_head_stats* stats) {
+                                                int N, int M, int uniform, int32_t* ppos,
+                                                int32_t* pidx, float* pw, int32_t* pslot,
+                                                spr_head_stats* stats) {
   __shared__ int sh[32];
   __shared__ long long shl[32];
   __shared__ long long rems[MAX_GROUPS];
@@ -344,11 +346,14 @@ __global__ void __launch_bounds__(256) k_probes(const int32_t* qoff, const int32
   __syncthreads();
   const long long covered =
       block_reduce(m > 0 ? (long long)cnt : 0ll, shl, [](long long a, long long b) { return a + b; });
+  const long long nsel =
+      block_reduce((long long)m, shl, [](long long a, long long b) { return a + b; });
   int base;
   block_exscan((int)m, sh, &base);
   if (g < Gq && m > 0) {
     const int q0 = qoff[(size_t)bh * (Gq + 1) + g];
-    const float w = (float)(((double)cnt / (double)m) / (double)covered);
+    const float w = uniform ? (float)(1.0 / (double)min(nsel, (long long)M))
+                            : (float)(((double)cnt / (double)m) / (double)covered);
     for (int t = 0; t < (int)m && base + t < M; ++t) {
       const int pos = q0 + (int)(((2ll * t + 1) * cnt) / (2 * m));
       ppos[(size_t)bh * M + base + t] = pos;
@@ -435,7 +440,8 @@ cudaError_t launch_route(const spr_params& p, const Layout& L, const Ptrs& P, cu
                                   P.runptr, P.runs, P.stats);
   if (cudaMemsetAsync(P.pslot, 0xFF, (size_t)BH * p.N * sizeof(int32_t), st) != cudaSuccess)
     return cudaGetLastError();
-  spr_launch(k_probes, BH, 256, 0, st, P.qoff, P.permq, p.Gq, p.N, p.M, P.ppos, P.pidx, P.pw,
+  spr_launch(k_probes, BH, 256, 0, st, P.qoff, P.permq, p.Gq, p.N, p.M,
+             p.weights == SPR_WEIGHTS_UNIFORM ? 1 : 0, P.ppos, P.pidx, P.pw,
              P.pslot, P.stats);
   if (p.M > 0) {
     const int grid = num_sms() * 4;

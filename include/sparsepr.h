@@ -82,6 +82,17 @@ enum { SPR_PARTITION_RESPONSE = 0, SPR_PARTITION_SEMANTIC = 1 };
 enum { SPR_INIT_SEEDED = 0, SPR_INIT_WARM = 1 };
 
 /*
+ * Probe weights of the residual fit.  SPR_WEIGHTS_COVERAGE is the method's
+ * coverage weighting [paperlayer §4 "Probe-Fitted Residual Reconstruction"]:
+ * a probe of query group g weighs |Q_g| / m_g, normalised to sum 1.
+ * SPR_WEIGHTS_UNIFORM weighs every probe 1 / M: the unweighted estimator of
+ * the probe-selection / estimator ablation [paperlayer §5 "Ablations",
+ * Table 4].  (The same ablation's estimator without the subspace restriction
+ * is r = d: the basis then spans the whole output space.)
+ */
+enum { SPR_WEIGHTS_COVERAGE = 0, SPR_WEIGHTS_UNIFORM = 1 };
+
+/*
  * Parameters of one call.  Shapes: B batches, H heads, N tokens (N_q = N_k =
  * N, full-sequence attention [paperlayer §2]), head dim d in {64, 128}.
  *
@@ -111,6 +122,7 @@ typedef struct {
   int32_t partition;  /* SPR_PARTITION_RESPONSE (0, default) or _SEMANTIC;
                          semantic mode ignores Ms and p */
   int32_t init;       /* SPR_INIT_SEEDED (0, default) or SPR_INIT_WARM */
+  int32_t weights;    /* SPR_WEIGHTS_COVERAGE (0, default) or SPR_WEIGHTS_UNIFORM */
 } spr_params;
 
 /* Per-(batch, head) results, copied out by sparsepr_get_stats. */

@@ -67,6 +67,11 @@ Readings (the pages leave these steps open; the plainest reading is taken):
      coordinates (z = W^T k is linear, so means map by W), and the previous
      query centroids kept in head-dimension form a_g = mean of (s / rms) q,
      whose query-response coordinates are Ctilde a_g.
+  R14 estimator ablation ([paperlayer §5 "Ablations", Table 4]; the pages
+     do not list its rows): the unweighted estimator gives every probe the
+     weight 1/M in place of the coverage weight; the estimator without the
+     subspace restriction is r = d (U_r then spans the output space, so
+     projecting onto it changes nothing).
 """
 from __future__ import annotations
 
@@ -108,6 +113,7 @@ class Params:
     scale: float | None = None  # default 1/sqrt(d)
     weight_power: float = 0.5
     partition: str = "response"  # "response" | "semantic" (reading R11)
+    weights: str = "coverage"  # "coverage" | "uniform" (reading R14)
 
 
 # ---------------------------------------------------------------------------
@@ -614,6 +620,8 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
                col_idx=col_idx)
     # Probes
     probe_pos, probe_idx, wts, m_g = select_probes(counts_q, q_off, perm_q, prm.M)
+    if prm.weights == "uniform" and len(wts):  # the unweighted estimator (reading R14)
+        wts = np.full(len(wts), 1.0 / len(wts))
     routed, probe_pairs, rho = rho_exec(counts_q, counts_k, row_ptr, col_idx, prm.M)
     out.update(probe_pos=probe_pos, probe_idx=probe_idx, probe_w=wts, probe_m=m_g,
                routed_pairs=routed, probe_pairs=probe_pairs, rho_exec=rho)

@@ -46,6 +46,7 @@ class Workload:
     lam: float
     center_scale: float = 2.0
     partition: str = "response"  # or "semantic" (the comparator)
+    weights: str = "coverage"  # or "uniform" (probe weights of the fit)
 
     @property
     def N(self) -> int:

@@ -28,7 +28,8 @@ TIE_PI = 1e-5
 
 def oracle_params(wl, **kw) -> Params:
     d = dict(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
-             tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index)
+             tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index,
+             weights=wl.weights)
     d.update(kw)
     return Params(**d)
 
@@ -44,7 +45,7 @@ def run_gpu(wl, N=None, heads=None, inputs=None, check=None, partition=None):
     prm = spr.make_params(Qd, Kd, Vd, Od, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
                           seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
                           rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
-                          partition=partition)
+                          partition=partition, weights=wl.weights)
     ws = spr.alloc_workspace(prm)
     spr.sparsepr_call(prm, Qd, Kd, Vd, Od, ws)
     stats, err = spr.sparsepr_get_stats(prm, ws)
