@@ -270,6 +270,86 @@ def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=1024, seed=0):
             "o3_orthogonal_energy_rel": e_orth / den}
 
 
+def support_and_mass(P, keep, alpha=0.9, pool=8):
+    """O1 / O2 on sampled query rows (measurement only, torch).
+
+    P: [n, N] attention probabilities of n sampled queries, consecutive blocks
+    of `pool` rows from the same query group; keep: [n, N] bool, the keys each
+    query's route keeps.  Returns (per-query minimal-support fractions at mass
+    alpha, the pooled support fraction of each block, retained masses).  A
+    query's support: keys by decreasing probability (ties to the lower index)
+    until the running mass reaches alpha.
+    """
+    n, N = P.shape
+    ps, order = torch.sort(P, dim=1, descending=True, stable=True)
+    cs = torch.cumsum(ps, dim=1)
+    k = ((cs < alpha * P.sum(1, keepdim=True)).sum(1) + 1).clamp(max=N)
+    per = k.double() / N
+    in_sorted = torch.arange(N, device=P.device)[None, :] < k[:, None]
+    member = torch.zeros_like(in_sorted).scatter_(1, order, in_sorted)
+    pooled = member.view(n // pool, pool, N).any(1).sum(1).double() / N
+    mass = (P * keep).sum(1).double()
+    return per, pooled, mass
+
+
+def diagnostics(spr, prm, ws, Q, K, V, wl, alpha=0.9, pool=8, groups_per_head=16, seed=0):
+    """O1 pooled support and O2 retained mass vs error [paperlayer §3.1] on
+    query groups sampled from every head (pool members each), measurement
+    only: dense probabilities in fp32 here, the hard-drop rows from the
+    workspace."""
+    BH, N, d = wl.BH, wl.N, wl.d
+    dev = Q.device
+    g = torch.Generator().manual_seed(seed)
+    q_off = spr.workspace_tensor(prm, ws, "q_off", torch.int32, (BH, wl.Gq + 1)).long().cpu()
+    perm_q = spr.workspace_tensor(prm, ws, "perm_q", torch.int32, (BH, N)).long()
+    lab_k = spr.workspace_tensor(prm, ws, "lab_k", torch.int32, (BH, N)).long()
+    row_ptr = spr.workspace_tensor(prm, ws, "row_ptr", torch.int32, (BH, wl.Gq + 1)).long().cpu()
+    col_idx = spr.workspace_tensor(prm, ws, "col_idx", torch.int32, (BH, wl.Gq * wl.Gk)).long()
+    osp = spr.workspace_tensor(prm, ws, "o_sparse", torch.float32, (BH, N, d))
+    q, k, v = (t.reshape(BH, N, d) for t in (Q, K, V))
+    scale = 1.0 / d ** 0.5
+    pers, pooleds, masses, errs = [], [], [], []
+    for bh in range(BH):
+        sizes = q_off[bh, 1:] - q_off[bh, :-1]
+        big = torch.nonzero(sizes >= pool).flatten()
+        if len(big) == 0:
+            continue
+        groups = big[torch.randperm(len(big), generator=g)[:groups_per_head]]
+        pos, keep_groups = [], []
+        for gi in groups.tolist():
+            o0, cnt = int(q_off[bh, gi]), int(sizes[gi])
+            pos.append(o0 + torch.randperm(cnt, generator=g)[:pool])
+            routed = col_idx[bh, int(row_ptr[bh, gi]):int(row_ptr[bh, gi + 1])]
+            keep_groups.append(torch.isin(lab_k[bh], routed))
+        pos = torch.cat(pos).to(dev)
+        rows = perm_q[bh, pos]
+        keep = torch.stack(keep_groups).repeat_interleave(pool, dim=0)
+        P = torch.softmax((q[bh, rows].float() @ k[bh].float().T) * scale, dim=-1)
+        per, pooled, mass = support_and_mass(P, keep, alpha, pool)
+        dense = P @ v[bh].float()
+        err = (osp[bh, pos] - dense).norm(dim=1) / dense.norm(dim=1)
+        pers.append(per)
+        pooleds.append(pooled)
+        masses.append(mass)
+        errs.append(err.double())
+    if not pers:
+        return {"alpha": alpha, "queries": 0, "pool": pool}
+    per, pooled, mass, err = (torch.cat(x).cpu() for x in (pers, pooleds, masses, errs))
+    # O2: how far retained mass ranks the errors (Spearman), and the spread of
+    # the error among the fifth of the queries closest to the median mass
+    rank = lambda x: torch.argsort(torch.argsort(x)).double()
+    rm, re = rank(mass), rank(err)
+    rm, re = rm - rm.mean(), re - re.mean()
+    spearman = float((rm * re).sum() / (rm.norm() * re.norm()))
+    near = torch.argsort((mass - mass.median()).abs())[: max(2, len(mass) // 5)]
+    e_near = err[near]
+    return {"alpha": alpha, "queries": int(len(per)), "pool": pool,
+            "o1_support_median": float(per.median()), "o1_pooled_median": float(pooled.median()),
+            "o2_mass_median": float(mass.median()), "o2_spearman_mass_error": spearman,
+            "o2_error_p90_over_p10_at_median_mass":
+                float(torch.quantile(e_near, 0.9) / torch.quantile(e_near, 0.1))}
+
+
 def run_ours(args, wl):
     import free_block_sparse_means_b200 as spr
     world, rank, local = dist_info()
@@ -402,6 +482,8 @@ def run_ours(args, wl):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": int(n1 - n0), "clocks": clocks, "device_error": err}
     line["rel_l2_vs_dense"] = quality_vs_dense(spr, prm, ws, Q, K, V, O, wl)
+    if args.diagnostics:
+        line["diagnostics"] = diagnostics(spr, prm, ws, Q, K, V, wl)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_baseline(wl, budget_s=args.cpu_budget)
     if world > 1:
@@ -428,6 +510,10 @@ def main(argv=None):
                     help="uniform: the unweighted estimator of the ablation")
     ap.add_argument("--rank", type=int, default=0,
                     help="r of the residual fit (0: the workload's; d: no subspace restriction)")
+    ap.add_argument("--diagnostics", action="store_true",
+                    help="add the O1 pooled-support and O2 retained-mass diagnostics")
+    ap.add_argument("--rho", type=float, default=0.0,
+                    help="executed-pair density target (0: the workload's), for density sweeps")
     ap.add_argument("--partition", default="response", choices=["response", "semantic"],
                     help="semantic: the raw-row k-means comparator instead of the method's "
                          "response-coupled partition")
@@ -437,6 +523,8 @@ def main(argv=None):
     wl = workload(args.workload, partition=args.partition, weights=args.weights)
     if args.rank > 0:
         wl = wl.replace(r=args.rank)
+    if args.rho > 0:
+        wl = wl.replace(route_mode="budget", rho_target=args.rho)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

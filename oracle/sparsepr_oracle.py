@@ -72,6 +72,11 @@ Readings (the pages leave these steps open; the plainest reading is taken):
      weight 1/M in place of the coverage weight; the estimator without the
      subspace restriction is r = d (U_r then spans the output space, so
      projecting onto it changes nothing).
+  R15 O1 / O2 ([paperlayer §3.1]): a query's support at mass alpha is the
+     smallest key set reaching alpha (keys ranked by probability, ties to the
+     lower index); the pooled support of a set of queries is the union of
+     theirs; the retained mass of a query is the attention mass on the keys
+     its route keeps.
 """
 from __future__ import annotations
 
@@ -87,6 +92,7 @@ __all__ = [
     "route_logits", "route_masses", "route_select", "route_to_csr",
     "select_probes", "hard_drop_attention", "fit_residual", "apply_correction",
     "rho_exec", "sparsepr_head", "sparsepr_call", "affine_residual_decomposition",
+    "attention_probs", "minimal_support", "pooled_support", "retained_mass",
 ]
 
 MASK64 = (1 << 64) - 1
@@ -667,6 +673,41 @@ def affine_residual_decomposition(O_sparse, O_dense):
     er, ep, eo = float((R * R).sum()), float((P * P).sum()), float((E * E).sum())
     return {"residual_energy": er, "affine_energy": ep, "orthogonal_energy": eo,
             "affine_fraction": ep / er if er > 0 else 0.0}
+
+
+def attention_probs(Qr, K, scale):
+    """Softmax attention probabilities of query rows Qr over all keys, fp64."""
+    S = scale * (np.asarray(Qr, np.float64) @ np.asarray(K, np.float64).T)
+    S -= S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    return P / P.sum(axis=1, keepdims=True)
+
+
+def minimal_support(p, alpha):
+    """O1 [paperlayer §3.1 O1]; reading R15.  The smallest key set of one
+    query reaching attention mass alpha: keys ranked by probability (ties to
+    the lower index), taken until the running mass reaches alpha."""
+    p = np.asarray(p, np.float64)
+    order = np.lexsort((np.arange(len(p)), -p))
+    k = int(np.searchsorted(np.cumsum(p[order]), alpha * p.sum(), side="left")) + 1
+    return np.sort(order[:min(k, len(p))])
+
+
+def pooled_support(P, alpha):
+    """O1: per-query minimal supports of the rows of P and their union (the
+    support a shared route must cover for these queries), as fractions of the
+    keys.  Returns (per_query_fractions, pooled_fraction)."""
+    P = np.asarray(P, np.float64)
+    sets = [minimal_support(row, alpha) for row in P]
+    per = np.array([len(s_) for s_ in sets], np.float64) / P.shape[1]
+    pooled = len(np.unique(np.concatenate(sets))) / P.shape[1]
+    return per, pooled
+
+
+def retained_mass(P, keep):
+    """O2 [paperlayer §3.1 O2]: attention mass each query keeps under a key
+    mask (rows of ``keep`` are the kept keys of each query)."""
+    return (np.asarray(P, np.float64) * np.asarray(keep, bool)).sum(axis=1)
 
 
 def sparsepr_call(Q, K, V, prm: Params, **kw):
