@@ -454,62 +454,46 @@ __global__ void __launch_bounds__(256) k_amat(const float* Ct, int G, int D,
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core row GEMM over the queries of one head (mma.sync m16n8k16 bf16,
-// fp32 accumulation) with the B operand split into bf16 hi + lo so that the
-// products carry ~16 bits of the fp32 B.
-//   QUAD  : B = A (D x D); per row qAq -> rms = sqrt(s^2 qAq / G'k + eps),
-//           ||u_hat||^2 = s^2 qAq / rms^2  (query-response RMS, reading R4)
-//   assign: B rows = Bq_g = A a_g; score_g = (s / rms_n) q.Bq_g - beta_g;
-//           label = argmax (ties to the lowest g)  (query k-means assignment
-//           in factored form: u.m_g - ||m_g||^2 / 2 with m_g = Ctilde a_g)
-// One block per rows_per_cta rows (sub-tiles of 128), 8 warps x 16 rows.
+// Query-response RMS on the tensor cores (mma.sync m16n8k16 bf16, fp32
+// accumulation), reading R4: per query row the quadratic form q A q with
+// A = Ctilde^T Ctilde split into bf16 hi + lo (the products carry ~16 bits
+// of the fp32 A); rms = sqrt(s^2 qAq / G'k + eps) and ||u_hat||^2 =
+// s^2 qAq / rms^2 (their chunk sums feed the query objective).
+// One block per CHUNK rows (sub-tiles of 128), 8 warps x 16 rows.
 // ---------------------------------------------------------------------------
-struct RowGemmArgs {
+struct RmsArgs {
   TensorView Q;
-  int N, G, nchunk, split_rows;
-  int rows_per_cta;     // multiple of ATT_BM; CHUNK for the quadratic form
-  const bf16* bsplit;   // [BH][2][split_rows][D]
-  const float* beta;    // [BH][G]
+  int N, nchunk, split_rows;
+  const bf16* bsplit;   // [BH][2][split_rows][D]: rows of A, bf16 hi then lo
   float scale;
   const spr_head_stats* stats;
   float* rms;
   float* un2;
-  int32_t* lab;
   double* part;
-  Header* hdr;
 };
 
-template <int D, bool QUAD>
-__global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
+template <int D>
+__global__ void __launch_bounds__(256) k_query_rms(RmsArgs a) {
   constexpr int CH = D / 8;  // 16-byte chunks per row
   extern __shared__ __align__(128) uint8_t rsm[];
-  const int NC = QUAD ? D : ((a.G + 31) / 32) * 32;  // padded B rows
   uint8_t* Bhi = rsm;
-  uint8_t* Blo = Bhi + NC * D * 2;
-  uint8_t* Qs = Blo + NC * D * 2;
-  float* betas = reinterpret_cast<float*>(Qs + ATT_BM * D * 2);
-  double* red = reinterpret_cast<double*>(betas + 2 * MAX_GROUPS);
+  uint8_t* Blo = Bhi + D * D * 2;
+  uint8_t* Qs = Blo + D * D * 2;
+  double* red = reinterpret_cast<double*>(Qs + ATT_BM * D * 2);
   const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
-  const int nrows_b = QUAD ? D : a.G;
-  // B operand, swizzled rows
+  // B operand = A, swizzled rows
   const bf16* bsrc = a.bsplit + (size_t)bh * 2 * a.split_rows * D;
-  for (int e = tid; e < NC * CH; e += 256) {
+  for (int e = tid; e < D * CH; e += 256) {
     const int r = e / CH, c = e % CH;
-    uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
-    if (r < nrows_b) {
-      hi = reinterpret_cast<const uint4*>(bsrc + (size_t)r * D)[c];
-      lo = reinterpret_cast<const uint4*>(bsrc + ((size_t)a.split_rows + r) * D)[c];
-    }
-    *reinterpret_cast<uint4*>(Bhi + swz<CH>(r, c)) = hi;
-    *reinterpret_cast<uint4*>(Blo + swz<CH>(r, c)) = lo;
+    *reinterpret_cast<uint4*>(Bhi + swz<CH>(r, c)) = reinterpret_cast<const uint4*>(bsrc + (size_t)r * D)[c];
+    *reinterpret_cast<uint4*>(Blo + swz<CH>(r, c)) =
+        reinterpret_cast<const uint4*>(bsrc + ((size_t)a.split_rows + r) * D)[c];
   }
-  if (!QUAD)
-    for (int g = tid; g < MAX_GROUPS; g += 256) betas[g] = g < a.G ? a.beta[(size_t)bh * a.G + g] : 0.f;
-  const float gk = QUAD ? (float)max(1, a.stats[bh].gk_nonempty) : 1.f;
+  const float gk = (float)max(1, a.stats[bh].gk_nonempty);
   double un2acc = 0.0;
-  for (int sub = 0; sub < a.rows_per_cta / ATT_BM; ++sub) {
-    const int row0 = chunk * a.rows_per_cta + sub * ATT_BM;
+  for (int sub = 0; sub < CHUNK / ATT_BM; ++sub) {
+    const int row0 = chunk * CHUNK + sub * ATT_BM;
     if (row0 >= a.N) break;
     __syncthreads();  // previous tile consumed
     for (int e = tid; e < ATT_BM * CH; e += 256) {
@@ -529,14 +513,8 @@ __global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
       ldsm_x4(af[ks][0], af[ks][1], af[ks][2], af[ks][3], Qs + swz<CH>(r, c));
     }
     const int r_lo = row0 + warp * 16 + gid, r_hi = r_lo + 8;
-    float alpha_lo = 1.f, alpha_hi = 1.f;
-    if (!QUAD) {
-      alpha_lo = r_lo < a.N ? a.scale / a.rms[(size_t)bh * a.N + r_lo] : 0.f;
-      alpha_hi = r_hi < a.N ? a.scale / a.rms[(size_t)bh * a.N + r_hi] : 0.f;
-    }
-    float best_lo = -FLT_MAX, best_hi = -FLT_MAX, quad_lo = 0.f, quad_hi = 0.f;
-    int arg_lo = 0, arg_hi = 0;
-    for (int nc = 0; nc < NC; nc += 32) {
+    float quad_lo = 0.f, quad_hi = 0.f;
+    for (int nc = 0; nc < D; nc += 32) {
       float acc[4][4];
 #pragma unroll
       for (int t = 0; t < 4; ++t)
@@ -558,79 +536,47 @@ __global__ void __launch_bounds__(256) k_rowgemm(RowGemmArgs a) {
         }
       }
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
+      for (int t = 0; t < 4; ++t) {  // (qA)_col q_col, from the swizzled tile
         const int col = nc + t * 8 + 2 * tig;
-        if (QUAD) {
-          // q values at (row, col), (row, col+1) from the swizzled tile
-          const int rl = warp * 16 + gid, rh = rl + 8;
-          const bf16* ql = reinterpret_cast<const bf16*>(Qs + swz<CH>(rl, col / 8)) + (col & 7);
-          const bf16* qh = reinterpret_cast<const bf16*>(Qs + swz<CH>(rh, col / 8)) + (col & 7);
-          quad_lo += acc[t][0] * bf2f(ql[0]) + acc[t][1] * bf2f(ql[1]);
-          quad_hi += acc[t][2] * bf2f(qh[0]) + acc[t][3] * bf2f(qh[1]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int g = col + e;
-            if (g < a.G) {
-              const float sl = alpha_lo * acc[t][e] - betas[g];
-              const float sh = alpha_hi * acc[t][2 + e] - betas[g];
-              if (sl > best_lo) { best_lo = sl; arg_lo = g; }
-              if (sh > best_hi) { best_hi = sh; arg_hi = g; }
-            }
-          }
-        }
+        const int rl = warp * 16 + gid, rh = rl + 8;
+        const bf16* ql = reinterpret_cast<const bf16*>(Qs + swz<CH>(rl, col / 8)) + (col & 7);
+        const bf16* qh = reinterpret_cast<const bf16*>(Qs + swz<CH>(rh, col / 8)) + (col & 7);
+        quad_lo += acc[t][0] * bf2f(ql[0]) + acc[t][1] * bf2f(ql[1]);
+        quad_hi += acc[t][2] * bf2f(qh[0]) + acc[t][3] * bf2f(qh[1]);
       }
     }
-    if (QUAD) {
-      quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 1);
-      quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 2);
-      quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 1);
-      quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 2);
-      if (tig == 0) {
-        const float s2 = a.scale * a.scale;
-        if (r_lo < a.N) {
-          const float ms = s2 * fmaxf(quad_lo, 0.f) / gk;
-          const float rr = sqrtf(ms + 1e-6f);
-          a.rms[(size_t)bh * a.N + r_lo] = rr;
-          const float u2 = s2 * fmaxf(quad_lo, 0.f) / (rr * rr);
-          a.un2[(size_t)bh * a.N + r_lo] = u2;
-          un2acc += u2;
-        }
-        if (r_hi < a.N) {
-          const float ms = s2 * fmaxf(quad_hi, 0.f) / gk;
-          const float rr = sqrtf(ms + 1e-6f);
-          a.rms[(size_t)bh * a.N + r_hi] = rr;
-          const float u2 = s2 * fmaxf(quad_hi, 0.f) / (rr * rr);
-          a.un2[(size_t)bh * a.N + r_hi] = u2;
-          un2acc += u2;
-        }
+    quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 1);
+    quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 2);
+    quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 1);
+    quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 2);
+    if (tig == 0) {
+      const float s2 = a.scale * a.scale;
+      if (r_lo < a.N) {
+        const float ms = s2 * fmaxf(quad_lo, 0.f) / gk;
+        const float rr = sqrtf(ms + 1e-6f);
+        a.rms[(size_t)bh * a.N + r_lo] = rr;
+        const float u2 = s2 * fmaxf(quad_lo, 0.f) / (rr * rr);
+        a.un2[(size_t)bh * a.N + r_lo] = u2;
+        un2acc += u2;
       }
-    } else {
-#pragma unroll
-      for (int o = 1; o <= 2; o <<= 1) {
-        const float bl = __shfl_xor_sync(0xffffffffu, best_lo, o);
-        const int al = __shfl_xor_sync(0xffffffffu, arg_lo, o);
-        if (bl > best_lo || (bl == best_lo && al < arg_lo)) { best_lo = bl; arg_lo = al; }
-        const float bhv = __shfl_xor_sync(0xffffffffu, best_hi, o);
-        const int ah = __shfl_xor_sync(0xffffffffu, arg_hi, o);
-        if (bhv > best_hi || (bhv == best_hi && ah < arg_hi)) { best_hi = bhv; arg_hi = ah; }
-      }
-      if (tig == 0) {
-        if (r_lo < a.N) a.lab[(size_t)bh * a.N + r_lo] = arg_lo;
-        if (r_hi < a.N) a.lab[(size_t)bh * a.N + r_hi] = arg_hi;
+      if (r_hi < a.N) {
+        const float ms = s2 * fmaxf(quad_hi, 0.f) / gk;
+        const float rr = sqrtf(ms + 1e-6f);
+        a.rms[(size_t)bh * a.N + r_hi] = rr;
+        const float u2 = s2 * fmaxf(quad_hi, 0.f) / (rr * rr);
+        a.un2[(size_t)bh * a.N + r_hi] = u2;
+        un2acc += u2;
       }
     }
   }
   __syncthreads();
-  if (QUAD) {
-    un2acc = warp_sum(un2acc);
-    if (lane == 0) red[warp] = un2acc;
-    __syncthreads();
-    if (tid == 0) {
-      double s = 0.0;
-      for (int i = 0; i < 8; ++i) s += red[i];
-      a.part[((size_t)bh * 2 + 1) * (a.nchunk + 1) + chunk] = s;
-    }
+  un2acc = warp_sum(un2acc);
+  if (lane == 0) red[warp] = un2acc;
+  __syncthreads();
+  if (tid == 0) {
+    double s = 0.0;
+    for (int i = 0; i < 8; ++i) s += red[i];
+    a.part[((size_t)bh * 2 + 1) * (a.nchunk + 1) + chunk] = s;
   }
 }
 
@@ -852,26 +798,21 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   spr_launch(k_amat, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, P.Ct, p.Gk, D, P.stats, P.Amat, P.bq16,
                                                          split_rows);
   // Query-response RMS (tensor-core quadratic form)
-  RowGemmArgs ra{};
+  RmsArgs ra{};
   ra.Q = Q;
   ra.N = N;
-  ra.G = p.Gq;
   ra.nchunk = nchunk;
   ra.split_rows = split_rows;
   ra.bsplit = P.bq16;
-  ra.beta = P.beta;
   ra.scale = scale;
   ra.stats = P.stats;
   ra.rms = P.rms;
   ra.un2 = P.un2;
-  ra.lab = P.labq;
-  ra.rows_per_cta = CHUNK;
   ra.part = P.part;
-  ra.hdr = P.hdr;
   {
-    const size_t sm = (size_t)2 * D * D * 2 + ATT_BM * D * 2 + MAX_GROUPS * 8 + 64;
-    cudaFuncSetAttribute(k_rowgemm<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    spr_launch(k_rowgemm<D, true>, dim3(nchunk, BH), 256, sm, st, ra);
+    const size_t sm = (size_t)2 * D * D * 2 + ATT_BM * D * 2 + 64;
+    cudaFuncSetAttribute(k_query_rms<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    spr_launch(k_query_rms<D>, dim3(nchunk, BH), 256, sm, st, ra);
   }
   // Query k-means in the head dimension
   if (p.init != SPR_INIT_WARM)  // warm: centq keeps the previous call's head-dim centroids
