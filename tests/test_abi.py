@@ -49,9 +49,10 @@ def test_struct_layout_matches_c(tmp_path):
 #include <stddef.h>
 #include "sparsepr.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(spr_params), offsetof(spr_params, scale),
-         offsetof(spr_params, seed), offsetof(spr_params, tau), offsetof(spr_params, M),
-         offsetof(spr_params, lambda), offsetof(spr_params, partition), sizeof(spr_head_stats),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(spr_params),
+         offsetof(spr_params, scale), offsetof(spr_params, seed), offsetof(spr_params, tau),
+         offsetof(spr_params, M), offsetof(spr_params, lambda), offsetof(spr_params, partition),
+         offsetof(spr_params, init), offsetof(spr_params, weights), sizeof(spr_head_stats),
          offsetof(spr_head_stats, gk_nonempty));
   return 0;
 }
@@ -61,7 +62,8 @@ int main(void) {
     got = list(map(int, subprocess.check_output([str(exe)]).split()))
     P, S = spr.SprParams, spr.SprHeadStats
     want = [ctypes.sizeof(P), P.scale.offset, P.seed.offset, P.tau.offset, P.M.offset,
-            P.lambda_.offset, P.partition.offset, ctypes.sizeof(S), S.gk_nonempty.offset]
+            P.lambda_.offset, P.partition.offset, P.init.offset, P.weights.offset, ctypes.sizeof(S),
+            S.gk_nonempty.offset]
     assert got == want
 
 
@@ -84,10 +86,15 @@ def test_validation(lib):
     prm.d = 96
     assert spr.sparsepr_check_params(prm) == spr._binding.SPR_EUNSUPPORTED
     assert spr.sparsepr_check_params(_params(partition="semantic")) == 0
-    prm = _params()
-    prm.partition = 2
-    assert spr.sparsepr_check_params(prm) == spr._binding.SPR_EINVAL
-    assert spr.sparsepr_workspace_size(prm) == 0
+    for field in ("partition", "init", "weights"):
+        prm = _params()
+        setattr(prm, field, 2)
+        assert spr.sparsepr_check_params(prm) == spr._binding.SPR_EINVAL, field
+        assert spr.sparsepr_workspace_size(prm) == 0, field
+    assert spr.sparsepr_check_params(_params(init="warm", weights="uniform")) == 0
+    # the options do not change the workspace a call needs
+    n = spr.sparsepr_workspace_size(_params())
+    assert spr.sparsepr_workspace_size(_params(init="warm", weights="uniform", partition="semantic")) == n
 
 
 def test_entry_points_reject_before_any_gpu_work(lib):
