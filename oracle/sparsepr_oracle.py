@@ -77,6 +77,10 @@ Readings (the pages leave these steps open; the plainest reading is taken):
      lower index); the pooled support of a set of queries is the union of
      theirs; the retained mass of a query is the attention mass on the keys
      its route keeps.
+  R16 distance-ranked probes (a probe-selection variant of [paperlayer §5
+     "Ablations", Table 4]): the same per-group probe counts, but each group
+     takes its rows nearest its centroid in query-response coordinates
+     (squared distance; ties to the lower original index).
 """
 from __future__ import annotations
 
@@ -120,6 +124,7 @@ class Params:
     weight_power: float = 0.5
     partition: str = "response"  # "response" | "semantic" (reading R11)
     weights: str = "coverage"  # "coverage" | "uniform" (reading R14)
+    probe_select: str = "stratified"  # "stratified" | "ranked" (reading R16)
 
 
 # ---------------------------------------------------------------------------
@@ -388,9 +393,13 @@ def route_to_csr(mask):
 # ---------------------------------------------------------------------------
 # Probe selection [paperlayer §4, App. A.2; gist-nl §2B]; reading R6
 # ---------------------------------------------------------------------------
-def select_probes(counts_q, q_off, perm_q, M):
-    """Stratified probe rows and coverage weights.
+def select_probes(counts_q, q_off, perm_q, M, dist=None):
+    """Stratified probe rows and coverage weights (reading R6).
 
+    With ``dist`` (one value per original row: its squared distance to its own
+    query centroid in query-response coordinates) the m_g rows of group g are
+    instead its m_g rows nearest the centroid, ties to the lower original
+    index (reading R16); counts and weights are unchanged.
     Returns (probe_pos, probe_idx, weights, m_g): permuted positions, original
     row indices (both ordered by group, then position), weights summing to 1,
     and the per-group probe counts.
@@ -424,8 +433,18 @@ def select_probes(counts_q, q_off, perm_q, M):
     pos, wt = [], []
     covered = int(counts_q[m > 0].sum())
     for g in range(G):
-        for t in range(int(m[g])):
-            pos.append(int(q_off[g]) + ((2 * t + 1) * int(counts_q[g])) // (2 * int(m[g])))
+        mg, cnt = int(m[g]), int(counts_q[g])
+        if mg == 0:
+            continue
+        if dist is None:
+            chosen = [int(q_off[g]) + ((2 * t + 1) * cnt) // (2 * mg) for t in range(mg)]
+        else:
+            span = np.arange(int(q_off[g]), int(q_off[g]) + cnt)
+            rows = np.asarray(perm_q)[span]
+            order = np.lexsort((rows, np.asarray(dist)[rows]))
+            chosen = np.sort(span[order[:mg]]).tolist()
+        for p_ in chosen:
+            pos.append(p_)
             wt.append((counts_q[g] / m[g]) / covered)
     pos = np.array(pos, np.int64)
     return pos, np.asarray(perm_q)[pos] if len(pos) else pos, np.array(wt, np.float64), m
@@ -562,6 +581,7 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
         ne_q = np.bincount(lab_q, minlength=prm.Gq) > 0
         out["obj_q"] = kmeans_objective(Q, lab_q, np.where(ne_q[:, None], Cu, 0.0))
         rms, Ct = None, None
+        Xq = Q
     else:
         # Key-response coordinates and paired K/V groups
         qs_idx = sample_query_indices(N, prm.Ms)
@@ -600,6 +620,7 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
         Cu = group_means(Uq, lab_q, prm.Gq)
         ne_q = np.bincount(lab_q, minlength=prm.Gq) > 0
         out["obj_q"] = kmeans_objective(Uq, lab_q, np.where(ne_q[:, None], Cu, 0.0))
+        Xq = Uq
     out.update(lab_k=lab_k, lab_q=lab_q, C=C, counts_k=counts_k, rms=rms, Ctilde=Ct,
                Cu=Cu)
     # what a warm-started next call starts from (reading R13): raw-key group
@@ -625,7 +646,11 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
     out.update(route_logits=L, route_pi=pi, route_entry=e, route_tail=tail, row_ptr=row_ptr,
                col_idx=col_idx)
     # Probes
-    probe_pos, probe_idx, wts, m_g = select_probes(counts_q, q_off, perm_q, prm.M)
+    dist = None
+    if prm.probe_select == "ranked":  # reading R16: nearest to the own query centroid
+        dist = ((Xq - Cu[lab_q]) ** 2).sum(axis=1)
+        out["probe_dist"] = dist
+    probe_pos, probe_idx, wts, m_g = select_probes(counts_q, q_off, perm_q, prm.M, dist)
     if prm.weights == "uniform" and len(wts):  # the unweighted estimator (reading R14)
         wts = np.full(len(wts), 1.0 / len(wts))
     routed, probe_pairs, rho = rho_exec(counts_q, counts_k, row_ptr, col_idx, prm.M)
