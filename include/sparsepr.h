@@ -155,6 +155,9 @@ spr_status sparsepr_check_params(const spr_params* prm);
  * groups (values follow their keys); queries are k-means-clustered on their
  * RMS-normalised logits against the centred nonempty K/V-group centroids;
  * Q, K, V are then permuted into group-major layouts inside the workspace.
+ * prm->partition = SPR_PARTITION_SEMANTIC clusters the raw key rows and the
+ * raw query rows instead (the comparator); prm->init = SPR_INIT_WARM starts
+ * both k-means from the centroids the previous call left in `ws`.
  * Reads Q, K, V (device, bf16, strides from prm); writes only `ws`.
  */
 spr_status sparsepr_partition(const spr_params* prm, const void* Q, const void* K,
@@ -167,8 +170,9 @@ spr_status sparsepr_partition(const spr_params* prm, const void* Q, const void* 
  * them is below tau, budget mode keeps the largest such prefix set whose
  * true pair cost plus the M*N probe pairs fits rho_target*N^2 (each group's
  * top cell always kept).  Emits the routed-cell CSR, merged key ranges, M
- * probe rows stratified over query groups with coverage weights, and the
- * attention work list.  Reads and writes only `ws`.
+ * probe rows stratified over query groups with coverage weights (1 / M each
+ * with prm->weights = SPR_WEIGHTS_UNIFORM), and the attention work list.
+ * Reads and writes only `ws`.
  */
 spr_status sparsepr_route(const spr_params* prm, void* ws, size_t ws_bytes, void* stream);
 
