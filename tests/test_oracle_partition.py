@@ -69,6 +69,14 @@ def test_init_indices_distinct_deterministic():
     assert sorted(kmeans_init_indices(12, 12, 1, 0, 0).tolist()) == list(range(12))
 
 
+def test_init_indices_hand_worked_vectors(golden_dir):
+    with open(os.path.join(golden_dir, "kmeans_init_vectors.txt")) as f:
+        rows = [list(map(int, l.split())) for l in f if l.strip() and not l.startswith("#")]
+    assert len(rows) == 2
+    for n, G, seed, bh, which, *want in rows:
+        assert kmeans_init_indices(n, G, seed, bh, which).tolist() == want
+
+
 def test_kmeans_vs_brute_force_and_monotone():
     rng = np.random.default_rng(2)
     for trial in range(20):
