@@ -145,3 +145,40 @@ def test_query_coords_explicit_logits():
     # a common shift of every key leaves the coordinates unchanged
     U2, _, _ = query_response_coords(Q, kv_centroids(K + 5.0, lab_k, Gk)[0], counts, s)
     np.testing.assert_allclose(U2, U, atol=1e-12)
+
+
+def test_kmeans_empty_cluster_keeps_centroid(golden_dir):
+    """A cluster that empties at iteration 2 keeps its centroid, which then
+    wins a row back at iteration 3 (tests/golden/kmeans_empty_cluster.txt,
+    worked by hand): a reset of the empty centroid (to zero, to the data
+    mean, or dropped) gives other labels."""
+    from fractions import Fraction
+    from oracle import kmeans
+    rows, init, labels, cents, obj = None, None, {}, {}, {}
+    with open(os.path.join(golden_dir, "kmeans_empty_cluster.txt")) as f:
+        for line in f:
+            if not line.strip() or line.startswith("#"):
+                continue
+            k, *rest = line.split()
+            if k == "rows":
+                rows = np.array([[float(v) for v in r.split(",")] for r in rest])
+            elif k == "init":
+                init = [int(v) for v in rest]
+            elif k == "labels":
+                labels[int(rest[0])] = [int(v) for v in rest[1:]]
+            elif k == "centroids":
+                cents[int(rest[0])] = [[float(Fraction(v)) for v in r.split(",")] for r in rest[1:]]
+            elif k == "objective":
+                obj[int(rest[0])] = float(Fraction(rest[1]))
+    assert rows is not None and len(labels) == 4
+    for T, want in labels.items():
+        lab, C, o, hist = kmeans(rows, 3, T, init)
+        assert lab.tolist() == want, (T, lab.tolist())
+        if T in cents:
+            np.testing.assert_allclose(C, cents[T], rtol=0, atol=1e-12)
+        if T in obj:
+            assert abs(o - obj[T]) < 1e-12
+    # the per-iteration objectives are not monotone here only if the rule is
+    # wrong: with the kept centroid they never rise
+    _, _, _, hist = kmeans(rows, 3, 4, init)
+    assert all(b <= a + 1e-12 for a, b in zip(hist, hist[1:]))

@@ -175,3 +175,28 @@ def test_csr_columns_ascending():
     mask = np.array([[0, 1, 1, 0], [0, 0, 0, 0], [1, 0, 0, 1]], bool)
     rp, ci = route_to_csr(mask)
     assert rp.tolist() == [0, 2, 2, 4] and ci.tolist() == [1, 2, 0, 3]
+
+
+def _fractions(s):
+    return [Fraction(x) for x in s.split(",")]
+
+
+def test_probe_coverage_weight_values(golden_dir):
+    """Probe counts, positions and coverage-weight values on unequal groups,
+    worked by hand (tests/golden/probe_coverage_weights.txt): catches an
+    inverted or mis-normalised weight that still sums to one."""
+    with open(os.path.join(golden_dir, "probe_coverage_weights.txt")) as f:
+        cases = [dict(kv.split("=") for kv in line.split()) for line in f
+                 if line.strip() and not line.startswith("#")]
+    assert len(cases) == 3
+    for c in cases:
+        counts = np.array([int(x) for x in c["counts"].split(",")], np.int64)
+        M = int(c["M"])
+        off = np.concatenate([[0], np.cumsum(counts)])
+        perm = np.arange(int(counts.sum()))[::-1].copy()  # any permutation
+        pos, idx, w, m = select_probes(counts, off, perm, M)
+        assert m.tolist() == [int(x) for x in c["m"].split(",")]
+        assert pos.tolist() == [int(x) for x in c["pos"].split(",")]
+        assert (idx == perm[pos]).all()
+        want = [float(x) for x in _fractions(c["w"])]
+        np.testing.assert_allclose(w, want, rtol=1e-15, atol=0)
