@@ -244,12 +244,33 @@ def sparsepr_attend_routed_noalloc(Qp, Kp, Vp, q_off, run_ptr, runs, Gk, O, stat
     Qp, Kp, Vp: [BH, N, d] bf16 group-major; q_off, run_ptr: [BH, Gq + 1]
     int32; runs: [BH, Gq * Gk, 2] int32 key ranges; O: [BH, N, d] fp32;
     status: optional int32[4] device tensor receiving the device error word.
+    Every tensor must be contiguous and on the same CUDA device; anything
+    else raises ValueError before the library is called.
     """
+    if Qp.dim() != 3:
+        raise ValueError("Qp must be [BH, N, d]")
     BH, N, d = Qp.shape
-    Gq = q_off.shape[1] - 1
+    Gq = q_off.shape[1] - 1 if q_off.dim() == 2 else -1
+    want = {"Qp": (Qp, torch.bfloat16, (BH, N, d)), "Kp": (Kp, torch.bfloat16, (BH, N, d)),
+            "Vp": (Vp, torch.bfloat16, (BH, N, d)), "q_off": (q_off, torch.int32, (BH, Gq + 1)),
+            "run_ptr": (run_ptr, torch.int32, (BH, Gq + 1)),
+            "runs": (runs, torch.int32, (BH, Gq * int(Gk), 2)), "O": (O, torch.float32, (BH, N, d))}
+    if status is not None:
+        want["status"] = (status, torch.int32, (4,))
+    for name, (t, dt, shape) in want.items():
+        if not isinstance(t, torch.Tensor):
+            raise ValueError(f"{name} must be a torch tensor")
+        if t.dtype != dt:
+            raise ValueError(f"{name} must be {dt}, got {t.dtype}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+        if not t.is_cuda or t.device != Qp.device:
+            raise ValueError(f"{name} must be on {Qp.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
     _check("sparsepr_attend_routed_noalloc", load_library().sparsepr_attend_routed_noalloc(
         Qp.data_ptr(), Kp.data_ptr(), Vp.data_ptr(), q_off.data_ptr(), run_ptr.data_ptr(),
-        runs.data_ptr(), BH, N, d, Gq, Gk, float(scale), O.data_ptr(),
+        runs.data_ptr(), BH, N, d, Gq, int(Gk), float(scale), O.data_ptr(),
         status.data_ptr() if status is not None else None, _stream(stream)))
 
 

@@ -53,8 +53,8 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_BQ16] = BH * 2 * (Gm > d ? Gm : d) * d * 2;  // semantic mode: key groups too
   sz[B_BETA] = BH * Gm * 4;
   sz[B_QBAR] = BH * Gq * d * 4;
-  sz[B_LOGIT] = BH * Gq * Gk * 4;
-  sz[B_ENTRY] = BH * Gq * Gk * 4;
+  sz[B_LOGIT] = BH * Gq * Gk * 8;
+  sz[B_ENTRY] = BH * Gq * Gk * 8;
   sz[B_TOP] = BH * Gq * Gk;
   sz[B_SEL] = BH * Gq * Gk;
   sz[B_ROWPTR] = BH * (Gq + 1) * 4;
@@ -79,11 +79,13 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_PART] = part_slots * 8;
   // k-means partial sums: per chunk, one slot per (group, warp segment)
   sz[B_CSUM] = BH * nchunk * (Gm + CSUM_SLOTS) * (d > P ? d : P) * 4;
-  if (sz[B_CSUM] < BH * Gm * 8 * d * 4) sz[B_CSUM] = BH * Gm * 8 * d * 4;  // group-mean slices
+  if (sz[B_CSUM] < BH * Gm * 8 * d * 8) sz[B_CSUM] = BH * Gm * 8 * d * 8;  // group-mean slices (fp64)
   // probe rows gathered for the fit: sparse outputs X, residuals R, block means
   sz[B_XP] = BH * (M ? M : 1) * d * 4;
   sz[B_RP] = BH * (M ? M : 1) * d * 4;
   sz[B_PMEAN] = BH * (M ? (M + 31) / 32 : 1) * 2 * d * 4;
+  sz[B_CRAW64] = BH * Gk * d * 8;
+  sz[B_QBAR64] = BH * Gq * d * 8;
   size_t off = 0;
   for (int i = 0; i < B_COUNT_; ++i) {
     L->off[i] = off;
@@ -136,8 +138,8 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.bq16 = AT(bf16*, B_BQ16);
   P.beta = AT(float*, B_BETA);
   P.qbar = AT(float*, B_QBAR);
-  P.logit = AT(float*, B_LOGIT);
-  P.entry = AT(float*, B_ENTRY);
+  P.logit = AT(double*, B_LOGIT);
+  P.entry = AT(double*, B_ENTRY);
   P.sel = AT(uint8_t*, B_SEL);
   P.top = AT(uint8_t*, B_TOP);
   P.rowptr = AT(int32_t*, B_ROWPTR);
@@ -164,6 +166,9 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.xp = AT(float*, B_XP);
   P.rp = AT(float*, B_RP);
   P.pmean = AT(float*, B_PMEAN);
+  P.craw64 = AT(double*, B_CRAW64);
+  P.qbar64 = AT(double*, B_QBAR64);
+  P.gpart = AT(double*, B_CSUM);
 #undef AT
   return P;
 }

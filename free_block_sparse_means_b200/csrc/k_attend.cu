@@ -233,6 +233,17 @@ __global__ void k_attend_reset(Header* hdr, spr_head_stats* stats, int BH) {
   for (int i = threadIdx.x; i < BH; i += blockDim.x) stats[i].tile_pairs = 0;
 }
 
+// Load the device code of every attention-stage kernel now (a kernel is
+// otherwise loaded at its first launch, which may take device memory).
+cudaError_t attend_preload() {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k_attend_reset);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, k_attend_mma<64>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, k_attend_mma<128>);
+  if (e == cudaSuccess) e = attend_tc_preload();
+  return e;
+}
+
 cudaError_t launch_attend(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st) {
   spr_launch(k_attend_reset, 1, 256, 0, st, P.hdr, P.stats, L.BH);
   if (attend_tc_enabled(p.d)) return launch_attend_tc(p, L, P, st);

@@ -479,6 +479,12 @@ bool attend_tc_enabled(int d) {
   return !(e && strcmp(e, "mma") == 0);
 }
 
+cudaError_t attend_tc_preload() {
+  if (!get_encode()) return cudaErrorInvalidValue;
+  cudaFuncAttributes fa;
+  return cudaFuncGetAttributes(&fa, k_attend_tc);
+}
+
 cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P,
                              cudaStream_t st) {
   CUtensorMap mQ, mQp, mK, mV;

@@ -14,8 +14,9 @@
 //      negative pivots of T - xI = L D L^T) at G points per step.
 //   3. Eigenvectors of T by inverse iteration on (T - lambda I) with partial
 //      pivoting (one thread per eigenvector, factors in shared memory), then
-//      orthonormalised in descending eigenvalue order by Cholesky QR
-//      (Y Y^T = L L^T, Y <- L^-1 Y).
+//      orthonormalised in descending eigenvalue order by Gram-Schmidt applied
+//      twice (a vector left in the span of the earlier ones, as happens for
+//      eigenvalues fp32 cannot separate, is replaced by a unit vector).
 //   4. Back-transformation x = H_0 H_1 ... H_{n-3} y, each warp holding its
 //      vectors in registers.
 // Outputs: evals[m][k] (descending, k < K), evecs[m][row][k] (stride n), and
@@ -60,10 +61,8 @@ struct EigSmem {
   static constexpr int Y = PART + EIG_WARPS;             // K x LD eigenvectors of T
   static constexpr int INV = 5 * NN * 32 + NN * 8;       // inverse-iteration factors of 32 vectors
   __host__ __device__ static int g_off(int K) { return Y + ((K * LD + 3) & ~3); }
-  __host__ __device__ static int total(int K) {
-    const int gm = K * (K + 1);
-    return g_off(K) + (gm > INV ? gm : INV);
-  }
+  // the inverse-iteration storage is reused by the orthonormalisation (NN + 1 floats)
+  __host__ __device__ static int total(int K) { return g_off(K) + INV; }
 };
 
 template <int NN>
@@ -85,7 +84,7 @@ __global__ void __launch_bounds__(EIG_THREADS, 1) k_eig_top(const float* Ain, in
   float* psb = esm + S::PS;
   float* part = esm + S::PART;
   float* Y = esm + S::Y;           // K x LD
-  float* Gr = esm + S::g_off(K);   // inverse-iteration factors, then the Cholesky-QR Gram
+  float* Gr = esm + S::g_off(K);   // inverse-iteration factors, then Gram-Schmidt scratch
   const int m = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* src = Ain + (size_t)m * NN * NN;
   if (warp == 0) {
@@ -448,56 +447,59 @@ __global__ void __launch_bounds__(EIG_THREADS, 1) k_eig_top(const float* Ain, in
     }
   }
   __syncthreads();
-  // Orthonormalise in descending eigenvalue order by Cholesky QR (the same
-  // basis as Gram-Schmidt in that order): Gm = Y Y^T = L L^T, Y <- L^-1 Y.
-  float* Gm = Gr;  // K x (K + 1), reuses the inverse-iteration storage
-  const int GL = K + 1;
-  for (int e = tid; e < K * K; e += EIG_THREADS) {
-    const int a = e / K, b = e % K;
-    if (b <= a) {
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < NN; i += 2) {
-        s0 = fmaf(Y[a * LD + i], Y[b * LD + i], s0);
-        s1 = fmaf(Y[a * LD + i + 1], Y[b * LD + i + 1], s1);
-      }
-      const float s = s0 + s1;
-      Gm[a * GL + b] = s;
-    }
-  }
-  __syncthreads();
-  // Cholesky of Gm, one barrier per column: the trailing update uses the
-  // unscaled column (G_ij -= G_ik G_jk / G_kk), the scaling comes at the end.
-  for (int kq = 0; kq < K - 1; ++kq) {
-    const float rkk = 1.f / fmaxf(Gm[kq * GL + kq], 1e-30f);
-    const int nt = K - 1 - kq;  // trailing order
-    for (int e = tid; e < nt * (nt + 1) / 2; e += EIG_THREADS) {
-      int i = (int)((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);  // e -> (i, j), j <= i
-      while (i * (i + 1) / 2 > e) --i;
-      while ((i + 1) * (i + 2) / 2 <= e) ++i;
-      const int j = e - i * (i + 1) / 2;
-      const int gi = kq + 1 + i, gj = kq + 1 + j;
-      Gm[gi * GL + gj] -= Gm[gi * GL + kq] * Gm[gj * GL + kq] * rkk;
-    }
-    __syncthreads();
-  }
-  for (int e = tid; e < K * K; e += EIG_THREADS) {
-    const int i = e / K, j = e % K;
-    if (j < i) Gm[i * GL + j] *= rsqrtf(fmaxf(Gm[j * GL + j], 1e-30f));
-  }
-  __syncthreads();
-  for (int i = tid; i < K; i += EIG_THREADS) Gm[i * GL + i] = sqrtf(fmaxf(Gm[i * GL + i], 1e-30f));
-  __syncthreads();
-  {  // Y <- L^-1 Y: TPC threads per column of Y split the sums, rows in order
-    constexpr int TPC = EIG_THREADS / NN;
-    const int col = tid / TPC, sub = tid % TPC;
+  // Orthonormalise in descending eigenvalue order by classical Gram-Schmidt
+  // applied twice per vector (Giraud, Langou & Rozloznik 2005: two passes
+  // give orthogonality to working precision).  Inverse iteration on
+  // eigenvalues that fp32 cannot separate (a cluster at the noise floor)
+  // returns nearly parallel vectors; a vector that keeps less than 1/8 of
+  // its length after the two passes lies in the span of the earlier ones and
+  // is replaced by the first unit vector e_j (j = a, a+1, ... mod n) that
+  // keeps more, so the basis stays orthonormal and finite.
+  {
+    float* dots = Gr;  // [NN], reuses the inverse-iteration storage
+    float* nrm_s = Gr + NN;
+    constexpr int TPE = EIG_THREADS / NN;  // threads per vector entry
+    const int ent = tid / TPE, sub = tid % TPE;
     for (int a = 0; a < K; ++a) {
-      float s = 0.f;
-      for (int b = sub; b < a; b += TPC) s = fmaf(Gm[a * GL + b], Y[b * LD + col], s);
+      for (int attempt = 0; attempt <= NN; ++attempt) {
+        if (attempt > 0) {  // replacement: e_j for the attempt-th candidate j
+          const int j = (a + attempt - 1) % NN;
+          for (int i = tid; i < NN; i += EIG_THREADS) Y[a * LD + i] = i == j ? 1.f : 0.f;
+          __syncthreads();
+        }
+        for (int pass = 0; pass < 2; ++pass) {
+          for (int bq = warp; bq < a; bq += EIG_WARPS) {  // dots with the earlier vectors
+            float d = 0.f;
+            for (int i = lane; i < NN; i += 32) d = fmaf(Y[a * LD + i], Y[bq * LD + i], d);
+            d = warp_sum(d);
+            if (lane == 0) dots[bq] = d;
+          }
+          __syncthreads();
+          float sacc = 0.f;  // sum_b dots[b] Y[b][ent], split over the TPE threads
+          for (int bq = sub; bq < a; bq += TPE) sacc = fmaf(dots[bq], Y[bq * LD + ent], sacc);
 #pragma unroll
-      for (int o = 1; o < TPC; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (sub == 0) Y[a * LD + col] = (Y[a * LD + col] - s) / Gm[a * GL + a];
-      __syncwarp();
+          for (int o = 1; o < TPE; o <<= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+          __syncthreads();  // every dot read before Y[a] changes
+          if (sub == 0) Y[a * LD + ent] -= sacc;
+          __syncthreads();
+        }
+        if (warp == 0) {
+          float q = 0.f;
+          for (int i = lane; i < NN; i += 32) q = fmaf(Y[a * LD + i], Y[a * LD + i], q);
+          q = warp_sum(q);
+          if (lane == 0) *nrm_s = q;
+        }
+        __syncthreads();
+        const float q = *nrm_s;
+        // the iterate and the replacements enter with unit length
+        if (isfinite(q) && q > 1.f / 64.f) {
+          const float inv = rsqrtf(q);
+          for (int i = tid; i < NN; i += EIG_THREADS) Y[a * LD + i] *= inv;
+          __syncthreads();
+          break;
+        }
+        __syncthreads();
+      }
     }
   }
   __syncthreads();

@@ -31,7 +31,16 @@ __device__ __align__(256) uint8_t g_na_scratch[NA_SCRATCH_BYTES];
 std::mutex g_na_mu;
 void* g_na_base[NA_MAX_DEVICES];
 
-// Address of the scratch area on the current device (looked up once).
+__global__ void k_na_check(const int32_t* qoff, const int32_t* runptr, const int2* runs, int BH,
+                           int N, int Gq, int Gk, int32_t* counts, Header* hdr);
+__global__ void k_na_plan(const int32_t* qoff, const int32_t* counts, int BH, int Gq,
+                          int max_items, int4* items, Header* hdr);
+__global__ void k_na_status(const Header* hdr, int32_t* status);
+
+// Address of the scratch area on the current device, with the one-time
+// set-up of that device: the symbol's address, and every kernel this entry
+// point can launch loaded now (device code is otherwise loaded at a kernel's
+// first launch, which may take device memory).
 cudaError_t na_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -42,6 +51,11 @@ cudaError_t na_scratch(void** out) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_na_scratch);
     if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, k_na_check)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, k_na_plan)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, k_na_status)) != cudaSuccess) return e;
+    if ((e = attend_preload()) != cudaSuccess) return e;
     g_na_base[dev] = p;
   }
   *out = g_na_base[dev];
@@ -57,76 +71,70 @@ int64_t na_max_items(int64_t BH, int64_t N, int64_t Gq) {
   return BH * ((N + ATT_BM - 1) / ATT_BM + Gq) + 1;
 }
 
+// Scratch layout: header | per-head stats | per-(head, group) tile counts | work list.
+size_t na_counts_off(int64_t BH) { return NA_HDR_BYTES + round256((size_t)BH * sizeof(spr_head_stats)); }
+size_t na_items_off(int64_t BH, int64_t Gq) {
+  return na_counts_off(BH) + round256((size_t)BH * Gq * sizeof(int32_t));
+}
 size_t na_bytes_needed(int64_t BH, int64_t N, int64_t Gq) {
-  return NA_HDR_BYTES + round256((size_t)BH * sizeof(spr_head_stats)) +
-         (size_t)na_max_items(BH, N, Gq) * sizeof(int4);
+  return na_items_off(BH, Gq) + (size_t)na_max_items(BH, N, Gq) * sizeof(int4);
 }
 
-// One block: reset the header, check every group offset and key range the
-// attention kernels will follow, then write the work list (query tiles of at
-// most 128 rows of each group that has rows and at least one key range, in
-// head-major, group-major order).  On a bad index the list stays empty and
-// the error word says where: info = {head, group, 0 query offsets | 1 range
-// pointers | 2 a key range}.
-__global__ void __launch_bounds__(1024) k_na_plan(const int32_t* qoff, const int32_t* runptr,
-                                                  const int2* runs, int BH, int N, int Gq,
-                                                  int Gk, int max_items, int4* items,
-                                                  Header* hdr) {
-  __shared__ int bad;
-  __shared__ int wsum[32];
-  __shared__ int total_s;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) {
-    hdr->err = 0;
-    hdr->err_info[0] = hdr->err_info[1] = hdr->err_info[2] = 0;
-    hdr->work_next = 0;
-    hdr->n_items = 0;
-    bad = 0;
-  }
-  __syncthreads();
-  const int nent = BH * Gq;
+// One thread per (head, query group): check the group's offsets and every key
+// range the attention kernels will follow, and store the group's tile count
+// (ceil(rows / 128) when it has rows and at least one range, else 0).  A bad
+// index stores 0 and sets the error word with info = {head, group, 0 query
+// offsets | 1 range pointers | 2 a key range}.  Block 0 first resets the
+// header's cursor and counts (the error word is reset by the host-side
+// memset below, before this kernel).
+__global__ void __launch_bounds__(256) k_na_check(const int32_t* qoff, const int32_t* runptr,
+                                                  const int2* runs, int BH, int N, int Gq, int Gk,
+                                                  int32_t* counts, Header* hdr) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= BH * Gq) return;
+  const int bh = e / Gq, i = e - bh * Gq;
   const int64_t run_cap = (int64_t)Gq * Gk;
-  for (int e = tid; e < nent; e += blockDim.x) {
-    const int bh = e / Gq, i = e - bh * Gq;
-    const int32_t* qo = qoff + (size_t)bh * (Gq + 1);
-    const int32_t* rp = runptr + (size_t)bh * (Gq + 1);
-    const int q0 = qo[i], q1 = qo[i + 1];
-    if (!(0 <= q0 && q0 <= q1 && q1 <= N)) {
-      set_error(hdr, ERR_INDEX, bh, i, 0);
-      bad = 1;
-      continue;
-    }
+  const int32_t* qo = qoff + (size_t)bh * (Gq + 1);
+  const int32_t* rp = runptr + (size_t)bh * (Gq + 1);
+  int c = 0;
+  const int q0 = qo[i], q1 = qo[i + 1];
+  if (!(0 <= q0 && q0 <= q1 && q1 <= N)) {
+    set_error(hdr, ERR_INDEX, bh, i, 0);
+  } else {
     const int r0 = rp[i], r1 = rp[i + 1];
     if (!(0 <= r0 && r0 <= r1 && r1 <= run_cap)) {
       set_error(hdr, ERR_INDEX, bh, i, 1);
-      bad = 1;
-      continue;
-    }
-    for (int r = r0; r < r1; ++r) {
-      const int2 kr = runs[(size_t)bh * run_cap + r];
-      if (!(0 <= kr.x && kr.x < kr.y && kr.y <= N)) {
-        set_error(hdr, ERR_INDEX, bh, i, 2);
-        bad = 1;
-        break;
+    } else {
+      bool ok = true;
+      for (int r = r0; r < r1 && ok; ++r) {
+        const int2 kr = runs[(size_t)bh * run_cap + r];
+        if (!(0 <= kr.x && kr.x < kr.y && kr.y <= N)) {
+          set_error(hdr, ERR_INDEX, bh, i, 2);
+          ok = false;
+        }
       }
+      if (ok && q1 > q0 && r1 > r0) c = (q1 - q0 + ATT_BM - 1) / ATT_BM;
     }
   }
-  __syncthreads();
-  if (bad) return;
+  counts[e] = c;
+}
 
-  // Contiguous slices of entries per thread keep the list in entry order.
+// One block: unless the check above found a bad index, the exclusive scan of
+// the tile counts and the work list (query tiles of at most 128 rows of each
+// group, in head-major, group-major order).
+__global__ void __launch_bounds__(1024) k_na_plan(const int32_t* qoff, const int32_t* counts,
+                                                  int BH, int Gq, int max_items, int4* items,
+                                                  Header* hdr) {
+  __shared__ int wsum[32];
+  __shared__ int total_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (hdr->err != 0) return;  // written by the check kernel before this launch
+  const int nent = BH * Gq;
+  // contiguous slices of entries per thread keep the list in entry order
   const int per = (nent + (int)blockDim.x - 1) / (int)blockDim.x;
   const int e0 = min(nent, tid * per), e1 = min(nent, e0 + per);
-  auto count = [&](int e) -> int {
-    const int bh = e / Gq, i = e - bh * Gq;
-    const int32_t* qo = qoff + (size_t)bh * (Gq + 1);
-    const int32_t* rp = runptr + (size_t)bh * (Gq + 1);
-    const int nq = qo[i + 1] - qo[i];
-    return (nq > 0 && rp[i + 1] > rp[i]) ? (nq + ATT_BM - 1) / ATT_BM : 0;
-  };
   int local = 0;
-  for (int e = e0; e < e1; ++e) local += count(e);
-  // block-wide exclusive scan of `local`
+  for (int e = e0; e < e1; ++e) local += counts[e];
   int incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(1024) k_na_plan(const int32_t* qoff, const int
   }
   int k = wsum[warp] + incl - local;
   for (int e = e0; e < e1; ++e) {
-    const int c = count(e);
+    const int c = counts[e];
     if (c == 0) continue;
     const int bh = e / Gq, i = e - bh * Gq;
     const int s = qoff[(size_t)bh * (Gq + 1) + i], en = qoff[(size_t)bh * (Gq + 1) + i + 1];
@@ -203,7 +211,8 @@ extern "C" spr_status sparsepr_attend_routed_noalloc(
   if (na_scratch(&base) != cudaSuccess) return SPR_ECUDA;
   uint8_t* b = static_cast<uint8_t*>(base);
   const size_t stats_off = NA_HDR_BYTES;
-  const size_t items_off = stats_off + round256((size_t)BH * sizeof(spr_head_stats));
+  const size_t counts_off = na_counts_off(BH);
+  const size_t items_off = na_items_off(BH, Gq);
   const int max_items = (int)na_max_items(BH, N, Gq);
 
   Ptrs P{};
@@ -235,8 +244,14 @@ extern "C" spr_status sparsepr_attend_routed_noalloc(
   L.max_items = max_items;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  spr_launch(k_na_plan, 1, 1024, 0, st, q_off, run_ptr, static_cast<const int2*>(P.runs), (int)BH,
-             (int)N, (int)Gq, (int)Gk, max_items, P.items, P.hdr);
+  int32_t* counts = reinterpret_cast<int32_t*>(b + counts_off);
+  // the header (error word, cursor, item count) starts each call at zero
+  if (cudaMemsetAsync(P.hdr, 0, sizeof(Header), st) != cudaSuccess) return SPR_ECUDA;
+  const int nent = BH * Gq;
+  spr_launch(k_na_check, (nent + 255) / 256, 256, 0, st, q_off, run_ptr,
+             static_cast<const int2*>(P.runs), (int)BH, (int)N, (int)Gq, (int)Gk, counts, P.hdr);
+  spr_launch(k_na_plan, 1, 1024, 0, st, q_off, static_cast<const int32_t*>(counts), (int)BH,
+             (int)Gq, max_items, P.items, P.hdr);
   if (cudaGetLastError() != cudaSuccess) return SPR_ECUDA;
   if (launch_attend(p, L, P, st) != cudaSuccess) return SPR_ECUDA;
   if (status) {

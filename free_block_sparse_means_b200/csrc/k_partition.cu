@@ -289,7 +289,7 @@ constexpr int GM_SLICES = 8;
 
 template <int D>
 __global__ void __launch_bounds__(256) k_gmean_part(const bf16* Xp, const int32_t* off, int N, int G,
-                                                    float* part) {
+                                                    double* part) {
   constexpr int NV = D / 32;  // values per lane (bf16 pairs: NV / 2)
   __shared__ double red[8][D];
   const int g = blockIdx.x, bh = blockIdx.y, sl = blockIdx.z;
@@ -329,18 +329,22 @@ __global__ void __launch_bounds__(256) k_gmean_part(const bf16* Xp, const int32_
     double t = 0.0;
 #pragma unroll
     for (int q = 0; q < 8; ++q) t += red[q][k];
-    part[(((size_t)bh * G + g) * GM_SLICES + sl) * D + k] = (float)t;
+    part[(((size_t)bh * G + g) * GM_SLICES + sl) * D + k] = t;
   }
 }
 
+// Group means in fp32 (out) and fp64 (out64: the routing logits use them).
 template <int D>
-__global__ void k_gmean_fin(const float* part, const int32_t* off, int G, float* out) {
+__global__ void k_gmean_fin(const double* part, const int32_t* off, int G, float* out,
+                            double* out64) {
   const int g = blockIdx.x, bh = blockIdx.y, k = threadIdx.x;
   const int cnt = off[(size_t)bh * (G + 1) + g + 1] - off[(size_t)bh * (G + 1) + g];
   double t = 0.0;
 #pragma unroll
-  for (int sl = 0; sl < GM_SLICES; ++sl) t += (double)part[(((size_t)bh * G + g) * GM_SLICES + sl) * D + k];
-  out[((size_t)bh * G + g) * D + k] = cnt > 0 ? (float)(t / cnt) : 0.f;
+  for (int sl = 0; sl < GM_SLICES; ++sl) t += part[(((size_t)bh * G + g) * GM_SLICES + sl) * D + k];
+  const double mean = cnt > 0 ? t / cnt : 0.0;
+  out[((size_t)bh * G + g) * D + k] = (float)mean;
+  out64[((size_t)bh * G + g) * D + k] = mean;
 }
 
 // Key objective with the final centroids: sum_n ||z_n - c_{lab_n}||^2 (fp64
@@ -716,8 +720,8 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
              P.part);
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
-  spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.csum);
-  spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.csum, P.kvoff, p.Gk, P.Craw);
+  spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.gpart);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.gpart, P.kvoff, p.Gk, P.Craw, P.craw64);
   spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
   // query groups from the raw queries
   if ((e = lloyd(Q, p.Gq, P.initq, P.centq, P.labq)) != cudaSuccess) return e;
@@ -731,8 +735,8 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
                       st) != cudaSuccess)
     return cudaGetLastError();
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, Q, P.permq, N, BH, P.Qp);
-  spr_launch(k_gmean_part<D>, dim3(p.Gq, BH, GM_SLICES), 256, 0, st, P.Qp, P.qoff, N, p.Gq, P.csum);
-  spr_launch(k_gmean_fin<D>, dim3(p.Gq, BH), D, 0, st, P.csum, P.qoff, p.Gq, P.qbar);
+  spr_launch(k_gmean_part<D>, dim3(p.Gq, BH, GM_SLICES), 256, 0, st, P.Qp, P.qoff, N, p.Gq, P.gpart);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gq, BH), D, 0, st, P.gpart, P.qoff, p.Gq, P.qbar, P.qbar64);
   return cudaGetLastError();
 }
 
@@ -790,8 +794,8 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   const int ggrid = sms * 8;
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
-  spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.csum);
-  spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.csum, P.kvoff, p.Gk, P.Craw);
+  spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.gpart);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.gpart, P.kvoff, p.Gk, P.Craw, P.craw64);
   // P.counts holds |K_j| now; keep a copy of key counts in kv_off differences.
   spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
   const int split_rows = p.Gq > D ? p.Gq : D;
@@ -848,8 +852,8 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
                                         split_rows, P.part + (size_t)BH * 2 * (nchunk + 1));
   // Group-major queries and raw query means
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, Q, P.permq, N, BH, P.Qp);
-  spr_launch(k_gmean_part<D>, dim3(p.Gq, BH, GM_SLICES), 256, 0, st, P.Qp, P.qoff, N, p.Gq, P.csum);
-  spr_launch(k_gmean_fin<D>, dim3(p.Gq, BH), D, 0, st, P.csum, P.qoff, p.Gq, P.qbar);
+  spr_launch(k_gmean_part<D>, dim3(p.Gq, BH, GM_SLICES), 256, 0, st, P.Qp, P.qoff, N, p.Gq, P.gpart);
+  spr_launch(k_gmean_fin<D>, dim3(p.Gq, BH), D, 0, st, P.gpart, P.qoff, p.Gq, P.qbar, P.qbar64);
   return cudaGetLastError();
 }
 

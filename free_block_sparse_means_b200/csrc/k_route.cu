@@ -6,7 +6,8 @@
 // attention mass when its keys sit at the centroid); cells of one query group
 // are ranked by softmax mass (ties to the lower j); a cell's tail mass is the
 // mass ranked at or after it (one minus the cumulative mass before it, summed
-// from the small end so that the tails of peaked rows stay distinct in fp32).
+// from the small end so that the tails of peaked rows stay distinct); all of
+// it in fp64.
 // Tau mode keeps cells whose mass before them is below tau (tail > 1 - tau);
 // budget mode keeps every cell whose tail is at least the smallest threshold
 // for which the true pair cost plus the M*N probe pairs fits rho_target*N^2.
@@ -60,26 +61,28 @@ __device__ int block_exscan(int v, int* sh, int* out) {
   return total;
 }
 
-// L[i][j] = s qbar_i . C_j + ln|K_j| (-inf for empty K/V groups).
+// L[i][j] = s qbar_i . C_j + ln|K_j| (-inf for empty K/V groups), fp64 from
+// the fp64 group means: the routing decision then agrees with an fp64
+// evaluation of the rule up to rounding of the last bits.
 // Grid (BH, ceil(Gq/32), ceil(Gk/32)), block 256.
-__global__ void __launch_bounds__(256) k_route_logits(const float* qbar, const float* Craw,
+__global__ void __launch_bounds__(256) k_route_logits(const double* qbar, const double* Craw,
                                                       const int32_t* kvoff, int Gq, int Gk, int D,
-                                                      float scale, float* L) {
-  __shared__ float As[32][33], Bs[32][33];
+                                                      double scale, double* L) {
+  __shared__ double As[32][33], Bs[32][33];
   const int bh = blockIdx.x, i0 = blockIdx.y * 32, j0 = blockIdx.z * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
   for (int c0 = 0; c0 < D; c0 += 32) {
     for (int e = threadIdx.x; e < 1024; e += 256) {
       const int rr = e >> 5, c = e & 31;
-      As[rr][c] = (i0 + rr < Gq) ? qbar[((size_t)bh * Gq + i0 + rr) * D + c0 + c] : 0.f;
-      Bs[rr][c] = (j0 + rr < Gk) ? Craw[((size_t)bh * Gk + j0 + rr) * D + c0 + c] : 0.f;
+      As[rr][c] = (i0 + rr < Gq) ? qbar[((size_t)bh * Gq + i0 + rr) * D + c0 + c] : 0.0;
+      Bs[rr][c] = (j0 + rr < Gk) ? Craw[((size_t)bh * Gk + j0 + rr) * D + c0 + c] : 0.0;
     }
     __syncthreads();
     for (int c = 0; c < 32; ++c) {
-      const float bv = Bs[tx][c];
+      const double bv = Bs[tx][c];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) acc[k] += As[ty * 4 + k][c] * bv;
+      for (int k = 0; k < 4; ++k) acc[k] = fma(As[ty * 4 + k][c], bv, acc[k]);
     }
     __syncthreads();
   }
@@ -90,81 +93,82 @@ __global__ void __launch_bounds__(256) k_route_logits(const float* qbar, const f
   for (int k = 0; k < 4; ++k) {
     const int i = i0 + ty * 4 + k;
     if (i < Gq)
-      L[((size_t)bh * Gq + i) * Gk + j] = nk > 0 ? scale * acc[k] + logf((float)nk) : -INFINITY;
+      L[((size_t)bh * Gq + i) * Gk + j] = nk > 0 ? scale * acc[k] + log((double)nk) : -INFINITY;
   }
 }
 
 // Softmax mass, rank and tail mass (mass ranked at or after the cell,
 // suffix-summed from the smallest so peaked rows keep distinct tails) of every
-// cell of one query group.  Grid (BH, Gq), block 256 (>= Gk).  Dead cells get
-// tail -1; the top-ranked cell of a live row is flagged in `top`.
-__global__ void __launch_bounds__(256) k_route_mass(const float* L, const int32_t* qoff,
+// cell of one query group, in fp64.  Grid (BH, Gq), block 256 (>= Gk).  Dead
+// cells get tail -1; the top-ranked cell of a live row is flagged in `top`.
+__global__ void __launch_bounds__(256) k_route_mass(const double* L, const int32_t* qoff,
                                                     const int32_t* kvoff, int Gq, int Gk,
-                                                    int tau_mode, double tau, float* tail,
+                                                    int tau_mode, double tau, double* tail,
                                                     uint8_t* top, uint8_t* sel) {
-  __shared__ float shf[32];
-  __shared__ float pis[MAX_GROUPS];
-  __shared__ float sorted[MAX_GROUPS];
+  __shared__ double shf[32];
+  __shared__ double pis[MAX_GROUPS];
+  __shared__ double sorted[MAX_GROUPS];
   const int bh = blockIdx.x, i = blockIdx.y, j = threadIdx.x;
   const int nq = qoff[(size_t)bh * (Gq + 1) + i + 1] - qoff[(size_t)bh * (Gq + 1) + i];
   const size_t cell = ((size_t)bh * Gq + i) * Gk + j;
   bool live = false;
-  float l = -INFINITY;
+  double l = -INFINITY;
   if (j < Gk) {
     const int nk = kvoff[(size_t)bh * (Gk + 1) + j + 1] - kvoff[(size_t)bh * (Gk + 1) + j];
     live = nq > 0 && nk > 0;
     if (live) l = L[cell];
   }
-  const float mx = block_reduce(l, shf, [](float a, float b) { return fmaxf(a, b); });
-  const float w = live ? __expf(l - mx) : 0.f;
-  const float sum = block_reduce(w, shf, [](float a, float b) { return a + b; });
-  const float pi = (live && sum > 0.f) ? w / sum : 0.f;
-  if (j < MAX_GROUPS) pis[j] = j < Gk ? (live ? pi : -1.f) : -2.f;
+  const double mx = block_reduce(l, shf, [](double a, double b) { return fmax(a, b); });
+  const double w = live ? exp(l - mx) : 0.0;
+  const double sum = block_reduce(w, shf, [](double a, double b) { return a + b; });
+  const double pi = (live && sum > 0.0) ? w / sum : 0.0;
+  if (j < MAX_GROUPS) pis[j] = j < Gk ? (live ? pi : -1.0) : -2.0;
   __syncthreads();
   int rank = 0;
   if (j < Gk) {
-    const float mine = live ? pi : -1.f;
+    const double mine = live ? pi : -1.0;
     for (int t = 0; t < Gk; ++t) {
-      const float o = pis[t];
+      const double o = pis[t];
       rank += (o > mine) || (o == mine && t < j);
     }
-    sorted[rank] = live ? pi : 0.f;
+    sorted[rank] = live ? pi : 0.0;
   }
   __syncthreads();
   // suffix (inclusive) sums over sorted masses: reverse index, warp scans
   const int jr = blockDim.x - 1 - j;  // reversed position handled by this thread
-  const float v = (jr < Gk) ? sorted[jr] : 0.f;
-  float x = v;
+  const double v = (jr < Gk) ? sorted[jr] : 0.0;
+  double x = v;
   const int lane = j & 31, wi = j >> 5;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const float t = __shfl_up_sync(0xffffffffu, x, o);
+    const double t = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += t;
   }
   if (lane == 31) shf[wi] = x;
   __syncthreads();
-  float before = 0.f;
+  double before = 0.0;
   for (int t = 0; t < wi; ++t) before += shf[t];
   __syncthreads();
   if (jr < Gk) pis[jr] = before + x;  // tail at sorted position jr
   __syncthreads();
   if (j < Gk) {
-    const float r = live ? pis[rank] : -1.f;
+    const double r = live ? pis[rank] : -1.0;
     tail[cell] = r;
     top[cell] = live && rank == 0;
-    if (tau_mode) sel[cell] = live && ((double)r > 1.0 - tau || rank == 0);
+    if (tau_mode) sel[cell] = live && (r > 1.0 - tau || rank == 0);
   }
 }
 
-// Budget mode: smallest threshold T on the tail-mass bit pattern with
+// Budget mode: smallest threshold T on the tail-mass bit pattern (fp64 tails
+// are non-negative, so their 64-bit patterns order like the values) with
 // cost(bits(tail) >= T) <= rho_target N^2 - M N (exact int64 costs); kept
 // cells are those at or above T plus every row's top cell.
-__global__ void __launch_bounds__(1024) k_route_budget(const float* tail, const uint8_t* top,
+__global__ void __launch_bounds__(1024) k_route_budget(const double* tail, const uint8_t* top,
                                                        const int32_t* qoff, const int32_t* kvoff,
                                                        int Gq, int Gk, int N, int M, double rho,
                                                        uint8_t* sel, spr_head_stats* stats) {
   __shared__ long long shl[32];
-  __shared__ float shf[32];
+  __shared__ double shf[32];
   __shared__ int nqs[MAX_GROUPS], nks[MAX_GROUPS];
   const int bh = blockIdx.x, tid = threadIdx.x;
   for (int g = tid; g < Gq; g += 1024)
@@ -174,13 +178,14 @@ __global__ void __launch_bounds__(1024) k_route_budget(const float* tail, const 
   __syncthreads();
   const double budget = rho * (double)N * (double)N - (double)M * (double)N;
   const int ncell = Gq * Gk;
-  const float* R = tail + (size_t)bh * ncell;
-  auto bits = [](float r) -> long long { return r < 0.f ? -1ll : (long long)__float_as_uint(r); };
+  const double* R = tail + (size_t)bh * ncell;
+  auto bits = [](double r) -> long long { return r < 0.0 ? -1ll : __double_as_longlong(r); };
   // the first RB_CACHE cells of every thread stay in registers (bit pattern,
   // pair count) for the whole search; more cells are read again each round
   constexpr int RB_CACHE = 8;
-  int cb[RB_CACHE];
+  long long cb[RB_CACHE];
   long long cw[RB_CACHE];
+  long long tmin = 0x7FF0000000000000ll, tmax = -1;
 #pragma unroll
   for (int q = 0; q < RB_CACHE; ++q) {
     const int t = tid + q * 1024;
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(1024) k_route_budget(const float* tail, const 
     if (t < ncell) {
       const int i = t / Gk, j = t - i * Gk;
       if (nqs[i] > 0 && nks[j] > 0) {
-        cb[q] = (int)bits(R[t]);
+        cb[q] = bits(R[t]);
         cw[q] = (long long)nqs[i] * nks[j];
       }
     }
@@ -197,19 +202,30 @@ __global__ void __launch_bounds__(1024) k_route_budget(const float* tail, const 
   auto cost = [&](long long T) {
     long long c = 0;
 #pragma unroll
-    for (int q = 0; q < RB_CACHE; ++q) c += (long long)cb[q] >= T ? cw[q] : 0ll;
+    for (int q = 0; q < RB_CACHE; ++q) c += cb[q] >= T ? cw[q] : 0ll;
     for (int t = tid + RB_CACHE * 1024; t < ncell; t += 1024) {
       const int i = t / Gk, j = t - i * Gk;
       if (nqs[i] > 0 && nks[j] > 0 && bits(R[t]) >= T) c += (long long)nqs[i] * nks[j];
     }
     return block_reduce(c, shl, [](long long a, long long b) { return a + b; });
   };
-  // cost(T) is non-increasing in T; cost(0x7F800000) = 0 (no tail reaches +inf).
-  long long lo = -1, hi = 0x7F800000ll;
-  if ((double)cost(0) <= budget) {
-    hi = 0;
+  // the search runs between the smallest and largest live tail patterns
+  for (int t = tid; t < ncell; t += 1024) {
+    const int i = t / Gk, j = t - i * Gk;
+    if (nqs[i] > 0 && nks[j] > 0) {
+      const long long b = bits(R[t]);
+      tmin = b < tmin ? b : tmin;
+      tmax = b > tmax ? b : tmax;
+    }
+  }
+  tmin = block_reduce(tmin, shl, [](long long a, long long b) { return a < b ? a : b; });
+  tmax = block_reduce(tmax, shl, [](long long a, long long b) { return a > b ? a : b; });
+  // cost(T) is non-increasing in T; cost(tmax + 1) = 0.
+  long long Tstar;
+  if (tmax < 0 || (double)cost(tmin) <= budget) {
+    Tstar = tmax < 0 ? 0 : tmin;
   } else {
-    lo = 0;  // infeasible
+    long long lo = tmin, hi = tmax + 1;  // cost(lo) > budget >= cost(hi)
     while (hi - lo > 1) {
       const long long mid = lo + (hi - lo) / 2;
       if ((double)cost(mid) <= budget)
@@ -217,9 +233,9 @@ __global__ void __launch_bounds__(1024) k_route_budget(const float* tail, const 
       else
         lo = mid;
     }
+    Tstar = hi;
   }
-  const long long Tstar = hi;
-  float kept_min = INFINITY;
+  double kept_min = INFINITY;
   int only_top = 1;
   for (int t = tid; t < ncell; t += 1024) {
     const int i = t / Gk, j = t - i * Gk;
@@ -228,11 +244,11 @@ __global__ void __launch_bounds__(1024) k_route_budget(const float* tail, const 
     const bool k = above || (live && top[(size_t)bh * ncell + t]);
     sel[(size_t)bh * ncell + t] = k;
     if (above) {
-      kept_min = fminf(kept_min, R[t]);
+      kept_min = fmin(kept_min, R[t]);
       if (!top[(size_t)bh * ncell + t]) only_top = 0;
     }
   }
-  kept_min = block_reduce(kept_min, shf, [](float a, float b) { return fminf(a, b); });
+  kept_min = block_reduce(kept_min, shf, [](double a, double b) { return fmin(a, b); });
   const long long nt = block_reduce((long long)(1 - only_top), shl,
                                     [](long long a, long long b) { return a + b; });
   if (tid == 0) {
@@ -427,9 +443,9 @@ __global__ void __launch_bounds__(256) k_gather_probe(const bf16* Qp, const int3
 
 cudaError_t launch_route(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st) {
   const int BH = L.BH, D = p.d;
-  const float scale = p.scale > 0.f ? p.scale : 1.f / sqrtf((float)D);
-  spr_launch(k_route_logits, dim3(BH, (p.Gq + 31) / 32, (p.Gk + 31) / 32), 256, 0, st, 
-      P.qbar, P.Craw, P.kvoff, p.Gq, p.Gk, D, scale, P.logit);
+  const double scale = p.scale > 0.f ? (double)p.scale : 1.0 / sqrt((double)D);
+  spr_launch(k_route_logits, dim3(BH, (p.Gq + 31) / 32, (p.Gk + 31) / 32), 256, 0, st,
+             P.qbar64, P.craw64, P.kvoff, p.Gq, p.Gk, D, scale, P.logit);
   const int tau_mode = p.route_mode == SPR_ROUTE_TAU;
   spr_launch(k_route_mass, dim3(BH, p.Gq), 256, 0, st, P.logit, P.qoff, P.kvoff, p.Gq, p.Gk,
              tau_mode, p.tau, P.entry, P.top, P.sel);

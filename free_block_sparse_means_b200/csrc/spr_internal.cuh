@@ -35,7 +35,8 @@ enum Buf : int {
   B_KP, B_VP, B_QP, B_CRAW, B_CT, B_AMAT, B_RMS, B_UN2, B_CENTQ, B_BQ16, B_BETA,
   B_QBAR, B_LOGIT, B_ENTRY, B_TOP, B_SEL, B_ROWPTR, B_COLIDX, B_RUNPTR, B_RUNS, B_PPOS,
   B_PIDX, B_PW, B_PSLOT, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
-  B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_CSUM, B_XP, B_RP, B_PMEAN, B_COUNT_
+  B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_CSUM, B_XP, B_RP, B_PMEAN, B_CRAW64, B_QBAR64,
+  B_COUNT_
 };
 
 struct Layout {
@@ -63,9 +64,12 @@ struct Ptrs {
   Header* hdr;
   spr_head_stats* stats;
   float *MK, *trace, *eval, *evec, *W, *Z, *centk, *Craw, *Ct, *Amat, *rms, *un2, *centq, *beta,
-      *qbar, *logit, *entry, *pw, *osp, *odn, *fitU, *fitB, *fitBv, *gram, *axx, *rxbar,
+      *qbar, *pw, *osp, *odn, *fitU, *fitB, *fitBv, *gram, *axx, *rxbar,
       *proj, *csum, *xp, *rp, *pmean;
   double* part;
+  double *logit, *entry;  // route logits and tail masses [BH][Gq][Gk] (fp64)
+  double *craw64, *qbar64;  // raw-key and raw-query group means (fp64)
+  double* gpart;          // group-mean slice sums (aliases the k-means partial sums)
   int32_t *initk, *initq, *labk, *labq, *chunk, *cbase, *counts, *permk, *kvoff, *permq,
       *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx, *pslot;
   int2* runs;
@@ -97,6 +101,10 @@ cudaError_t launch_attend(const spr_params& p, const Layout& L, const Ptrs& P, c
 // launch_attend uses it for this head dim.
 cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st);
 bool attend_tc_enabled(int d);
+// Load the attention kernels' device code ahead of their first launch (and
+// resolve the tensor-map encoder the tcgen05 kernel needs).
+cudaError_t attend_preload();
+cudaError_t attend_tc_preload();
 cudaError_t launch_reconstruct(const spr_params& p, const Layout& L, const Ptrs& P,
                                bf16* O, cudaStream_t st);
 // Leading eigenpairs of `count` symmetric n x n matrices (fp32, row-major):

@@ -169,7 +169,8 @@ spr_status sparsepr_partition(const spr_params* prm, const void* Q, const void* 
  * s*qbar_i.c_j + ln|K_j|; tau mode keeps cells whose cumulative mass before
  * them is below tau, budget mode keeps the largest such prefix set whose
  * true pair cost plus the M*N probe pairs fits rho_target*N^2 (each group's
- * top cell always kept).  Emits the routed-cell CSR, merged key ranges, M
+ * top cell always kept).  Group means, logits, masses and tails are fp64.
+ * Emits the routed-cell CSR, merged key ranges, M
  * probe rows stratified over query groups with coverage weights (1 / M each
  * with prm->weights = SPR_WEIGHTS_UNIFORM), and the attention work list.
  * Reads and writes only `ws`.
@@ -236,7 +237,7 @@ typedef enum {
   SPR_VIEW_CTILDE = 16,  /* [BH, Gk, d] fp32 centred nonempty K/V centroids,
                             compacted (first gk_nonempty rows) */
   SPR_VIEW_RMS = 17,     /* [BH, N] fp32 query RMS (original order) */
-  SPR_VIEW_TAIL = 18,    /* [BH, Gq, Gk] fp32 tail mass of each cell: softmax mass of
+  SPR_VIEW_TAIL = 18,    /* [BH, Gq, Gk] fp64 tail mass of each cell: softmax mass of
                             the cells ranked at or after it (-1: empty group) */
   SPR_VIEW_FIT_U = 19,   /* [BH, d, d] fp32 residual basis (first r_eff cols) */
   SPR_VIEW_FIT_B = 20,   /* [BH, d, d] fp32 ridge coefficients B (first r_eff
@@ -249,16 +250,17 @@ spr_status sparsepr_workspace_view(const spr_params* prm, int32_t which, size_t*
                                    size_t* bytes);
 
 /*
- * Routed attention with no device memory allocation.  The method has no
- * counterpart to this entry point: it runs the stage-3 computation above
- * (every row of query group i attends, softmax renormalised over the kept
- * keys, to the key ranges routed to i [paperlayer §4 "Sparse Execution"])
- * on group-major inputs the caller supplies, for callers that cannot
+ * Routed attention with no device memory allocation.  The paper has no
+ * counterpart to this entry point: it runs the computation of
+ * sparsepr_attend's routed cells, declared above (every row of query group i
+ * attends, softmax renormalised over the kept keys, to the key ranges routed
+ * to i), on group-major inputs the caller supplies, for callers that cannot
  * allocate device memory where they run it (a launch sequence replayed
  * with fixed addresses, a memory pool partitioned ahead of time, a thread
  * that must not enter the allocator).  It enqueues kernels only: no
  * cudaMalloc, cudaFree or allocating library call, ever.  Its own state (error
- * word, work cursor, per-head counters, work list) lives in a fixed 4 MiB
+ * word, work cursor, per-head counters, per-group tile counts, work list)
+ * lives in a fixed 4 MiB
  * area of device memory inside the library image; nothing has to start at
  * zero, since each call re-initialises that state before using it.
  *
@@ -287,13 +289,17 @@ spr_status sparsepr_workspace_view(const spr_params* prm, int32_t which, size_t*
  * Sizes: BH heads (batch x heads) >= 1, N >= 1 with BH * N < 2^31, d in
  * {64, 128}, 1 <= Gq, Gk <= 256.  scale <= 0 selects 1/sqrt(d).
  *
- * Limit: 256 + 80 * BH (rounded up to 256) + 16 * (BH * (ceil(N / 128) + Gq)
- * + 1) bytes must fit in 4 MiB (e.g. 40 heads of 75,600 tokens with Gq = 256
- * need 0.52 MiB); larger problems return SPR_ESCRATCH and enqueue nothing.
+ * Limit: 256 + 80 * BH (rounded up to 256) + 4 * BH * Gq (rounded up to 256)
+ * + 16 * (BH * (ceil(N / 128) + Gq) + 1) bytes must fit in 4 MiB (e.g. 40
+ * heads of 75,600 tokens with Gq = 256 need 0.56 MiB); larger problems
+ * return SPR_ESCRATCH and enqueue nothing.
  *
- * The first call on each device looks up the scratch area's address and sets
- * the attention kernel's shared-memory limit (runtime calls that may load the
- * library's device code); make that first call before capturing a stream.
+ * The first call on each device does a one-time set-up: it looks up the
+ * scratch area's address, loads every kernel this entry point can launch
+ * (both head dimensions, both attention kernels) and resolves the driver's
+ * tensor-map encoder.  Loading device code may take device memory, so make
+ * that first call before capturing a stream and before any point where
+ * allocation is not allowed; later calls on that device take none.
  * All calls on one device share the one scratch area: two calls that may
  * overlap on the GPU (different streams without ordering between them, or
  * different host threads) race on it and both results are undefined.  Calls

@@ -5,12 +5,15 @@ sampled heads and, for the long sequences, on sampled rows.
   mid      24 heads x 8192 tokens (the benchmark workload): three whole heads
   hunyuan  24 heads x 118,800 tokens: two heads, 2048 sampled rows each
   wan      40 heads x 75,600 tokens: one head, 2048 sampled rows
-The oracle runs driven by the GPU's cluster labels (see gpu_support).
+The oracle runs driven by the GPU's cluster labels (see gpu_support); the
+GPU's k-means is also compared with the oracle's own independent run on one
+head of each, route near-ties are reported and bounded, and every head's
+output must be finite.
 """
 import numpy as np
 import pytest
 
-from gpu_support import check_head, run_gpu
+from gpu_support import check_head, check_kmeans_independent, near_tie_bound, run_gpu
 from synthetic import workload
 
 pytestmark = pytest.mark.gpu
@@ -20,8 +23,13 @@ def test_mid_benchmark_launch_sampled_heads():
     wl = workload("mid")
     check = [0, 11, 23]
     g = run_gpu(wl, check=check)
+    assert g["all_finite"]
     for bh in check:
-        check_head(g, wl, bh)
+        res, _ = check_head(g, wl, bh)
+        near_tie_bound(res)
+        assert res["near_ties"] == 0
+    for bh in check:
+        check_kmeans_independent(g, wl, bh)
     for st in g["stats"]:
         assert 0.2 < st["rho_exec"] <= 0.25 + 1e-9, st["rho_exec"]
 
@@ -30,8 +38,11 @@ def test_mid_benchmark_launch_sampled_heads():
 def test_long_sequences_sampled_rows(name, check):
     wl = workload(name)
     g = run_gpu(wl, check=check)
+    assert g["all_finite"]
     rows = np.sort(np.random.default_rng(7).choice(wl.N, 2048, replace=False))
     for bh in check:
-        check_head(g, wl, bh, rows=rows)
+        res, _ = check_head(g, wl, bh, rows=rows)
+        near_tie_bound(res)
+    check_kmeans_independent(g, wl, check[0])
     for st in g["stats"]:
         assert st["rho_exec"] <= 0.25 + 1e-9, st["rho_exec"]

@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import free_block_sparse_means_b200 as spr
-from gpu_support import check_head, oracle_params, rel_l2, run_gpu
+from gpu_support import (check_head, check_kmeans_independent, near_tie_bound, oracle_params,
+                         rel_l2, run_gpu)
 from oracle import dense_attention
 from synthetic import workload
 
@@ -22,15 +23,19 @@ pytestmark = pytest.mark.gpu
 def test_tiny_full_parity():
     wl = workload("tiny")
     g = run_gpu(wl)
+    assert g["all_finite"]
     res, orc = check_head(g, wl, 0)
     assert res["near_ties"] == 0
+    check_kmeans_independent(g, wl, 0)
 
 
 def test_mid_two_heads_full_length():
     wl = workload("mid", H=2)
     g = run_gpu(wl)
+    assert g["all_finite"]
     for bh in range(2):
         res, _ = check_head(g, wl, bh)
+        assert res["near_ties"] == 0
         st = g["stats"][bh]
         assert 0.2 < st["rho_exec"] <= 0.25 + 1e-9, st["rho_exec"]
 
