@@ -7,8 +7,9 @@
 One step = one whole SparsePR call (partition, route, routed attention with
 exact probe rows, probe-fitted reconstruction and un-permute) over a batch of
 seeded synthetic Voronoi-center video tokens.  The default workload is the
-single-layer mid size: 24 heads x 8192 tokens (8x32x32 grid), d = 128, bf16,
-budget routing at rho_exec = 25% including probes.
+HunyuanVideo-13B-shaped attention call: 24 heads x 118,800 tokens (33x45x80
+latent grid), d = 128, bf16, 256 K/V and 256 query groups, budget routing at
+rho_exec = 25% including probes, M = 1024 probes, r = 32.
 
 Metric: dense-equivalent TFLOP/s = 4 d N^2 (heads) / call time (higher is
 better); the JSON line also carries ms per call, executed-pair TFLOP/s, the
@@ -51,12 +52,15 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def profiled_traffic(workload_name: str):
+def profiled_traffic(workload_name: str, heads: int):
     """DRAM bytes per attention launch from the committed ncu summary, or None.
 
-    The figure holds only for the kernel source it was captured from and for
-    the same workload: a changed source (its hash no longer matches) or another
-    workload gives None.
+    The summary states the DRAM bytes of one launch over `heads_captured`
+    heads of the workload (a capture of every head of the long workloads
+    would break the capture-size rule); heads are independent units of equal
+    size, so the figure scales by heads / heads_captured.  It holds only for
+    the kernel source it was captured from: a changed source (its hash no
+    longer matches) or another workload gives None.
     """
     import hashlib
     prof = os.path.join(ROOT, "profiles", f"k_attend_tc_{workload_name}.md")
@@ -67,13 +71,15 @@ def profiled_traffic(workload_name: str):
     with open(prof) as f:
         for line in f:
             k, sep, v = line.strip().partition(":")
-            if sep and k in ("kernel_source_sha256_16", "workload", "traffic_bytes_per_launch"):
+            if sep and k in ("kernel_source_sha256_16", "workload", "traffic_bytes_per_launch",
+                             "heads_captured"):
                 fields[k] = v.strip()
     with open(src, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()[:16]
     if fields.get("kernel_source_sha256_16") != sha or fields.get("workload") != workload_name:
         return None
-    return int(fields["traffic_bytes_per_launch"])
+    captured = int(fields.get("heads_captured", heads))
+    return int(round(int(fields["traffic_bytes_per_launch"]) * heads / captured))
 
 
 def dist_info():
@@ -166,30 +172,68 @@ def blas_cores():
         return os.cpu_count() or 1
 
 
-def oracle_head_seconds(wl, bh):
-    """Seconds the fp64 oracle takes for one whole head (independent mode)."""
-    from oracle import Params, sparsepr_head
+ORACLE_WHOLE_HEAD_MAX_N = 16384  # longer heads: attention rows sampled and extrapolated
+
+
+def oracle_head_seconds(wl, bh, sample_rows=2048):
+    """Seconds the fp64 oracle takes for one whole head (independent mode).
+
+    Up to ORACLE_WHOLE_HEAD_MAX_N tokens the head runs whole.  Longer heads
+    run the whole partition, route, probes (exact dense rows) and fit, but
+    the hard-drop attention of only `sample_rows` rows; that part's time is
+    measured on its own (the oracle's hard_drop_attention on the sampled
+    rows) and scaled to all N rows (rows are independent, each costs about
+    the same).  Returns (seconds, description of the sample).
+    """
+    from oracle import Params, hard_drop_attention, sparsepr_head
     prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
                  tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index,
                  partition=wl.partition, weights=wl.weights)
     Q, K, V = voronoi_qkv(wl, heads=[bh])
     q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
+    if wl.N <= ORACLE_WHOLE_HEAD_MAX_N:
+        t0 = time.perf_counter()
+        sparsepr_head(q, k, v, prm, bh=bh)
+        return time.perf_counter() - t0, "whole head"
+    import numpy as np
+    rows = np.sort(np.random.default_rng(bh).choice(wl.N, sample_rows, replace=False))
     t0 = time.perf_counter()
-    sparsepr_head(q, k, v, prm, bh=bh)
-    return time.perf_counter() - t0
+    out = sparsepr_head(q, k, v, prm, bh=bh, rows=rows)
+    t1 = time.perf_counter()
+    hard_drop_attention(q, k, v, out["lab_q"], out["lab_k"], out["row_ptr"], out["col_idx"],
+                        out["scale"], rows=rows)
+    t_rows = time.perf_counter() - t1
+    total = (t1 - t0) + t_rows * (wl.N / sample_rows - 1.0)
+    return total, (f"whole partition, route, probes and fit; hard-drop attention of "
+                   f"{sample_rows} sampled rows scaled to {wl.N}")
 
 
 def oracle_baseline(wl, budget_s=10.0):
-    """The oracle as it stands on whole heads of the workload, ~budget_s of CPU work."""
-    heads, t_tot = 0, 0.0
+    """The oracle as it stands on heads of the workload, ~budget_s of CPU work
+    (at least one head), scaled to all heads."""
+    heads, t_tot, how = 0, 0.0, ""
     while heads < wl.BH and (heads == 0 or t_tot < budget_s):
-        t_tot += oracle_head_seconds(wl, heads)
+        t, how = oracle_head_seconds(wl, heads)
+        t_tot += t
         heads += 1
     flops = 4.0 * wl.d * wl.N * wl.N * heads
     return {"value": flops / t_tot / 1e12, "unit": "TFLOP/s (dense-equivalent)",
             "cores": blas_cores(), "kind": "oracle",
-            "sample": f"{heads} of {wl.BH} heads of {wl.name}, whole call, fp64 numpy, "
+            "sample": f"{heads} of {wl.BH} heads of {wl.name} ({how}), fp64 numpy, "
                       f"{t_tot:.1f} s"}
+
+
+def partition_bytes(wl):
+    """Algorithmic HBM bytes of the partition stage per call: every pass reads
+    its input once and writes its output once.  Per head, with row bytes
+    qb = kb = 2d (bf16) and zb = 128 (32 fp32 key coordinates):
+      query RMS pass and T query assignments: (T + 1) qb N;
+      key projection: kb N read + zb N written; T key assignments: T zb N;
+      group-major copies of Q, K and V: 3 (read + write) 2d N;
+      group means of the permuted keys and queries: 2 qb N."""
+    qb, zb, T, N = 2.0 * wl.d, 128.0, wl.iters, wl.N
+    per_head = ((T + 1) * qb + qb + zb + T * zb + 3 * 2 * qb + 2 * qb) * N
+    return per_head * wl.BH
 
 
 def config_of(wl, world):
@@ -209,9 +253,9 @@ def run_reference(args, wl):
     world, rank, _ = dist_info()
     if rank != 0:
         return 0
-    times = []
+    times, how = [], ""
     for s in range(args.warmup + args.steps):
-        t = oracle_head_seconds(wl, s % wl.BH)
+        t, how = oracle_head_seconds(wl, s % wl.BH, sample_rows=args.ref_rows)
         if s >= args.warmup:
             times.append(t)
     t = statistics.mean(times)
@@ -220,9 +264,10 @@ def run_reference(args, wl):
     line = {"metric": METRIC, "value": val, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference", "config": config_of(wl, 1),
+            "data": "synthetic", "impl": "reference",
+            "config": dict(config_of(wl, 1), kmeans_start="seeded"),
             "cpu_baseline": {"value": val, "unit": unit, "cores": blas_cores(), "kind": "oracle",
-                             "sample": f"one whole head of {wl.name} per step"},
+                             "sample": f"one head of {wl.name} per step ({how})"},
             "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -250,6 +295,7 @@ def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=1024, seed=0):
     q, k, v, o = (t.reshape(BH, N, d) for t in (Q, K, V, O))
     scale = 1.0 / d ** 0.5
     num_hd = num_sp = den = e_res = e_aff = e_orth = 0.0
+    row_hd, row_sp = [], []
     for bh in range(BH):
         s = (q[bh, rows].float() @ k[bh].float().T) * scale
         dense = torch.softmax(s, dim=-1) @ v[bh].float()
@@ -257,6 +303,9 @@ def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=1024, seed=0):
         sp = o[bh, rows].float()
         num_hd += float(((hd - dense) ** 2).sum())
         num_sp += float(((sp - dense) ** 2).sum())
+        dn = dense.norm(dim=1).clamp_min(1e-30)
+        row_hd.append(((hd - dense).norm(dim=1) / dn).double().cpu())
+        row_sp.append(((sp - dense).norm(dim=1) / dn).double().cpu())
         den += float((dense ** 2).sum())
         R = (dense - hd).double()
         F = torch.cat([hd.double(), torch.ones(hd.shape[0], 1, dtype=torch.float64, device=dev)], 1)
@@ -264,8 +313,13 @@ def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=1024, seed=0):
         e_res += float((R * R).sum())
         e_aff += float((P * P).sum())
         e_orth += float(((R - P) ** 2).sum())
+    row_hd, row_sp = torch.cat(row_hd), torch.cat(row_sp)
     return {"rows_sampled_per_head": int(rows.numel()), "dense": 0.0,
             "hard_drop": (num_hd / den) ** 0.5, "sparsepr": (num_sp / den) ** 0.5,
+            "row_error_hard_drop": {"mean": float(row_hd.mean()),
+                                    "p99": float(torch.quantile(row_hd, 0.99))},
+            "row_error_sparsepr": {"mean": float(row_sp.mean()),
+                                   "p99": float(torch.quantile(row_sp, 0.99))},
             "o3_affine_fraction": e_aff / e_res if e_res > 0 else 0.0,
             "o3_orthogonal_energy_rel": e_orth / den}
 
@@ -422,8 +476,11 @@ def run_ours(args, wl):
     per_call = [sum(x) for x in stage]
     total_ms = sum(per_call)
     stage_mean = [statistics.mean(x[i] for x in stage) for i in range(4)]
-    mx = reduce_max([total_ms] + stage_mean, world, dev)
-    total_ms_max, stage_max = mx[0], mx[1:]
+    srt = sorted(per_call)
+    med = statistics.median(srt)
+    p90 = srt[min(len(srt) - 1, int(0.9 * (len(srt) - 1) + 0.5))]
+    mx = reduce_max([total_ms] + stage_mean + [med, p90], world, dev)
+    total_ms_max, stage_max, med_max, p90_max = mx[0], mx[1:5], mx[5], mx[6]
     ms_per_call = total_ms_max / args.steps
     dense_flop = 4.0 * wl.d * wl.N * wl.N * wl.BH  # per rank
     value = dense_flop * world / (ms_per_call * 1e-3) / 1e12
@@ -437,10 +494,10 @@ def run_ours(args, wl):
     roof = {"bound": "tensor", "kernel": "k_attend (routed cells + probe rows)",
             "achieved": att_achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": att_achieved / peaks["bf16_tflops"], "peak_source": f"{peak_kind} bf16 burst",
-            "traffic": profiled_traffic(wl.name), "algorithmic_flop_per_launch": 4.0 * wl.d * pairs,
+            "traffic": profiled_traffic(wl.name, wl.BH),
+            "algorithmic_flop_per_launch": 4.0 * wl.d * pairs,
             "executed_tile_pairs": tile_pairs, "true_pairs": pairs}
-    # partition: algorithmic HBM bytes (reads of Q, K, V per pass and the permuted copies)
-    part_bytes = float(wl.BH * wl.N * wl.d * 2) * ((wl.iters + 3) + (wl.iters + 2) + 2 * 3)
+    part_bytes = partition_bytes(wl)
     part_gbs = part_bytes / (stage_max[0] * 1e-3) / 1e9
     # end to end through the public API with host buffers (pinned)
     Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
@@ -470,7 +527,7 @@ def run_ours(args, wl):
                 {"iters": args.warm_iters,
                  "kmeans_start": "warm (previous call's centroids; first warm-up call seeded)"}
                 if args.warm_iters > 0 else {"kmeans_start": "seeded"})),
-            "ms_per_call": ms_per_call,
+            "ms_per_call": ms_per_call, "ms_per_call_median": med_max, "ms_per_call_p90": p90_max,
             "exec_pair_tflops": exec_tflops * world, "rho_exec": rho,
             "stage_ms": {"partition": stage_max[0], "route": stage_max[1], "attend": stage_max[2],
                          "reconstruct": stage_max[3]},
@@ -499,10 +556,12 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mid")
+    ap.add_argument("--workload", default="hunyuan")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=2048,
+                    help="reference arm on long workloads: attention rows sampled per head")
     ap.add_argument("--warm-iters", type=int, default=0,
                     help="T > 0: the first warm-up call is seeded, every later call starts its "
                          "k-means from the previous call's centroids and runs T iterations")

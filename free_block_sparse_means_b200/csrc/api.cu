@@ -50,7 +50,7 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_RMS] = BH * N * 4;
   sz[B_UN2] = BH * N * 4;
   sz[B_CENTQ] = BH * Gq * d * 4;
-  sz[B_BQ16] = BH * 2 * (Gm > d ? Gm : d) * d * 2;  // semantic mode: key groups too
+  sz[B_BQ16] = BH * 2 * (size_t)bq_rows((int)Gm, (int)d) * d * 2;  // semantic mode: key groups too
   sz[B_BETA] = BH * Gm * 4;
   sz[B_QBAR] = BH * Gq * d * 4;
   sz[B_LOGIT] = BH * Gq * Gk * 8;
@@ -77,15 +77,21 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_RXBAR] = BH * 2 * d * 4;
   sz[B_PROJ] = BH * (M ? (M + 63) / 64 : 1) * d * (p->r > 0 ? p->r : 1) * 4;  // fit rhs partials
   sz[B_PART] = part_slots * 8;
-  // k-means partial sums: per chunk, one slot per (group, warp segment)
-  sz[B_CSUM] = BH * nchunk * (Gm + CSUM_SLOTS) * (d > P ? d : P) * 4;
-  if (sz[B_CSUM] < BH * Gm * 8 * d * 8) sz[B_CSUM] = BH * Gm * 8 * d * 8;  // group-mean slices (fp64)
+  // k-means partial sums (one per label present in each 128-row tile), also
+  // the group-mean slices (fp64)
+  sz[B_CSUM] = lloyd_slot_bytes((int)BH, (int)N, (int)d);
+  if (sz[B_CSUM] < BH * Gm * 8 * d * 8) sz[B_CSUM] = BH * Gm * 8 * d * 8;
   // probe rows gathered for the fit: sparse outputs X, residuals R, block means
   sz[B_XP] = BH * (M ? M : 1) * d * 4;
   sz[B_RP] = BH * (M ? M : 1) * d * 4;
   sz[B_PMEAN] = BH * (M ? (M + 31) / 32 : 1) * 2 * d * 4;
   sz[B_CRAW64] = BH * Gk * d * 8;
   sz[B_QBAR64] = BH * Gq * d * 8;
+  const size_t ntile = (N + 127) / 128, nword = (ntile + 31) / 32;
+  sz[B_SLOTCNT] = BH * ntile * LLOYD_SLOTS * 4;
+  sz[B_TMASK] = BH * ntile * 8 * 4;
+  sz[B_GBITS] = BH * Gm * nword * 4;
+  sz[B_BK16] = BH * 2 * (size_t)lloyd_ncrows((int)Gk) * 64 * 2;
   size_t off = 0;
   for (int i = 0; i < B_COUNT_; ++i) {
     L->off[i] = off;
@@ -169,6 +175,10 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.craw64 = AT(double*, B_CRAW64);
   P.qbar64 = AT(double*, B_QBAR64);
   P.gpart = AT(double*, B_CSUM);
+  P.slotcnt = AT(int32_t*, B_SLOTCNT);
+  P.tmask = AT(uint32_t*, B_TMASK);
+  P.gbits = AT(uint32_t*, B_GBITS);
+  P.bk16 = AT(bf16*, B_BK16);
 #undef AT
   return P;
 }
@@ -206,7 +216,8 @@ spr_status sparsepr_check_params(const spr_params* p) {
   if (p->d != 64 && p->d != 128) return SPR_EUNSUPPORTED;
   if ((int64_t)p->B * p->H * p->N > (int64_t)1 << 30) return SPR_EUNSUPPORTED;
   if (p->Ms < 1 || p->Ms > p->N) return SPR_EINVAL;
-  if (p->p < 1 || p->p > p->d || p->p > MAX_P) return SPR_EINVAL;
+  if (p->p < 1 || p->p > p->d) return SPR_EINVAL;
+  if (p->p > MAX_P) return SPR_EUNSUPPORTED;
   if (p->Gk < 1 || p->Gq < 1 || p->Gk > p->N || p->Gq > p->N) return SPR_EINVAL;
   if (p->Gk > MAX_GROUPS || p->Gq > MAX_GROUPS) return SPR_EUNSUPPORTED;
   if (p->iters < 1 || p->iters > 100) return SPR_EINVAL;

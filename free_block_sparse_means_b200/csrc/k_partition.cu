@@ -10,7 +10,7 @@
 
 namespace spr {
 
-int padded_p(int p) { return p <= 8 ? 8 : p <= 16 ? 16 : p <= 32 ? 32 : 64; }
+int padded_p(int) { return 32; }
 
 // ---------------------------------------------------------------------------
 // M_K = Q_s^T Q_s / M_s with Q_s the rows floor(i N / M_s), i < M_s.
@@ -216,69 +216,6 @@ __global__ void __launch_bounds__(CHUNK) k_scatter(const int32_t* lab, int N, in
     else
       perm[(size_t)bh * N + pos] = n;
   }
-}
-
-// Group means from the chunk partial sums.  Grid (G, BH), one thread per
-// coordinate; an empty group keeps its previous centroid.  The block first
-// lists the slots holding the group (chunk by chunk, warp segment by warp
-// segment), then every thread adds its coordinate over the list with four
-// interleaved fp64 accumulators (fixed assignment, so the order is fixed).
-template <int DD>
-__global__ void k_chunk_reduce(const float* part, const int32_t* chunk_cnt, const int32_t* loff,
-                               int G, int nchunk, float* out) {
-  extern __shared__ int cred[];  // [nchunk] counts, [nchunk] list starts, slot list
-  int* cc = cred;
-  int* cs = cred + nchunk;
-  int* list = cred + 2 * nchunk;
-  __shared__ int nlist;
-  __shared__ long long tot_s;
-  const int bh = blockIdx.y, g = blockIdx.x, i = threadIdx.x;
-  for (int c = i; c < nchunk; c += blockDim.x) {
-    const size_t idx = ((size_t)bh * nchunk + c) * G + g;
-    const int n = chunk_cnt[idx];
-    cc[c] = n;
-    cs[c] = n > 0 ? min((loff[idx] + n - 1) >> 5, CSUM_SLOTS - 1) - (loff[idx] >> 5) + 1 : 0;
-    list[c] = n > 0 ? loff[idx] >> 5 : 0;  // first warp segment, moved below
-  }
-  __syncthreads();
-  if (i == 0) {  // exclusive scan of the per-chunk slot counts, totals
-    int acc = 0;
-    long long tot = 0;
-    for (int c = 0; c < nchunk; ++c) {
-      const int k = cs[c];
-      cs[c] = acc;
-      acc += k;
-      tot += cc[c];
-    }
-    nlist = acc;
-    tot_s = tot;
-  }
-  __syncthreads();
-  // slot offsets (relative to the part buffer of this head), chunk-major
-  for (int c = i; c < nchunk; c += blockDim.x) cc[c] = cc[c] > 0 ? list[c] : -1;
-  __syncthreads();
-  int* slots = list + nchunk;
-  for (int c = i; c < nchunk; c += blockDim.x) {
-    if (cc[c] < 0) continue;
-    const int n = (c + 1 < nchunk ? cs[c + 1] : nlist) - cs[c];
-    for (int k = 0; k < n; ++k) slots[cs[c] + k] = c * (G + CSUM_SLOTS) + g + cc[c] + k;
-  }
-  __syncthreads();
-  if (i >= DD || tot_s == 0) return;
-  const float* base = part + (size_t)bh * nchunk * (G + CSUM_SLOTS) * DD + i;
-  const int n = nlist;
-  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-  int k = 0;
-  for (; k + 3 < n; k += 4) {
-    s0 += (double)base[(size_t)slots[k] * DD];
-    s1 += (double)base[(size_t)slots[k + 1] * DD];
-    s2 += (double)base[(size_t)slots[k + 2] * DD];
-    s3 += (double)base[(size_t)slots[k + 3] * DD];
-  }
-  if (k < n) s0 += (double)base[(size_t)slots[k] * DD];
-  if (k + 1 < n) s1 += (double)base[(size_t)slots[k + 1] * DD];
-  if (k + 2 < n) s2 += (double)base[(size_t)slots[k + 2] * DD];
-  out[((size_t)bh * G + g) * DD + i] = (float)(((s0 + s1) + (s2 + s3)) / (double)tot_s);
 }
 
 // Means of the contiguous group-major bf16 rows of each group, balanced over
@@ -676,7 +613,7 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
   const int BH = L.BH, N = p.N, nchunk = L.nchunk;
   const float scale = p.scale > 0.f ? p.scale : 1.f / sqrtf((float)D);
   const int Gm = p.Gk > p.Gq ? p.Gk : p.Gq;
-  const int split_rows = Gm > D ? Gm : D;
+  const int split_rows = bq_rows(Gm, D);
   const int ggrid = num_sms() * 8;
   cudaError_t e;
   spr_launch(k_semantic_setup, dim3(64, BH), 256, 0, st, P.Amat, P.rms, D, N, scale);
@@ -685,30 +622,37 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
                    int32_t* lab) -> cudaError_t {
     if (p.init != SPR_INIT_WARM)  // warm: cent holds the previous call's raw-row centroids
       spr_launch(k_init_centq, BH, 256, 0, st, X, N, G, D, init, P.rms, scale, cent);
+    if (cudaMemsetAsync(P.gbits, 0, L.bytes[B_GBITS], st) != cudaSuccess) return cudaGetLastError();
+    LloydStep ls{};
+    ls.mode = KM_QUERY;
+    ls.d = D;
+    ls.N = N;
+    ls.G = G;
+    ls.BH = BH;
+    ls.split_rows = split_rows;
+    ls.X = X;
+    ls.bq = P.bq16;
+    ls.rms = P.rms;
+    ls.scale = scale;
+    ls.beta = P.beta;
+    ls.cent = cent;
+    ls.lab = lab;
+    ls.slots = P.csum;
+    ls.slot_cnt = P.slotcnt;
+    ls.tmask = P.tmask;
+    ls.gbits = P.gbits;
+    ls.hdr = P.hdr;
+    ls.slots_bytes = L.bytes[B_CSUM];
+    ls.slot_cnt_bytes = L.bytes[B_SLOTCNT];
+    ls.tmask_bytes = L.bytes[B_TMASK];
+    ls.gbits_bytes = L.bytes[B_GBITS];
     for (int it = 0; it < p.iters; ++it) {
       spr_launch(k_qprep, dim3(BH, G), D, 0, st, P.Amat, cent, G, D, P.counts, P.beta, P.bq16,
                  split_rows, nullptr);
-      KmArgs a{};
-      a.Q = X;
-      a.rms = P.rms;
-      a.scale = scale;
-      a.bsplit = P.bq16;
-      a.split_rows = split_rows;
-      a.beta = P.beta;
-      a.N = N;
-      a.G = G;
-      a.nchunk = nchunk;
-      a.lab = lab;
-      a.chunk_cnt = P.chunk;
-      a.loff = P.cbase;
-      a.part = P.csum;
-      a.hdr = P.hdr;
-      const cudaError_t e2 = launch_kmeans_step(KM_QUERY, D, a, nchunk, BH, st);
+      const cudaError_t e2 = lloyd_step(ls, st);
       if (e2 != cudaSuccess) return e2;
-      spr_launch(k_chunk_reduce<D>, dim3(G, BH), D, (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int), st,
-                 P.csum, P.chunk, P.cbase, G, nchunk, cent);
     }
-    return cudaSuccess;
+    return label_hist(lab, N, G, nchunk, BH, P.chunk, P.hdr, st);
   };
   // K/V groups from the raw keys; the k-means centroids live in Craw until
   // the group means of the permuted keys replace them
@@ -762,34 +706,39 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   else
     spr_launch(k_init_centk, BH, 256, 0, st, P.Z, N, p.Gk, pp, P.initk, P.centk);
   // Key k-means
-  for (int it = 0; it < p.iters; ++it) {
-    KmArgs ka{};
-    ka.Z = P.Z;
-    ka.cent = P.centk;
-    ka.N = N;
-    ka.G = p.Gk;
-    ka.nchunk = nchunk;
-    ka.lab = P.labk;
-    ka.chunk_cnt = P.chunk;
-    ka.loff = P.cbase;
-    ka.part = P.csum;
-    ka.hdr = P.hdr;
-    if ((e = launch_kmeans_step(KM_KEY, pp, ka, nchunk, BH, st)) != cudaSuccess) return e;
-    const size_t rsm = (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int);
-#define KRED(PPV)                                                                             \
-  spr_launch(k_chunk_reduce<PPV>, dim3(p.Gk, BH), ((PPV) + 31) / 32 * 32, rsm, st, P.csum, \
-             P.chunk, P.cbase, p.Gk, nchunk, P.centk)
-    if (pp == 8) KRED(8); else if (pp == 16) KRED(16); else if (pp == 32) KRED(32); else KRED(64);
-#undef KRED
+  if (cudaMemsetAsync(P.gbits, 0, L.bytes[B_GBITS], st) != cudaSuccess) return cudaGetLastError();
+  if ((e = lloyd_key_operand(P.centk, p.Gk, BH, P.bk16, P.beta, st)) != cudaSuccess) return e;
+  {
+    LloydStep ks{};
+    ks.mode = KM_KEY;
+    ks.d = D;
+    ks.N = N;
+    ks.G = p.Gk;
+    ks.BH = BH;
+    ks.Z = P.Z;
+    ks.bk = P.bk16;
+    ks.beta = P.beta;
+    ks.cent = P.centk;
+    ks.lab = P.labk;
+    ks.slots = P.csum;
+    ks.slot_cnt = P.slotcnt;
+    ks.tmask = P.tmask;
+    ks.gbits = P.gbits;
+    ks.hdr = P.hdr;
+    ks.slots_bytes = L.bytes[B_CSUM];
+    ks.slot_cnt_bytes = L.bytes[B_SLOTCNT];
+    ks.tmask_bytes = L.bytes[B_TMASK];
+    ks.gbits_bytes = L.bytes[B_GBITS];
+    for (int it = 0; it < p.iters; ++it)
+      if ((e = lloyd_step(ks, st)) != cudaSuccess) return e;
   }
+  if ((e = label_hist(P.labk, N, p.Gk, nchunk, BH, P.chunk, P.hdr, st)) != cudaSuccess) return e;
   // group-major key order of the final labels
   spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gk, N, P.cbase, P.kvoff, P.counts);
   spr_launch(k_scatter, dim3(nchunk, BH), CHUNK, 0, st, P.labk, N, p.Gk, nchunk, P.cbase, P.kvoff,
              P.permk, P.hdr);
-#define OBJZ(PPV) \
-  spr_launch(k_obj_z<PPV>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.labk, nchunk, P.part)
-  if (pp == 8) OBJZ(8); else if (pp == 16) OBJZ(16); else if (pp == 32) OBJZ(32); else OBJZ(64);
-#undef OBJZ
+spr_launch(k_obj_z<32>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.labk, nchunk,
+             P.part);
   // Paired K/V groups: permuted keys and values, raw-key centroids
   const int ggrid = sms * 8;
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
@@ -798,7 +747,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.gpart, P.kvoff, p.Gk, P.Craw, P.craw64);
   // P.counts holds |K_j| now; keep a copy of key counts in kv_off differences.
   spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
-  const int split_rows = p.Gq > D ? p.Gq : D;
+  const int split_rows = bq_rows(p.Gk > p.Gq ? p.Gk : p.Gq, D);
   spr_launch(k_amat, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, P.Ct, p.Gk, D, P.stats, P.Amat, P.bq16,
                                                          split_rows);
   // Query-response RMS (tensor-core quadratic form)
@@ -821,28 +770,38 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   // Query k-means in the head dimension
   if (p.init != SPR_INIT_WARM)  // warm: centq keeps the previous call's head-dim centroids
     spr_launch(k_init_centq, BH, 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale, P.centq);
-  for (int it = 0; it < p.iters; ++it) {
-    spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta, P.bq16,
-                                          split_rows, nullptr);
-    KmArgs qa{};
-    qa.Q = Q;
-    qa.rms = P.rms;
-    qa.scale = scale;
-    qa.bsplit = P.bq16;
-    qa.split_rows = split_rows;
-    qa.beta = P.beta;
-    qa.N = N;
-    qa.G = p.Gq;
-    qa.nchunk = nchunk;
-    qa.lab = P.labq;
-    qa.chunk_cnt = P.chunk;
-    qa.loff = P.cbase;
-    qa.part = P.csum;
-    qa.hdr = P.hdr;
-    if ((e = launch_kmeans_step(KM_QUERY, D, qa, nchunk, BH, st)) != cudaSuccess) return e;
-    spr_launch(k_chunk_reduce<D>, dim3(p.Gq, BH), D, (size_t)(3 + CSUM_SLOTS) * nchunk * sizeof(int), st, P.csum,
-               P.chunk, P.cbase, p.Gq, nchunk, P.centq);
+  if (cudaMemsetAsync(P.gbits, 0, L.bytes[B_GBITS], st) != cudaSuccess) return cudaGetLastError();
+  {
+    LloydStep qs{};
+    qs.mode = KM_QUERY;
+    qs.d = D;
+    qs.N = N;
+    qs.G = p.Gq;
+    qs.BH = BH;
+    qs.split_rows = split_rows;
+    qs.X = Q;
+    qs.bq = P.bq16;
+    qs.rms = P.rms;
+    qs.scale = scale;
+    qs.beta = P.beta;
+    qs.cent = P.centq;
+    qs.lab = P.labq;
+    qs.slots = P.csum;
+    qs.slot_cnt = P.slotcnt;
+    qs.tmask = P.tmask;
+    qs.gbits = P.gbits;
+    qs.hdr = P.hdr;
+    qs.slots_bytes = L.bytes[B_CSUM];
+    qs.slot_cnt_bytes = L.bytes[B_SLOTCNT];
+    qs.tmask_bytes = L.bytes[B_TMASK];
+    qs.gbits_bytes = L.bytes[B_GBITS];
+    for (int it = 0; it < p.iters; ++it) {
+      spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta,
+                 P.bq16, split_rows, nullptr);
+      if ((e = lloyd_step(qs, st)) != cudaSuccess) return e;
+    }
   }
+  if ((e = label_hist(P.labq, N, p.Gq, nchunk, BH, P.chunk, P.hdr, st)) != cudaSuccess) return e;
   // group-major query order of the final labels
   spr_launch(k_chunk_scan, BH, 256, 0, st, P.chunk, nchunk, p.Gq, N, P.cbase, P.qoff, P.counts);
   spr_launch(k_scatter, dim3(nchunk, BH), CHUNK, 0, st, P.labq, N, p.Gq, nchunk, P.cbase, P.qoff,

@@ -14,10 +14,9 @@ typedef __nv_bfloat16 bf16;
 
 constexpr int CHUNK = 512;         // rows per histogram chunk (k-means, permutation)
 constexpr int MAX_GROUPS = 256;    // Gk, Gq upper bound
-constexpr int MAX_P = 64;          // eigen-coordinate upper bound
+constexpr int MAX_P = 32;          // eigen-coordinate upper bound (coordinates padded to 32)
 constexpr int MAX_PROBES = 4096;   // M upper bound
 constexpr int ATT_BM = 128;        // query rows per attention work item
-constexpr int CSUM_SLOTS = CHUNK / 32;  // extra partial-sum slots per chunk (one per warp)
 
 // Device error word codes (first error wins; info words carry details).
 enum : int32_t {
@@ -36,7 +35,7 @@ enum Buf : int {
   B_QBAR, B_LOGIT, B_ENTRY, B_TOP, B_SEL, B_ROWPTR, B_COLIDX, B_RUNPTR, B_RUNS, B_PPOS,
   B_PIDX, B_PW, B_PSLOT, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
   B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_CSUM, B_XP, B_RP, B_PMEAN, B_CRAW64, B_QBAR64,
-  B_COUNT_
+  B_SLOTCNT, B_TMASK, B_GBITS, B_BK16, B_COUNT_
 };
 
 struct Layout {
@@ -56,8 +55,13 @@ struct Header {
 };
 
 bool make_layout(const spr_params* p, Layout* L);
-// Eigen-coordinate count rounded up to 8, 16, 32 or 64 (zero-padded columns).
+// Eigen-coordinate width: 32 (p <= 32; columns past p are zero).
 int padded_p(int p);
+// Rows per head of the query k-means operand buffer: max(round32(Gmax), d).
+inline int bq_rows(int Gmax, int d) {
+  const int nc = (Gmax + 31) / 32 * 32;
+  return nc > d ? nc : d;
+}
 
 // Pointers of one call, resolved from the workspace base.
 struct Ptrs {
@@ -71,7 +75,9 @@ struct Ptrs {
   double *craw64, *qbar64;  // raw-key and raw-query group means (fp64)
   double* gpart;          // group-mean slice sums (aliases the k-means partial sums)
   int32_t *initk, *initq, *labk, *labq, *chunk, *cbase, *counts, *permk, *kvoff, *permq,
-      *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx, *pslot;
+      *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx, *pslot, *slotcnt;
+  uint32_t *tmask, *gbits;  // k-means update bookkeeping
+  bf16* bk16;               // key k-means operand [BH][2][round32(Gk)][64]
   int2* runs;
   int4* items;
   uint8_t *sel, *top;
@@ -114,28 +120,41 @@ cudaError_t launch_eig(const float* A, int count, int n, int K, float* evals, fl
                        float* trace, cudaStream_t st);
 int num_sms();
 
-// One fused Lloyd iteration (assignment, chunk histogram and sort, segmented
-// partial sums) of the query (KM_QUERY, width = d) or key (KM_KEY, width =
-// padded eigen-coordinate count) k-means; grid (nchunk, BH).
 enum { KM_QUERY = 0, KM_KEY = 1 };
-struct KmArgs {
-  TensorView Q;           // query rows
-  const float* Z;         // key rows [BH][N][width]
-  const float* rms;       // query row RMS; the update rows are (scale / rms) q
+// One Lloyd iteration (assignment on the tensor cores, then the update) of
+// the query (KM_QUERY: rows of X, width d, operand bq from k_qprep) or key
+// (KM_KEY: rows of Z, 32 coordinates, operand bk) k-means; cent receives the
+// new centroids (and, key mode, bk the next operand).
+constexpr int LLOYD_SLOTS = 128;
+struct LloydStep {
+  int mode, d, N, G, BH, split_rows;
+  TensorView X;        // query mode: the rows ([B, H, N, d] view)
+  const float* Z;      // key mode: [BH][N][32] coordinates
+  const bf16* bq;      // query mode: [BH][2][split_rows][d] operand (hi, lo)
+  bf16* bk;            // key mode: [BH][2][lloyd_ncrows(G)][64] operand (hi, lo)
+  const float* rms;    // query mode: row RMS (factor scale / rms)
   float scale;
-  const bf16* bsplit;     // query: [BH][2][split_rows][d] bf16 hi, lo of Bq_g
-  int split_rows;
-  const float* beta;      // query: [BH][G]
-  const float* cent;      // key: [BH][G][width] centroids
-  int N, G, nchunk;
-  int32_t* lab;           // [BH][N] labels (out)
-  int32_t* chunk_cnt;     // [BH][nchunk][G] chunk label histograms (out)
-  int32_t* loff;          // [BH][nchunk][G] chunk-local group offsets (out)
-  float* part;            // [BH][nchunk][G + CSUM_SLOTS][width] partial sums (out)
+  const float* beta;   // [BH][G]: query beta_g (k_qprep); key ||c_g||^2 / 2 (written by the update)
+  float* cent;         // [BH][G][width] centroids, updated in place
+  int32_t* lab;        // [BH][N] labels (out)
+  float* slots;        // lloyd_slot_bytes(BH, N, d): per-tile partial sums
+  int32_t* slot_cnt;   // [BH * ceil(N / 128)][LLOYD_SLOTS]
+  uint32_t* tmask;     // [BH * ceil(N / 128)][8]
+  uint32_t* gbits;     // [BH][G][ceil(ceil(N / 128) / 32)], zero before the first step
   Header* hdr;
+  // capacities in bytes of slots, slot_cnt, tmask, gbits (checked before launch)
+  size_t slots_bytes, slot_cnt_bytes, tmask_bytes, gbits_bytes;
 };
-cudaError_t launch_kmeans_step(int mode, int width, const KmArgs& a, int nchunk, int BH,
-                               cudaStream_t st);
+cudaError_t lloyd_step(const LloydStep& s, cudaStream_t st);
+// Key operand rows and beta_g = ||c_g||^2 / 2 from centroids (first iteration).
+cudaError_t lloyd_key_operand(const float* cent, int G, int BH, bf16* bk, float* beta,
+                              cudaStream_t st);
+int lloyd_ncrows(int G);
+size_t lloyd_slot_bytes(int BH, int N, int d);
+// Chunk label histograms [BH][nchunk][G] (for k_chunk_scan / k_scatter).
+cudaError_t label_hist(const int32_t* lab, int N, int G, int nchunk, int BH, int32_t* chunk_cnt,
+                       Header* hdr, cudaStream_t st);
+
 // Key-response coordinates Z = K W (tensor cores); W is [BH][d][pp] fp32.
 cudaError_t launch_project(const TensorView& K, int N, int D, int PP, int BH, const float* W,
                            float* Z, Header* hdr, cudaStream_t st);

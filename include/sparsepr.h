@@ -107,7 +107,8 @@ typedef struct {
   float scale;        /* softmax scale; <= 0 selects 1/sqrt(d) */
   /* Response-Coupled Partitioning [paperlayer App. B.1, B.2] */
   int32_t Ms;         /* sampled queries, 1..N (rows floor(i*N/Ms)) */
-  int32_t p;          /* key-response eigen-coordinates, 1..min(d, 64) */
+  int32_t p;          /* key-response eigen-coordinates, 1..min(d, 32)
+                         (SPR_EUNSUPPORTED above 32) */
   int32_t Gk, Gq;     /* K/V groups and query groups, 1..min(N, 256) */
   int32_t iters;      /* Lloyd iterations of both k-means, 1..100 */
   uint64_t seed;      /* k-means initial rows (splitmix64 partial shuffle) */
@@ -229,9 +230,9 @@ typedef enum {
   SPR_VIEW_PROBE_W = 10, /* [BH, M] fp32 coverage weights (sum 1) */
   SPR_VIEW_O_SPARSE = 11,/* [BH, N, d] fp32 hard-drop output, permuted order */
   SPR_VIEW_O_PROBE = 12, /* [BH, M, d] fp32 exact dense probe rows */
-  SPR_VIEW_W_KEY = 13,   /* [BH, d, pp] fp32 key-response projection; pp = p rounded
-                            up to 8, 16, 32 or 64, extra columns zero */
-  SPR_VIEW_CENT_K = 14,  /* [BH, Gk, pp] fp32 key centroids (eigen-coordinates) */
+  SPR_VIEW_W_KEY = 13,   /* [BH, d, 32] fp32 key-response projection; columns
+                            p .. 31 are zero */
+  SPR_VIEW_CENT_K = 14,  /* [BH, Gk, 32] fp32 key centroids (eigen-coordinates) */
   SPR_VIEW_CENT_Q = 15,  /* [BH, Gq, d] fp32 query centroids a_g: the u-space
                             centroid is Ctilde a_g */
   SPR_VIEW_CTILDE = 16,  /* [BH, Gk, d] fp32 centred nonempty K/V centroids,

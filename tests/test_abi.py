@@ -85,6 +85,9 @@ def test_validation(lib):
     prm = _params()
     prm.d = 96
     assert spr.sparsepr_check_params(prm) == spr._binding.SPR_EUNSUPPORTED
+    # key coordinates are padded to 32 columns: p up to 32
+    assert spr.sparsepr_check_params(_params(p=33)) == spr._binding.SPR_EUNSUPPORTED
+    assert spr.sparsepr_check_params(_params(p=7)) == 0
     assert spr.sparsepr_check_params(_params(partition="semantic")) == 0
     for field in ("partition", "init", "weights"):
         prm = _params()

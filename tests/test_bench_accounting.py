@@ -1,0 +1,27 @@
+"""The bench's partition byte count, worked by hand for the mid workload."""
+import importlib.util
+import os
+
+from synthetic import workload
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+def test_partition_bytes_mid_by_hand():
+    # mid: 24 heads x 8192 rows, d = 128 (256 B per bf16 row), 32 fp32 key
+    # coordinates (128 B per row), T = 10 iterations.  Per row:
+    #   RMS + 10 query assignments 11 x 256; projection 256 + 128;
+    #   10 key assignments 10 x 128; three permuted copies 3 x 512;
+    #   two group-mean passes 2 x 256
+    #   2816 + 384 + 1280 + 1536 + 512            -> 6528 B per row
+    wl = workload("mid")
+    per_row = 11 * 256 + 256 + 128 + 10 * 128 + 3 * 512 + 2 * 256
+    assert per_row == 6528
+    assert _bench().partition_bytes(wl) == per_row * 8192 * 24
