@@ -92,6 +92,7 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_TMASK] = BH * ntile * 8 * 4;
   sz[B_GBITS] = BH * Gm * nword * 4;
   sz[B_BK16] = BH * 2 * (size_t)lloyd_ncrows((int)Gk) * 64 * 2;
+  sz[B_ZHL] = BH * N * 64 * 2;
   size_t off = 0;
   for (int i = 0; i < B_COUNT_; ++i) {
     L->off[i] = off;
@@ -179,6 +180,7 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.tmask = AT(uint32_t*, B_TMASK);
   P.gbits = AT(uint32_t*, B_GBITS);
   P.bk16 = AT(bf16*, B_BK16);
+  P.zhl = AT(bf16*, B_ZHL);
 #undef AT
   return P;
 }

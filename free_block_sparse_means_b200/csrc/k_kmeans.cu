@@ -1,5 +1,5 @@
 // Key-response coordinates Z = K W on the tensor cores [paperlayer App. B.1]
-// (the input rows of the key k-means).
+// (the input rows of the key k-means), in fp32 and as bf16 hi | lo rows.
 #include <float.h>
 
 #include "spr_internal.cuh"
@@ -34,10 +34,12 @@ __device__ __forceinline__ uint4 split8(const float* v, bool lo) {
 // products), fp32 accumulation in TMEM.  One 128-row tile per block:
 // A = the tile (K-major SW128, cp.async), B = W^T hi / lo ([n][k] rows, n
 // padded to NP >= 32 with zeros), D = 128 x NP in TMEM; four warps write one
-// Z row (pp floats) per thread.
+// Z row (pp floats) per thread, and its split z_hi = bf16(z), z_lo =
+// bf16(z - z_hi) as one 128-byte row (the k-means assignment's operand).
 template <int D, int PP>
 __global__ void __launch_bounds__(KM_THREADS, 1) k_project_tc(TensorView K, int N, const float* W, float* Z,
-                                                              Header* hdr) {
+                                                              bf16* Zhl, Header* hdr) {
+  static_assert(PP == 32, "the hi | lo rows hold 32 coordinates");
   constexpr int NP = PP < 32 ? 32 : PP;  // UMMA N (and TMEM columns)
   constexpr int NCH = D / 8, NBOX = D / 64;
   extern __shared__ uint8_t pr_raw[];
@@ -113,6 +115,15 @@ __global__ void __launch_bounds__(KM_THREADS, 1) k_project_tc(TensorView K, int 
           for (int q = 0; q < (PP < 32 ? PP : 32) / 4; ++q)
             dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
                                  __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+          float z[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) z[i] = __uint_as_float(v[i]);
+          uint4* hl = reinterpret_cast<uint4*>(Zhl + ((size_t)bh * N + n) * 64);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            hl[j] = split8(z + 8 * j, false);
+            hl[4 + j] = split8(z + 8 * j, true);
+          }
         }
       }
     }
@@ -135,22 +146,22 @@ __global__ void __launch_bounds__(KM_THREADS, 1) k_project_tc(TensorView K, int 
 
 template <int D, int PP>
 static cudaError_t proj_launch(const TensorView& K, int N, int BH, const float* W, float* Z,
-                               Header* hdr, cudaStream_t st) {
+                               bf16* Zhl, Header* hdr, cudaStream_t st) {
   constexpr int NP = PP < 32 ? 32 : PP;
   const size_t sm = 1024 + (size_t)(D / 64) * (KM_BOX + 2 * NP * 128) + 64;
   cudaError_t e = cudaFuncSetAttribute(k_project_tc<D, PP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sm);
   if (e != cudaSuccess) return e;
   spr_launch(k_project_tc<D, PP>, dim3((N + KM_TILE - 1) / KM_TILE, BH), KM_THREADS, sm, st, K, N, W,
-             Z, hdr);
+             Z, Zhl, hdr);
   return cudaGetLastError();
 }
 
 cudaError_t launch_project(const TensorView& K, int N, int D, int PP, int BH, const float* W,
-                           float* Z, Header* hdr, cudaStream_t st) {
-if (PP != 32) return cudaErrorInvalidValue;
-  if (D == 128) return proj_launch<128, 32>(K, N, BH, W, Z, hdr, st);
-  if (D == 64) return proj_launch<64, 32>(K, N, BH, W, Z, hdr, st);
+                           float* Z, bf16* Zhl, Header* hdr, cudaStream_t st) {
+  if (PP != 32) return cudaErrorInvalidValue;
+  if (D == 128) return proj_launch<128, 32>(K, N, BH, W, Z, Zhl, hdr, st);
+  if (D == 64) return proj_launch<64, 32>(K, N, BH, W, Z, Zhl, hdr, st);
   return cudaErrorInvalidValue;
 }
 

@@ -1,30 +1,36 @@
 // One Lloyd iteration of the partition's two k-means [paperlayer App. B.1,
-// B.2; App. C.1 names a GPU k-means] as a persistent, warp-specialised kernel
-// plus a reducer.
+// B.2; App. C.1 names a GPU k-means]: a persistent, warp-specialised
+// assignment kernel on the tensor cores, an update kernel that sums each
+// tile's rows per label, and a reducer.
 //
-// Assignment (k_lloyd): each block takes a contiguous range of 128-row tiles
-// of the flattened (head, tile) sequence; the tensor cores score every row of
-// a tile against every centroid (tcgen05.mma kind::f16, bf16 operands in
-// 128-byte-swizzled shared memory, fp32 accumulators in TMEM) and one thread
-// per row takes the argmax (ties to the lowest group index):
+// Assignment (k_lloyd_assign): each block takes a contiguous range of
+// 128-row tiles of the flattened (head, tile) sequence; the tensor cores
+// score every row of a tile against every centroid (tcgen05.mma kind::f16,
+// bf16 operands in 128-byte-swizzled shared memory, fp32 accumulators in
+// TMEM) and one thread per row takes the argmax (ties to the lowest group
+// index):
 //   query rows: score_g = (s / rms_n) q . Bq_g - beta_g; q exact in bf16, Bq_g
 //               split into bf16 hi + lo (two products);
 //   key rows:   score_g = z . c_g - beta_g with beta_g = ||c_g||^2 / 2 in
-//               fp32; z and c_g split into hi + lo (three products: hh, hl,
-//               lh).
-// Roles: warp 0 lane 0 issues TMA loads (data tiles into an NS-stage ring; the
-// centroid operand once per head); warp 1 owns TMEM (two score buffers) and
-// one of its threads issues the products; warps 4-7 hold one row each (=
-// TMEM lane): they convert key tiles to hi / lo, take the argmax of tile t
-// while the products of tile t + 1 run, then sort the tile's rows stably by
-// label and sum each label's run of update rows ((s / rms) q or z, read from
-// the tile in shared memory) in fixed order.  A tile writes one partial sum
-// and row count per label present, at the label's rank among the labels
-// present; its 256-bit presence mask; and, per label, one bit of a
-// group-major tile bitmap (integer OR, so its final value does not depend on
-// timing).
+//               fp32; z (read as its bf16 hi | lo copy) and c_g split into
+//               hi + lo (three products: hh, hl, lh).
+// Roles: warp 8 lane 0 issues TMA loads (data tiles into an NS-stage ring, the
+// centroid operand once per head); warp 9 owns TMEM (two score buffers) and
+// one of its threads issues the products; a data stage is released by the
+// commit of its products.  Warps 0-3 and 4-7 are two groups of row threads
+// (warp w reads TMEM lanes 32 (w % 4) ..) that take alternate tiles, each with
+// its own score buffer, so two row warps share every scheduler.
 //
-// Update (k_lloyd_reduce): per (head, group), the tiles holding the group
+// Update (k_lloyd_update): one warp per tile sorts the tile's 128 (label,
+// row) keys in registers (bitonic network, keys unique so the order within a
+// label is the row order) and sums the update rows ((s / rms) q or the fp32
+// z) of each label in that order, one run per label; run r of the sorted
+// order (the rank of its label among the labels present) goes to slot r of
+// the tile, with its row count, the tile's 256-bit label mask and, per label,
+// one bit of a group-major tile bitmap (integer OR, so its final value does
+// not depend on timing).
+//
+// Reduction (k_lloyd_reduce): per (head, group), the tiles holding the group
 // (from the bitmap, in tile order), their partial sums added in that order in
 // fp64, divided by the count; an empty group keeps its centroid.  Every sum is
 // taken in an order fixed by the data alone, so results are deterministic.
@@ -42,26 +48,29 @@ namespace spr {
 
 namespace {
 
-constexpr int LL_THREADS = 256;
+constexpr int LL_THREADS = 320;              // warps 0-7 rows, 8 producer, 9 TMEM / products
+constexpr int LL_PRODUCER = 8;
+constexpr int LL_MMA = 9;
 constexpr int LL_TILE = 128;                 // rows per tile (the UMMA M)
 constexpr uint32_t LL_BOX = LL_TILE * 128;   // one 64-column bf16 SW128 box of a tile: 16 KB
 constexpr int LL_KW = 32;                    // key coordinates per row (p padded)
 constexpr int LL_KSTEPS_KEY = LL_KW / 16;    // key K = 32 coordinates
-constexpr uint32_t LL_MISC = 8192;
+constexpr uint32_t LL_MISC = 8 * 1024 + 256; // eight warps' beta rows, barriers
 constexpr uint32_t LL_SMEM_LIMIT = 227 * 1024;
 constexpr uint64_t LL_WAIT_NS = 2000000000ull;
-constexpr int LL_ROW0 = 128;                 // first thread of the row role (warps 4-7)
-constexpr int LL_SLOTS = LLOYD_SLOTS;        // partial sums per tile: at most one per row
+constexpr int LL_SLOTS = LLOYD_SLOTS;        // partial sums per tile (labels present <= 128)
+constexpr int LU_WARPS = 4;                  // update: tiles per block
 
 struct LlPlan {
-  int NC, NCS, nboxA, nboxB, NS;
-  uint32_t tcols, stage_bytes, b_bytes, aset_bytes;
-  uint32_t off_bl, off_aset, off_stage, off_misc, total;
+  int NC, NCS, nboxB, NS;
+  uint32_t tcols, stage_bytes, b_bytes;
+  uint32_t off_bl, off_stage, off_misc, total;
 };
 
 // Shared memory (from a 1024-aligned base): centroid operand hi, lo (nboxB
-// boxes of NC rows x 128 B each); key mode: two hi / lo conversion sets; the
-// data stages; the misc area.  TMEM: two score buffers of NCS columns.
+// boxes of NC rows x 128 B each); the data stages (query: d / 64 boxes of the
+// bf16 rows; key: one box of the hi | lo rows); the misc area.  TMEM: two
+// score buffers of NCS columns.
 template <int MODE, int DK>
 __host__ __device__ inline LlPlan ll_plan(int G) {
   LlPlan p;
@@ -69,21 +78,11 @@ __host__ __device__ inline LlPlan ll_plan(int G) {
   p.NCS = 32;
   while (p.NCS < p.NC) p.NCS <<= 1;
   p.tcols = 2u * (uint32_t)p.NCS;
-  if (MODE == KM_QUERY) {
-    p.nboxA = DK / 64;
-    p.nboxB = DK / 64;
-    p.stage_bytes = (uint32_t)p.nboxA * LL_BOX;
-    p.aset_bytes = 0;
-  } else {
-    p.nboxA = 1;
-    p.nboxB = 1;
-    p.stage_bytes = LL_TILE * LL_KW * 4;
-    p.aset_bytes = 2 * LL_BOX;  // hi box, lo box (64 of their 128 bytes per row used)
-  }
+  p.nboxB = MODE == KM_QUERY ? DK / 64 : 1;
+  p.stage_bytes = MODE == KM_QUERY ? (uint32_t)(DK / 64) * LL_BOX : LL_BOX;
   p.b_bytes = (uint32_t)p.nboxB * (uint32_t)p.NC * 128u;
   p.off_bl = p.b_bytes;
-  p.off_aset = 2 * p.b_bytes;
-  p.off_stage = p.off_aset + 2 * p.aset_bytes;
+  p.off_stage = 2 * p.b_bytes;
   const int avail = (int)LL_SMEM_LIMIT - 1024 - (int)LL_MISC - (int)p.off_stage;
   int ns = avail > 0 ? avail / (int)p.stage_bytes : 0;
   p.NS = ns > 4 ? 4 : ns;
@@ -93,33 +92,13 @@ __host__ __device__ inline LlPlan ll_plan(int G) {
 }
 
 struct LlArgs {
-  int N, G, BH, H, ntile, nword;
+  int N, G, BH, H, ntile;
   float scale;
   const float* rms;    // query: row RMS; the factor of row n is scale / rms[n]
   const float* beta;   // [BH][G]: query beta_g; key ||c_g||^2 / 2
   int32_t* lab;        // [BH][N] labels (out)
-  float* slots;        // [BH * ntile][LL_SLOTS][W] partial sums (out)
-  int32_t* slot_cnt;   // [BH * ntile][LL_SLOTS] rows per partial sum (out)
-  uint32_t* tmask;     // [BH * ntile][8] labels present in each tile (out)
-  uint32_t* gbits;     // [BH][G][nword] tiles holding each label (OR-ed in)
   Header* hdr;
 };
-
-__device__ __forceinline__ uint4 split8(const float* v, bool lo) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const bf16 h0 = __float2bfloat16_rn(v[2 * i]), h1 = __float2bfloat16_rn(v[2 * i + 1]);
-    w[i] = lo ? pack_bf16(v[2 * i] - __bfloat162float(h0), v[2 * i + 1] - __bfloat162float(h1))
-              : pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Byte offset of 16-byte chunk c of row r inside a 128-byte-swizzled box.
-__device__ __forceinline__ uint32_t swz128(int r, int c) {
-  return (uint32_t)(r * 128 + (((c ^ r) & 7) << 4));
-}
 
 __device__ __forceinline__ int warp_incl_scan(int x, int lane) {
 #pragma unroll
@@ -130,12 +109,78 @@ __device__ __forceinline__ int warp_incl_scan(int x, int lane) {
   return x;
 }
 
+// Scores of one row (this thread's TMEM lane) in columns 0 .. NC - 1 of a
+// score buffer: argmax over g < G of f * s_g - beta_g (query) or s_g - beta_g
+// (key), ties to the lowest g.  Eight chains take the columns in increasing
+// order with a strict comparison; the chains are merged by (score, index).
+template <int MODE>
+__device__ __forceinline__ int row_argmax(uint32_t taddr, int NC, int G, float f,
+                                          const float* betas) {
+  float best[8];
+  int bi[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    best[q] = -FLT_MAX;
+    bi[q] = 0;
+  }
+  for (int c0 = 0; c0 < NC; c0 += 64) {
+    uint32_t v[64];
+    const bool two = c0 + 32 < NC;
+    __syncwarp();
+    tc::tmem_ld32(taddr + (uint32_t)c0, v);
+    if (two) tc::tmem_ld32(taddr + (uint32_t)c0 + 32u, v + 32);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int cb = c0 + 32 * h;
+      if (h == 1 && !two) break;
+      if (cb + 32 <= G) {
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 be = *reinterpret_cast<const float4*>(betas + cb + 4 * j4);
+          const float bq[4] = {be.x, be.y, be.z, be.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * j4 + e, q = j & 7;
+            const float x = __uint_as_float(v[32 * h + j]);
+            const float sc = MODE == KM_QUERY ? fmaf(f, x, -bq[e]) : x - bq[e];
+            if (sc > best[q]) {
+              best[q] = sc;
+              bi[q] = cb + j;
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int g = cb + j, q = j & 7;
+          if (g < G) {
+            const float x = __uint_as_float(v[32 * h + j]);
+            const float sc = MODE == KM_QUERY ? fmaf(f, x, -betas[g]) : x - betas[g];
+            if (sc > best[q]) {
+              best[q] = sc;
+              bi[q] = g;
+            }
+          }
+        }
+      }
+    }
+  }
+  float bb = best[0];
+  int arg = bi[0];
+#pragma unroll
+  for (int q = 1; q < 8; ++q)
+    if (best[q] > bb || (best[q] == bb && bi[q] < arg)) {
+      bb = best[q];
+      arg = bi[q];
+    }
+  return arg;
+}
+
 template <int MODE, int DK>
 __global__ void __launch_bounds__(LL_THREADS, 1)
-    k_lloyd(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
-            LlArgs a) {
-  constexpr int W = MODE == KM_QUERY ? DK : LL_KW;  // update-row width
-  constexpr int VPL = W / 32;                        // update values per lane
+    k_lloyd_assign(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                   LlArgs a) {
   extern __shared__ uint8_t ll_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ll_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -144,29 +189,18 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
   const int NC = pl.NC, NCS = pl.NCS, NS = pl.NS;
   uint8_t* Bh = sm;
   uint8_t* Bl = sm + pl.off_bl;
-  uint8_t* Aset = sm + pl.off_aset;
   uint8_t* stg = sm + pl.off_stage;
   uint8_t* misc = sm + pl.off_misc;
-  float* betas = reinterpret_cast<float*>(misc);           // [256]
-  float* rowf = betas + 256;                               // [128]
-  int* lof = reinterpret_cast<int*>(rowf + 128);           // [256] run start of each label
-  int* lidx = lof + 256;                                   // [256] rank among labels present
-  int* srt = lidx + 256;                                   // [128] row | label << 8, sorted
-  uint32_t* cntw32 = reinterpret_cast<uint32_t*>(srt + 128);  // [256] words = [4][256] bytes
-  uint8_t* cntw = reinterpret_cast<uint8_t*>(cntw32);
-  int* scanw = reinterpret_cast<int*>(cntw32 + 256);       // [8]
-  int* sbeg = scanw + 8;                                   // [4] first run start per warp
-  int* stop_s = sbeg + 4;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 5376);
+  float* betas_all = reinterpret_cast<float*>(misc);       // [8 warps][256]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 8 * 1024);
   uint64_t* d_full = bars;        // [4]
   uint64_t* d_empty = bars + 4;   // [4]
-  uint64_t* a_ready = bars + 8;   // [2]
-  uint64_t* s_full = bars + 10;   // [2]
-  uint64_t* s_free = bars + 12;   // [2]
-  uint64_t* b_full = bars + 14;
-  uint64_t* b_free = bars + 15;
-  uint64_t* drain = bars + 16;
-  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* s_full = bars + 8;    // [2]
+  uint64_t* s_free = bars + 10;   // [2]
+  uint64_t* b_full = bars + 12;
+  uint64_t* b_free = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_s + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -177,10 +211,9 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
   if (tid == 0) {
     for (int s = 0; s < 4; ++s) {
       tc::mbar_init(d_full + s, 1);
-      tc::mbar_init(d_empty + s, 4);
+      tc::mbar_init(d_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(a_ready + s, 4);
       tc::mbar_init(s_full + s, 1);
       tc::mbar_init(s_free + s, 4);
     }
@@ -188,14 +221,13 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
     tc::mbar_init(b_free, 1);
     tc::mbar_init(drain, 1);
     *abort_s = 0;
-    *stop_s = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == LL_PRODUCER && lane == 0) {
     tc::prefetch_tmap(&tmX);
     tc::prefetch_tmap(&tmB);
   }
-  if (warp == 1) {
+  if (warp == LL_MMA) {
     tc::tmem_alloc(tmem_s, pl.tcols);
     tc::tmem_relinquish();
   }
@@ -205,7 +237,7 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
   const uint32_t tbase = *tmem_s;
   auto head_of = [&](int t) { return t / a.ntile; };
 
-  if (warp == 0) {
+  if (warp == LL_PRODUCER) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int k = 0, nb = 0, loads = 0;
@@ -227,7 +259,7 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
         if (MODE == KM_QUERY) {
           // [B, H, N, d] view: coordinates (column, row, head, batch)
           const int bb = bh / a.H, hh = bh - bb * a.H;
-          for (int j = 0; j < pl.nboxA; ++j)
+          for (int j = 0; j < DK / 64; ++j)
             tc::tma_load_4d(dst + (uint32_t)j * LL_BOX, &tmX, 64 * j, tl * LL_TILE, hh, bb,
                             d_full + s);
         } else {
@@ -240,14 +272,13 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
           if (q >= 0) tc::mbar_wait_bounded(d_full + (q % NS), (q / NS) & 1, 100000000ull);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == LL_MMA) {
     // ------------------------------------------------------------ products
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16(LL_TILE, NC, 0);
       const uint32_t bh_addr = smem_u32(Bh), bl_addr = smem_u32(Bl);
       int k = 0, nb = 0;
-      bool ok = true;
-      for (int t = tb; t < te && ok; ++t, ++k) {
+      for (int t = tb; t < te; ++t, ++k) {
         const int bh = head_of(t);
         const bool hstart = t == tb || bh != head_of(t - 1);
         const bool hend = t + 1 == te || head_of(t + 1) != bh;
@@ -256,16 +287,12 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
           ++nb;
         }
         const int s = k % NS, b = k & 1;
-        if (MODE == KM_QUERY) {
-          if (!tc::mbar_wait(d_full + s, (k / NS) & 1, abort_s, LL_WAIT_NS)) break;
-        } else {
-          if (!tc::mbar_wait(a_ready + b, (k >> 1) & 1, abort_s, LL_WAIT_NS)) break;
-        }
+        if (!tc::mbar_wait(d_full + s, (k / NS) & 1, abort_s, LL_WAIT_NS)) break;
         if (k >= 2 && !tc::mbar_wait(s_free + b, ((k >> 1) - 1) & 1, abort_s, LL_WAIT_NS)) break;
         tc::tc_fence_after();
         const uint32_t d = tbase + (uint32_t)(b * NCS);
+        const uint32_t a_addr = smem_u32(stg + (uint32_t)s * pl.stage_bytes);
         if (MODE == KM_QUERY) {
-          const uint32_t a_addr = smem_u32(stg + (uint32_t)s * pl.stage_bytes);
 #pragma unroll
           for (int ks = 0; ks < DK / 16; ++ks) {
             const uint32_t ao = (ks >> 2) * LL_BOX + (ks & 3) * 32;
@@ -276,295 +303,247 @@ __global__ void __launch_bounds__(LL_THREADS, 1)
                        tc::smem_desc_sw128(bl_addr + bo, 16, 1024), idesc, 1);
           }
         } else {
-          const uint32_t ah = smem_u32(Aset + (uint32_t)b * pl.aset_bytes), al = ah + LL_BOX;
+          // row = z_hi (columns 0-31) | z_lo (columns 32-63)
 #pragma unroll
           for (int ks = 0; ks < LL_KSTEPS_KEY; ++ks) {
             const uint32_t o = ks * 32;
-            tc::mma_ss(d, tc::smem_desc_sw128(ah + o, 16, 1024),
+            tc::mma_ss(d, tc::smem_desc_sw128(a_addr + o, 16, 1024),
                        tc::smem_desc_sw128(bh_addr + o, 16, 1024), idesc, ks > 0);
-            tc::mma_ss(d, tc::smem_desc_sw128(ah + o, 16, 1024),
+            tc::mma_ss(d, tc::smem_desc_sw128(a_addr + o, 16, 1024),
                        tc::smem_desc_sw128(bl_addr + o, 16, 1024), idesc, 1);
-            tc::mma_ss(d, tc::smem_desc_sw128(al + o, 16, 1024),
+            tc::mma_ss(d, tc::smem_desc_sw128(a_addr + 64 + o, 16, 1024),
                        tc::smem_desc_sw128(bh_addr + o, 16, 1024), idesc, 1);
           }
         }
+        tc::mma_commit(d_empty + s);  // the stage is free once these products are done
         tc::mma_commit(s_full + b);
         if (hend) tc::mma_commit(b_free);
       }
       tc::mma_commit(drain);  // every product issued so far completes before TMEM is freed
       tc::mbar_wait_bounded(drain, 0, LL_WAIT_NS);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ rows
-    const int r = tid - LL_ROW0, rw = warp - 4;
-    const uint32_t lane_f = (uint32_t)(rw * 32) << 16;
-    const unsigned lt_mask = (1u << lane) - 1u;
+    const int grp = warp >> 2, quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_f = (uint32_t)(quarter * 32) << 16;
+    float* betas = betas_all + warp * 256;
     int cur_bh = -1;
-    bool ok = true;
-    // key tiles: fp32 rows -> hi / lo bf16 conversion set (k & 1)
-    auto convert = [&](int kk) -> bool {
-      const int s = kk % NS;
-      bool got = tc::mbar_wait(d_full + s, (kk / NS) & 1, abort_s, LL_WAIT_NS);
-      got = __all_sync(0xffffffffu, got);
-      if (!got) return false;
-      const uint8_t* src = stg + (uint32_t)s * pl.stage_bytes;
-      float z[LL_KW];
-#pragma unroll
-      for (int c = 0; c < LL_KW / 4; ++c) {
-        const float4 v = *reinterpret_cast<const float4*>(src + swz128(r, c));
-        z[4 * c] = v.x;
-        z[4 * c + 1] = v.y;
-        z[4 * c + 2] = v.z;
-        z[4 * c + 3] = v.w;
-      }
-      uint8_t* ah = Aset + (uint32_t)(kk & 1) * pl.aset_bytes;
-#pragma unroll
-      for (int j = 0; j < LL_KW / 8; ++j) {
-        *reinterpret_cast<uint4*>(ah + swz128(r, j)) = split8(z + 8 * j, false);
-        *reinterpret_cast<uint4*>(ah + LL_BOX + swz128(r, j)) = split8(z + 8 * j, true);
-      }
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(a_ready + (kk & 1));
-      return true;
-    };
-    if (MODE == KM_KEY && te > tb) ok = convert(0);
-    int k = 0;
-    for (int t = tb; t < te; ++t, ++k) {
-      // a uniform stop decision for the four row warps
-      tc::named_sync(1, 128);
-      if (r == 0) *stop_s = *abort_s;
-      tc::named_sync(1, 128);
-      if (*stop_s) break;
+    for (int k = grp, t = tb + grp; t < te; k += 2, t += 2) {
       const int bh = head_of(t), tl = t - bh * a.ntile;
-      const int n0 = tl * LL_TILE, n = n0 + r;
+      const int n = tl * LL_TILE + r;
       const bool valid = n < a.N;
-      const int nvalid = min(LL_TILE, a.N - n0);
-      if (MODE == KM_KEY && t + 1 < te) ok = convert(k + 1) && ok;
+      if (bh != cur_bh) {  // this head's beta_g, in this warp's own copy
+        __syncwarp();
+        for (int g = lane; g < NC; g += 32) betas[g] = g < G ? a.beta[(size_t)bh * G + g] : 0.f;
+        __syncwarp();
+        cur_bh = bh;
+      }
       float f = 1.f;
       if (MODE == KM_QUERY) f = valid ? a.scale / a.rms[(size_t)bh * a.N + n] : 0.f;
-      if (bh != cur_bh) {  // this head's beta_g (every row warp is past the last argmax)
-        for (int g = r; g < NC; g += 128) betas[g] = g < G ? a.beta[(size_t)bh * G + g] : 0.f;
-        tc::named_sync(1, 128);
-      }
-      cur_bh = bh;
-      // ---- scores of tile k from TMEM, argmax (ties to the lowest index)
-      const int b = k & 1;
-      bool got = tc::mbar_wait(s_full + b, (k >> 1) & 1, abort_s, LL_WAIT_NS);
+      bool got = tc::mbar_wait(s_full + grp, (k >> 1) & 1, abort_s, LL_WAIT_NS);
       got = __all_sync(0xffffffffu, got);
-      int arg = 0;
-      if (got) {
-        tc::tc_fence_after();
-        float best[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
-        int bi[4] = {0, 0, 0, 0};
-        for (int c0 = 0; c0 < NC; c0 += 32) {
-          uint32_t v[32];
-          __syncwarp();
-          tc::tmem_ld32(tbase + lane_f + (uint32_t)(b * NCS + c0), v);
-          tc::tmem_wait_ld();
-          if (c0 + 32 <= G) {
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 be = *reinterpret_cast<const float4*>(betas + c0 + 4 * j4);
-              const float bq[4] = {be.x, be.y, be.z, be.w};
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int j = 4 * j4 + q;
-                const float sc = MODE == KM_QUERY ? fmaf(f, __uint_as_float(v[j]), -bq[q])
-                                                  : __uint_as_float(v[j]) - bq[q];
-                if (sc > best[q]) {
-                  best[q] = sc;
-                  bi[q] = c0 + j;
-                }
-              }
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int g = c0 + j;
-              if (g < G) {
-                const float sc = MODE == KM_QUERY ? fmaf(f, __uint_as_float(v[j]), -betas[g])
-                                                  : __uint_as_float(v[j]) - betas[g];
-                if (sc > best[j & 3]) {
-                  best[j & 3] = sc;
-                  bi[j & 3] = g;
-                }
-              }
-            }
-          }
-        }
-        float bb = best[0];
-        arg = bi[0];
-#pragma unroll
-        for (int q = 1; q < 4; ++q)
-          if (best[q] > bb || (best[q] == bb && bi[q] < arg)) {
-            bb = best[q];
-            arg = bi[q];
-          }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(s_free + b);
-      } else {
-        ok = false;
-      }
-      const int g = valid ? arg : -1;
-      if (valid && got) a.lab[(size_t)bh * a.N + n] = g;
-      rowf[r] = f;
-      // ---- stable sort of the tile's rows by label
-      cntw32[r] = 0u;
-      cntw32[r + 128] = 0u;
-      const unsigned mt = __match_any_sync(0xffffffffu, g);
-      const int rank = __popc(mt & lt_mask);
-      tc::named_sync(1, 128);
-      if (g >= 0 && (__ffs(mt) - 1) == lane) cntw[rw * 256 + g] = (uint8_t)__popc(mt);
-      tc::named_sync(1, 128);
-      int hcount[2];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {  // bins r and r + 128: counts over warps, prefix in place
-        const int bin = r + 128 * q;
-        const int c0 = cntw[bin], c1 = cntw[256 + bin], c2 = cntw[512 + bin], c3 = cntw[768 + bin];
-        cntw[bin] = 0;
-        cntw[256 + bin] = (uint8_t)c0;
-        cntw[512 + bin] = (uint8_t)(c0 + c1);
-        cntw[768 + bin] = (uint8_t)(c0 + c1 + c2);
-        hcount[q] = c0 + c1 + c2 + c3;
-      }
-      // exclusive scans over the 256 bins of (count, present) packed in one int
-      const int x0 = hcount[0] | ((hcount[0] > 0) << 16), x1 = hcount[1] | ((hcount[1] > 0) << 16);
-      const int i0 = warp_incl_scan(x0, lane), i1 = warp_incl_scan(x1, lane);
-      if (lane == 31) {
-        scanw[rw] = i0;
-        scanw[4 + rw] = i1;
-      }
-      tc::named_sync(1, 128);
-      int b0 = 0, b1 = 0, tot0 = 0;
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        tot0 += scanw[w];
-        if (w < rw) {
-          b0 += scanw[w];
-          b1 += scanw[4 + w];
-        }
-      }
-      const int e0 = b0 + i0 - x0, e1 = tot0 + b1 + i1 - x1;
-      lof[r] = e0 & 0xFFFF;
-      lidx[r] = e0 >> 16;
-      lof[r + 128] = e1 & 0xFFFF;
-      lidx[r + 128] = e1 >> 16;
-      // labels present: the tile's mask and the group-major tile bitmap
-      const unsigned m0 = __ballot_sync(0xffffffffu, hcount[0] > 0);
-      const unsigned m1 = __ballot_sync(0xffffffffu, hcount[1] > 0);
-      if (lane == 0) {
-        a.tmask[(size_t)t * 8 + rw] = m0;
-        a.tmask[(size_t)t * 8 + 4 + rw] = m1;
-      }
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int bin = r + 128 * q;
-        if (hcount[q] > 0 && bin < G)
-          atomicOr(a.gbits + ((size_t)bh * G + bin) * a.nword + (tl >> 5), 1u << (tl & 31));
-      }
-      tc::named_sync(1, 128);
-      if (g >= 0) {
-        const int pos = lof[g] + cntw[rw * 256 + g] + rank;
-        if (pos < 0 || pos >= nvalid)
-          set_error(a.hdr, ERR_INDEX, 9, bh, n);
-        else
-          srt[pos] = r | (g << 8);
-      }
-      tc::named_sync(1, 128);
-      {  // first run start in this warp's 32 sorted positions
-        const int p = 32 * rw + lane;
-        const int lp = p < nvalid ? srt[p] >> 8 : -1;
-        const int lq = (p > 0 && p - 1 < nvalid) ? srt[p - 1] >> 8 : -2;
-        const unsigned st = __ballot_sync(0xffffffffu, p < nvalid && lp != lq);
-        if (lane == 0) sbeg[rw] = st ? 32 * rw + __ffs(st) - 1 : -1;
-      }
-      tc::named_sync(1, 128);
-      // ---- run sums: this warp takes the runs that start in its positions
-      const int beg = sbeg[rw];
-      if (beg >= 0) {
-        int end = nvalid;
-        for (int w2 = rw + 1; w2 < 4; ++w2)
-          if (sbeg[w2] >= 0) {
-            end = sbeg[w2];
-            break;
-          }
-        const uint8_t* tile = stg + (uint32_t)(k % NS) * pl.stage_bytes;
-        float acc[VPL];
-#pragma unroll
-        for (int q = 0; q < VPL; ++q) acc[q] = 0.f;
-        int cur = -1, cnt = 0;
-        float* sbase = a.slots + (size_t)t * LL_SLOTS * W;
-        auto flush = [&]() {
-          if (cur < 0) return;
-          const int slot = lidx[cur];
-          float* dst = sbase + (size_t)slot * W + lane * VPL;
-          if (VPL == 4)
-            *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-          else if (VPL == 2)
-            *reinterpret_cast<float2*>(dst) = make_float2(acc[0], acc[1]);
-          else
-            dst[0] = acc[0];
-          if (lane == 0) a.slot_cnt[(size_t)t * LL_SLOTS + slot] = cnt;
-        };
-        for (int pb = beg; pb < end; pb += 32) {
-          const int e_l = pb + lane < end ? srt[pb + lane] : -1;
-          const int row_l = e_l & 255;
-          const int g_l = e_l >= 0 ? e_l >> 8 : -1;
-          const float f_l = e_l >= 0 ? rowf[row_l] : 0.f;
-          const int nu = min(32, end - pb);
-          for (int u = 0; u < nu; ++u) {
-            const int gu = __shfl_sync(0xffffffffu, g_l, u);
-            const int ru = __shfl_sync(0xffffffffu, row_l, u);
-            const float fu = __shfl_sync(0xffffffffu, f_l, u);
-            if (gu != cur) {
-              flush();
-#pragma unroll
-              for (int q = 0; q < VPL; ++q) acc[q] = 0.f;
-              cur = gu;
-              cnt = 0;
-            }
-            ++cnt;
-            if (MODE == KM_QUERY) {
-              if (DK == 128) {
-                const uint32_t off = (uint32_t)(lane >> 4) * LL_BOX + swz128(ru, (lane & 15) >> 1) +
-                                     ((lane & 1) << 3);
-                const uint2 x = *reinterpret_cast<const uint2*>(tile + off);
-                const float2 xa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.x));
-                const float2 xb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x.y));
-                acc[0] = fmaf(fu, xa.x, acc[0]);
-                acc[1] = fmaf(fu, xa.y, acc[1]);
-                acc[2] = fmaf(fu, xb.x, acc[2]);
-                acc[3] = fmaf(fu, xb.y, acc[3]);
-              } else {
-                const uint32_t off = swz128(ru, lane >> 2) + ((lane & 3) << 2);
-                const float2 xa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tile + off));
-                acc[0] = fmaf(fu, xa.x, acc[0]);
-                acc[1] = fmaf(fu, xa.y, acc[1]);
-              }
-            } else {
-              const uint32_t off = swz128(ru, lane >> 2) + ((lane & 3) << 2);
-              acc[0] += *reinterpret_cast<const float*>(tile + off);
-            }
-          }
-        }
-        flush();
-      }
-      // the tile's data stage is free again
+      if (!got) break;
+      tc::tc_fence_after();
+      const int arg = row_argmax<MODE>(tbase + lane_f + (uint32_t)(grp * NCS), NC, G, f, betas);
+      tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(d_empty + (k % NS));
-      tc::named_sync(1, 128);  // sort arrays and row factors are reused by the next tile
+      if (lane == 0) tc::mbar_arrive(s_free + grp);
+      if (valid) a.lab[(size_t)bh * a.N + n] = arg;
     }
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   if (tid == 0 && *abort_s) set_error(a.hdr, ERR_TIMEOUT, 9, blockIdx.x, 0);
-  if (warp == 1) {
+  if (warp == LL_MMA) {
     __syncwarp();
     tc::tmem_dealloc(tbase, pl.tcols);
   }
+}
+
+struct LuArgs {
+  int N, G, BH, ntile, nword;
+  float scale;
+  TensorView X;        // query mode rows
+  const float* Z;      // key mode: [BH][N][32] fp32 coordinates
+  const float* rms;    // query mode: row RMS
+  const int32_t* lab;  // [BH][N]
+  float* slots;        // [BH * ntile][LL_SLOTS][W]
+  int32_t* slot_cnt;   // [BH * ntile][LL_SLOTS]
+  uint32_t* tmask;     // [BH * ntile][8]
+  uint32_t* gbits;     // [BH][G][nword]
+  Header* hdr;
+};
+
+// Ascending bitonic sort of 128 distinct keys held by one warp, key[q] of
+// lane l at position 32 q + l.
+__device__ __forceinline__ void warp_sort128(int (&key)[4], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 128; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {  // partner in this lane, register q ^ (j / 32)
+        const int jq = j >> 5;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if ((q & jq) == 0) {
+            const int q2 = q | jq;
+            const bool asc = ((32 * q) & k) == 0;
+            const int lo = min(key[q], key[q2]), hi = max(key[q], key[q2]);
+            key[q] = asc ? lo : hi;
+            key[q2] = asc ? hi : lo;
+          }
+        }
+      } else {  // partner in lane ^ j, same register
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int o = __shfl_xor_sync(0xffffffffu, key[q], j);
+          const bool asc = ((32 * q + lane) & k) == 0;
+          const bool lower = (lane & j) == 0;
+          key[q] = (asc == lower) ? min(key[q], o) : max(key[q], o);
+        }
+      }
+    }
+  }
+}
+
+// Grid ceil(BH * ntile / LU_WARPS), LU_WARPS warps: warp w of block b takes
+// tile t = LU_WARPS b + w.
+template <int MODE, int DK>
+__global__ void __launch_bounds__(LU_WARPS * 32) k_lloyd_update(LuArgs a) {
+  constexpr int W = MODE == KM_QUERY ? DK : LL_KW;  // update-row width
+  constexpr int VPL = W / 32;                        // update values per lane
+  constexpr int INVALID = 0x7fffffff;
+  __shared__ float rowf_all[LU_WARPS][LL_TILE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * LU_WARPS + warp;
+  if (t >= a.BH * a.ntile) return;
+  float* rowf = rowf_all[warp];
+  const int bh = t / a.ntile, tl = t - bh * a.ntile;
+  const int n0 = tl * LL_TILE, nvalid = min(LL_TILE, a.N - n0);
+  // keys label << 7 | row; rows past N and out-of-range labels sort last
+  int key[4];
+  uint32_t mword = 0u;  // this lane's share of the label mask word `lane` (lanes 0-7)
+  uint32_t bits[8];
+#pragma unroll
+  for (int w = 0; w < 8; ++w) bits[w] = 0u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int rr = 32 * q + lane, n = n0 + rr;
+    key[q] = INVALID;
+    float f = 0.f;
+    if (rr < nvalid) {
+      const int g = a.lab[(size_t)bh * a.N + n];
+      if (g >= 0 && g < a.G) {
+        key[q] = (g << 7) | rr;
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+          if ((g >> 5) == w) bits[w] |= 1u << (g & 31);
+      } else {
+        set_error(a.hdr, ERR_INDEX, 9, bh, n);
+      }
+      if (MODE == KM_QUERY) f = a.scale / a.rms[(size_t)bh * a.N + n];
+    }
+    if (MODE == KM_QUERY) rowf[rr] = f;
+  }
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const uint32_t m = __reduce_or_sync(0xffffffffu, bits[w]);
+    if (lane == w) mword = m;
+  }
+  if (lane < 8) a.tmask[(size_t)t * 8 + lane] = mword;
+  // rows with a label in range (all of them, unless the error word is set)
+  int nkeys = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) nkeys += __popc(__ballot_sync(0xffffffffu, key[q] != INVALID));
+  warp_sort128(key, lane);
+  // run starts (a label differing from the previous position's)
+  uint32_t sb[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    int pk = __shfl_up_sync(0xffffffffu, key[q], 1);
+    const int carry = q > 0 ? __shfl_sync(0xffffffffu, key[q > 0 ? q - 1 : 0], 31) : -1;
+    if (lane == 0) pk = q > 0 ? carry : -1;
+    const bool st = key[q] != INVALID && (pk < 0 || (pk >> 7) != (key[q] >> 7));
+    sb[q] = __ballot_sync(0xffffffffu, st);
+  }
+  __syncwarp();  // row factors visible to the whole warp
+  float acc[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
+  int run = -1, run_start = 0, cur_g = -1;
+  float* sbase = a.slots + (size_t)t * LL_SLOTS * W + lane * VPL;
+  auto flush = [&](int count) {
+    float* dst = sbase + (size_t)run * W;
+    if (VPL == 4)
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    else if (VPL == 2)
+      *reinterpret_cast<float2*>(dst) = make_float2(acc[0], acc[1]);
+    else
+      dst[0] = acc[0];
+    if (lane == 0) {
+      a.slot_cnt[(size_t)t * LL_SLOTS + run] = count;
+      atomicOr(a.gbits + ((size_t)bh * a.G + cur_g) * a.nword + (tl >> 5), 1u << (tl & 31));
+    }
+  };
+  constexpr int UB = 8;  // rows loaded ahead of the in-order sums
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int base = 32 * q;
+    if (base >= nkeys) break;
+    const int cnt_q = min(32, nkeys - base);
+    for (int u0 = 0; u0 < cnt_q; u0 += UB) {
+      int kk[UB];
+      float x[UB][VPL];
+#pragma unroll
+      for (int e = 0; e < UB; ++e) {
+        kk[e] = __shfl_sync(0xffffffffu, key[q], (u0 + e) & 31);
+        const int rr = kk[e] & 127;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) x[e][v] = 0.f;
+        if (u0 + e < cnt_q) {
+          const int n = n0 + rr;
+          if constexpr (MODE == KM_QUERY && VPL == 4) {  // bf16 -> fp32 is a shift
+            const uint2 raw = *reinterpret_cast<const uint2*>(a.X.row(bh, n) + lane * 4);
+            x[e][0] = __uint_as_float(raw.x << 16);
+            x[e][1] = __uint_as_float(raw.x & 0xffff0000u);
+            x[e][2] = __uint_as_float(raw.y << 16);
+            x[e][3] = __uint_as_float(raw.y & 0xffff0000u);
+          } else if constexpr (MODE == KM_QUERY) {
+            const uint32_t raw = *reinterpret_cast<const uint32_t*>(a.X.row(bh, n) + lane * 2);
+            x[e][0] = __uint_as_float(raw << 16);
+            x[e][1] = __uint_as_float(raw & 0xffff0000u);
+          } else {
+            x[e][0] = a.Z[((size_t)bh * a.N + n) * LL_KW + lane];
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < UB; ++e) {
+        const int u = u0 + e;
+        if (u < cnt_q) {
+          const int p = base + u;
+          if ((sb[q] >> u) & 1u) {
+            if (run >= 0) flush(p - run_start);
+            ++run;
+            run_start = p;
+            cur_g = kk[e] >> 7;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
+          }
+          if (MODE == KM_QUERY) {
+            const float f = rowf[kk[e] & 127];
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) acc[v] = fmaf(f, x[e][v], acc[v]);
+          } else {
+            acc[0] += x[e][0];
+          }
+        }
+      }
+    }
+  }
+  if (run >= 0) flush(nkeys - run_start);
 }
 
 // Key operand of the next assignment from centroid c_g (32 coordinates, one
@@ -692,13 +671,19 @@ cudaError_t lloyd_launch(const CUtensorMap& tmX, const CUtensorMap& tmB, const L
                          cudaStream_t st) {
   const LlPlan pl = ll_plan<MODE, DK>(a.G);
   if (pl.NS < 2) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_lloyd<MODE, DK>,
+  cudaError_t e = cudaFuncSetAttribute(k_lloyd_assign<MODE, DK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.total);
   if (e != cudaSuccess) return e;
   const int T = a.BH * a.ntile;
   const int grid = T < num_sms() ? T : num_sms();
-  spr_launch(k_lloyd<MODE, DK>, grid, LL_THREADS, pl.total, st, tmX, tmB, a);
+  spr_launch(k_lloyd_assign<MODE, DK>, grid, LL_THREADS, pl.total, st, tmX, tmB, a);
   return cudaGetLastError();
+}
+
+template <int MODE, int DK>
+void update_launch(const LuArgs& u, cudaStream_t st) {
+  const int T = u.BH * u.ntile;
+  spr_launch(k_lloyd_update<MODE, DK>, (T + LU_WARPS - 1) / LU_WARPS, LU_WARPS * 32, 0, st, u);
 }
 
 }  // namespace
@@ -735,10 +720,12 @@ cudaError_t lloyd_step(const LloydStep& s, cudaStream_t st) {
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   } else {
-    const uint64_t dims[3] = {(uint64_t)LL_KW, (uint64_t)s.N, (uint64_t)s.BH};
-    const uint64_t str[2] = {(uint64_t)LL_KW * 4, (uint64_t)s.N * LL_KW * 4};
-    const uint32_t box[3] = {LL_KW, LL_TILE, 1};
-    if (!encode_tmap(&tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, s.Z, dims, str, box,
+    // bf16 rows z_hi | z_lo: [BH][N][64]
+    const uint64_t dims[3] = {64, (uint64_t)s.N, (uint64_t)s.BH};
+    const uint64_t str[2] = {128, (uint64_t)s.N * 128};
+    const uint32_t box[3] = {64, LL_TILE, 1};
+    if (s.Zhl == nullptr || s.Z == nullptr ||
+        !encode_tmap(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, s.Zhl, dims, str, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     const uint64_t bd[3] = {64, (uint64_t)NC, (uint64_t)(2 * s.BH)};
@@ -754,15 +741,10 @@ cudaError_t lloyd_step(const LloydStep& s, cudaStream_t st) {
   a.BH = s.BH;
   a.H = s.X.H > 0 ? s.X.H : 1;
   a.ntile = ntile;
-  a.nword = nword;
   a.scale = s.scale;
   a.rms = s.rms;
   a.beta = s.beta;
   a.lab = s.lab;
-  a.slots = s.slots;
-  a.slot_cnt = s.slot_cnt;
-  a.tmask = s.tmask;
-  a.gbits = s.gbits;
   a.hdr = s.hdr;
   cudaError_t e;
   if (s.mode == KM_QUERY)
@@ -771,6 +753,31 @@ cudaError_t lloyd_step(const LloydStep& s, cudaStream_t st) {
   else
     e = lloyd_launch<KM_KEY, LL_KW>(tmX, tmB, a, st);
   if (e != cudaSuccess) return e;
+  // per-tile sums of each label's rows
+  LuArgs u{};
+  u.N = s.N;
+  u.G = s.G;
+  u.BH = s.BH;
+  u.ntile = ntile;
+  u.nword = nword;
+  u.scale = s.scale;
+  u.X = s.X;
+  u.Z = s.Z;
+  u.rms = s.rms;
+  u.lab = s.lab;
+  u.slots = s.slots;
+  u.slot_cnt = s.slot_cnt;
+  u.tmask = s.tmask;
+  u.gbits = s.gbits;
+  u.hdr = s.hdr;
+  if (s.mode == KM_QUERY) {
+    if (s.d == 64)
+      update_launch<KM_QUERY, 64>(u, st);
+    else
+      update_launch<KM_QUERY, 128>(u, st);
+  } else {
+    update_launch<KM_KEY, LL_KW>(u, st);
+  }
   // the update
   const dim3 rg(s.G, s.BH);
   if (s.mode == KM_QUERY) {

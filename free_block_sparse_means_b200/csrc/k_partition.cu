@@ -699,7 +699,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   spr_launch(k_metric<D>, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, Q, N, p.Ms, P.MK);
   if ((e = launch_eig(P.MK, BH, D, p.p, P.eval, P.evec, P.trace, st)) != cudaSuccess) return e;
   spr_launch(k_keyweights, BH, 256, 0, st, P.eval, P.evec, P.trace, D, p.p, pp, P.W);
-  if ((e = launch_project(K, N, D, pp, BH, P.W, P.Z, P.hdr, st)) != cudaSuccess) return e;
+  if ((e = launch_project(K, N, D, pp, BH, P.W, P.Z, P.zhl, P.hdr, st)) != cudaSuccess) return e;
   spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
   if (p.init == SPR_INIT_WARM)  // the previous call's centroids, mapped (Craw still holds them)
     spr_launch(k_warm_centk, BH, 256, 0, st, P.Craw, P.W, p.Gk, D, pp, P.centk);
@@ -716,6 +716,7 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
     ks.G = p.Gk;
     ks.BH = BH;
     ks.Z = P.Z;
+    ks.Zhl = P.zhl;
     ks.bk = P.bk16;
     ks.beta = P.beta;
     ks.cent = P.centk;

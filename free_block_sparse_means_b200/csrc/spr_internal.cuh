@@ -35,7 +35,7 @@ enum Buf : int {
   B_QBAR, B_LOGIT, B_ENTRY, B_TOP, B_SEL, B_ROWPTR, B_COLIDX, B_RUNPTR, B_RUNS, B_PPOS,
   B_PIDX, B_PW, B_PSLOT, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
   B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_CSUM, B_XP, B_RP, B_PMEAN, B_CRAW64, B_QBAR64,
-  B_SLOTCNT, B_TMASK, B_GBITS, B_BK16, B_COUNT_
+  B_SLOTCNT, B_TMASK, B_GBITS, B_BK16, B_ZHL, B_COUNT_
 };
 
 struct Layout {
@@ -78,6 +78,7 @@ struct Ptrs {
       *qoff, *rowptr, *colidx, *runptr, *ppos, *pidx, *pslot, *slotcnt;
   uint32_t *tmask, *gbits;  // k-means update bookkeeping
   bf16* bk16;               // key k-means operand [BH][2][round32(Gk)][64]
+  bf16* zhl;                // key coordinates as bf16 hi | lo rows [BH][N][64]
   int2* runs;
   int4* items;
   uint8_t *sel, *top;
@@ -129,7 +130,8 @@ constexpr int LLOYD_SLOTS = 128;
 struct LloydStep {
   int mode, d, N, G, BH, split_rows;
   TensorView X;        // query mode: the rows ([B, H, N, d] view)
-  const float* Z;      // key mode: [BH][N][32] coordinates
+  const float* Z;      // key mode: [BH][N][32] coordinates (fp32, summed by the update)
+  const bf16* Zhl;     // key mode: [BH][N][64] the same rows as bf16 hi | lo (scored)
   const bf16* bq;      // query mode: [BH][2][split_rows][d] operand (hi, lo)
   bf16* bk;            // key mode: [BH][2][lloyd_ncrows(G)][64] operand (hi, lo)
   const float* rms;    // query mode: row RMS (factor scale / rms)
@@ -157,7 +159,7 @@ cudaError_t label_hist(const int32_t* lab, int N, int G, int nchunk, int BH, int
 
 // Key-response coordinates Z = K W (tensor cores); W is [BH][d][pp] fp32.
 cudaError_t launch_project(const TensorView& K, int N, int D, int PP, int BH, const float* W,
-                           float* Z, Header* hdr, cudaStream_t st);
+                           float* Z, bf16* Zhl, Header* hdr, cudaStream_t st);
 
 // Every kernel launch of the library goes through spr_launch, which counts it
 // (sparsepr_launch_count reports the total).
