@@ -188,7 +188,7 @@ def oracle_head_seconds(wl, bh, sample_rows=2048):
     from oracle import Params, hard_drop_attention, sparsepr_head
     prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
                  tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index,
-                 partition=wl.partition, weights=wl.weights)
+                 partition=wl.partition, weights=wl.weights, probe_select=wl.probes)
     Q, K, V = voronoi_qkv(wl, heads=[bh])
     q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
     if wl.N <= ORACLE_WHOLE_HEAD_MAX_N:
@@ -244,6 +244,7 @@ def config_of(wl, world):
                         else f"tau={wl.tau}"),
             "M": wl.M, "r": wl.r, "lambda": wl.lam, "partition": wl.partition,
             "probe_weights": wl.weights,
+            "probes": wl.probes,
             "parallelism": f"heads x{world} (weak)",
             "l2": "flushed (256 MiB write) before every timed call"}
 
@@ -425,14 +426,15 @@ def run_ours(args, wl):
     prm = spr.make_params(Q, K, V, O, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
                           seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
                           rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
-                          partition=wl.partition, weights=wl.weights)
+                          partition=wl.partition, weights=wl.weights, probes=wl.probes)
     ws = spr.alloc_workspace(prm, device=dev)
     prm_seeded = prm
     if args.warm_iters > 0:  # every call after the first starts from the previous centroids
         prm = spr.make_params(Q, K, V, O, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq,
                               iters=args.warm_iters, seed=wl.index, route_mode=wl.route_mode,
                               tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
-                              partition=wl.partition, weights=wl.weights, init="warm")
+                              partition=wl.partition, weights=wl.weights, probes=wl.probes,
+                              init="warm")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -499,20 +501,26 @@ def run_ours(args, wl):
             "executed_tile_pairs": tile_pairs, "true_pairs": pairs}
     part_bytes = partition_bytes(wl)
     part_gbs = part_bytes / (stage_max[0] * 1e-3) / 1e9
-    # end to end through the public API with host buffers (pinned)
+    # end to end through the public API with host buffers (pinned): the
+    # host-buffer call pipelined over chunks of heads (copies of one chunk
+    # overlap the computation of the next); every byte of the inputs and of
+    # the output crosses PCIe inside the timed region
     Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
     Oh = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    e2e_chunk = max(1, -(-wl.BH // E2E_CHUNKS))
+    pipe = spr.HostPipeline(shape, e2e_chunk, device=dev, Ms=wl.Ms, p=wl.p, Gk=wl.Gk,
+                            Gq=wl.Gq, iters=wl.iters, seed=wl.index, route_mode=wl.route_mode,
+                            tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
+                            partition=wl.partition, weights=wl.weights, probes=wl.probes)
     e2e_steps = max(3, min(args.steps, 10))
     ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(e2e_steps)]
+    flush.zero_()
+    pipe(Qh, Kh, Vh, Oh, stream)  # warm-up of the pipeline's own buffers
     for s in range(e2e_steps):
         flush.zero_()
         ee[s][0].record(stream)
-        Q.copy_(Qh, non_blocking=True)
-        K.copy_(Kh, non_blocking=True)
-        V.copy_(Vh, non_blocking=True)
-        spr.sparsepr_call(prm, Q, K, V, O, ws, stream)
-        Oh.copy_(O, non_blocking=True)
+        pipe(Qh, Kh, Vh, Oh, stream)
         ee[s][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = reduce_max([statistics.mean(a.elapsed_time(b) for a, b in ee)], world, dev)[0]
@@ -536,7 +544,10 @@ def run_ours(args, wl):
                               "frac": part_gbs / peaks["hbm_gbs"], "algorithmic_bytes": part_bytes},
             "e2e": {"value": dense_flop * world / (e2e_ms * 1e-3) / 1e12,
                     "unit": "TFLOP/s (dense-equivalent)", "ms_per_step": e2e_ms,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": f"HostPipeline: pinned host Q, K, V in and O out, "
+                           f"{len(pipe.chunks())} chunks of {e2e_chunk} heads, the copies "
+                           f"of one chunk overlapping the computation of the next"},
             "gpu_launches": int(n1 - n0), "clocks": clocks, "device_error": err}
     line["rel_l2_vs_dense"] = quality_vs_dense(spr, prm, ws, Q, K, V, O, wl)
     if args.diagnostics:
@@ -551,12 +562,87 @@ def run_ours(args, wl):
     return 0
 
 
+E2E_CHUNKS = 4  # head chunks of the pipelined host-buffer call
+SWEEP_RHO = (0.10, 0.20, 0.25, 0.35, 0.50)
+SWEEP_M = (64, 256, 1024)
+SWEEP_R = (8, 32)
+SWEEP_LAMBDA = (1e-2, 1e-1, 1.0)  # ridge strengths beside the workload's, at rho 0.25, r 8
+
+
+def run_sweep(args, wl):
+    """Density / probe-budget / rank sweep on one GPU (the sweep workload by
+    default): every executed-pair density in SWEEP_RHO with the method's
+    response-coupled partition for every probe budget M x rank r, and with
+    the semantic comparator at the workload's M and r; then, at rho 0.25 and
+    r 8, every M with the ridge strengths of SWEEP_LAMBDA.  One JSON line per
+    point: ms per call (median of the timed calls, L2 flushed before each),
+    dense-equivalent and executed-pair TFLOP/s, realised rho_exec and the
+    errors against dense attention on sampled rows (quality_vs_dense)."""
+    import free_block_sparse_means_b200 as spr
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    dev = torch.device("cuda", 0)
+    spr.load_library()
+    Qc, Kc, Vc = voronoi_qkv(wl)
+    shape = (wl.B, wl.H, wl.N, wl.d)
+    Q, K, V = (t.reshape(shape).contiguous().to(dev) for t in (Qc, Kc, Vc))
+    O = torch.empty_like(Q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    points = [("response", rho, M, r, wl.lam) for rho in SWEEP_RHO for M in SWEEP_M
+              for r in SWEEP_R]
+    points += [("semantic", rho, wl.M, wl.r, wl.lam) for rho in SWEEP_RHO]
+    points += [("response", 0.25, M, 8, lam) for M in SWEEP_M for lam in SWEEP_LAMBDA]
+    ws = None
+    for part, rho, M, r, lam in points:
+        pw = wl.replace(partition=part, route_mode="budget", rho_target=rho, M=M, r=r, lam=lam)
+        prm = spr.make_params(Q, K, V, O, Ms=pw.Ms, p=pw.p, Gk=pw.Gk, Gq=pw.Gq, iters=pw.iters,
+                              seed=pw.index, route_mode="budget", rho_target=rho, M=M, r=r,
+                              lam=lam, partition=part, weights=pw.weights, probes=pw.probes)
+        need = spr.sparsepr_workspace_size(prm)
+        if ws is None or ws.numel() < need:
+            ws = spr.alloc_workspace(prm, device=dev)
+        for _ in range(args.warmup):
+            flush.zero_()
+            spr.sparsepr_call(prm, Q, K, V, O, ws, stream)
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            spr.sparsepr_call(prm, Q, K, V, O, ws, stream)
+            b.record(stream)
+            times.append((a, b))
+        torch.cuda.synchronize(dev)
+        ms = statistics.median(x.elapsed_time(y) for x, y in times)
+        stats, err = spr.sparsepr_get_stats(prm, ws, stream)
+        if err:
+            raise SystemExit(f"device error word {err} at {part} rho={rho} M={M} r={r} "
+                             f"lambda={lam}")
+        pairs = sum(h["routed_pairs"] + h["probe_pairs"] for h in stats)
+        q = quality_vs_dense(spr, prm, ws, Q, K, V, O, pw, rows_per_head=512)
+        print(json.dumps({
+            "sweep": pw.name, "partition": part, "rho_target": rho, "M": M, "r": r,
+            "lambda": lam,
+            "rho_exec": pairs / (wl.N * wl.N * wl.BH), "ms_per_call_median": ms,
+            "dense_equiv_tflops": 4.0 * wl.d * wl.N * wl.N * wl.BH / (ms * 1e-3) / 1e12,
+            "exec_pair_tflops": 4.0 * wl.d * pairs / (ms * 1e-3) / 1e12,
+            "rel_l2_hard_drop": q["hard_drop"], "rel_l2_sparsepr": q["sparsepr"],
+            "row_error_hard_drop": q["row_error_hard_drop"],
+            "row_error_sparsepr": q["row_error_sparsepr"],
+            "o3_affine_fraction": q["o3_affine_fraction"]}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="hunyuan")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="H > 0: that many heads of the workload (a smaller case of the same "
+                         "kernels, for profiler captures)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
@@ -567,23 +653,35 @@ def main(argv=None):
                          "k-means from the previous call's centroids and runs T iterations")
     ap.add_argument("--weights", default="coverage", choices=["coverage", "uniform"],
                     help="uniform: the unweighted estimator of the ablation")
+    ap.add_argument("--probes", default="stratified", choices=["stratified", "ranked"],
+                    help="ranked: each group's probes are its rows nearest the centroid")
     ap.add_argument("--rank", type=int, default=0,
                     help="r of the residual fit (0: the workload's; d: no subspace restriction)")
     ap.add_argument("--diagnostics", action="store_true",
                     help="add the O1 pooled-support and O2 retained-mass diagnostics")
     ap.add_argument("--rho", type=float, default=0.0,
                     help="executed-pair density target (0: the workload's), for density sweeps")
+    ap.add_argument("--sweep", action="store_true",
+                    help="density x probe budget x rank sweep (one JSON line per point; "
+                         "default workload: sweep)")
     ap.add_argument("--partition", default="response", choices=["response", "semantic"],
                     help="semantic: the raw-row k-means comparator instead of the method's "
                          "response-coupled partition")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    wl = workload(args.workload, partition=args.partition, weights=args.weights)
+    wl = workload(args.workload, partition=args.partition, weights=args.weights,
+                  probes=args.probes)
+    if args.heads > 0:
+        wl = wl.replace(H=args.heads)
     if args.rank > 0:
         wl = wl.replace(r=args.rank)
     if args.rho > 0:
         wl = wl.replace(route_mode="budget", rho_target=args.rho)
+    if args.sweep:
+        if args.workload == "hunyuan":
+            wl = workload("sweep", weights=args.weights, probes=args.probes)
+        return run_sweep(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

@@ -11,9 +11,10 @@ from ._binding import (EXPORTS, LIB_PATH, PARTITION_RESPONSE, PARTITION_SEMANTIC
                        sparsepr_launch_count, sparsepr_partition, sparsepr_reconstruct,
                        sparsepr_route, sparsepr_version, sparsepr_workspace_size,
                        sparsepr_workspace_view, workspace_tensor)
+from .host_call import HostPipeline
 
 __all__ = [
-    "EXPORTS", "LIB_PATH", "PARTITION_RESPONSE", "PARTITION_SEMANTIC", "ROUTE_BUDGET", "ROUTE_TAU",
+    "EXPORTS", "HostPipeline", "LIB_PATH", "PARTITION_RESPONSE", "PARTITION_SEMANTIC", "ROUTE_BUDGET", "ROUTE_TAU",
     "VIEWS", "SparsePRError", "SprHeadStats", "SprParams", "alloc_workspace", "load_library",
     "make_params", "sparsepr_attend", "sparsepr_attend_routed_noalloc", "sparsepr_call",
     "sparsepr_check_params", "sparsepr_get_stats", "sparsepr_launch_count", "sparsepr_partition",

@@ -22,12 +22,13 @@ ROUTE_TAU, ROUTE_BUDGET = 0, 1
 PARTITION_RESPONSE, PARTITION_SEMANTIC = 0, 1
 INIT_SEEDED, INIT_WARM = 0, 1
 WEIGHTS_COVERAGE, WEIGHTS_UNIFORM = 0, 1
+PROBES_STRATIFIED, PROBES_RANKED = 0, 1
 
 VIEWS = {
     "lab_k": 0, "lab_q": 1, "perm_k": 2, "perm_q": 3, "kv_off": 4, "q_off": 5, "row_ptr": 6,
     "col_idx": 7, "probe_pos": 8, "probe_idx": 9, "probe_w": 10, "o_sparse": 11,
     "o_probe": 12, "w_key": 13, "cent_k": 14, "cent_q": 15, "ctilde": 16, "rms": 17,
-    "tail": 18, "fit_u": 19, "fit_b": 20, "fit_bvec": 21,
+    "tail": 18, "fit_u": 19, "fit_b": 20, "fit_bvec": 21, "probe_dist": 22,
 }
 
 
@@ -45,6 +46,7 @@ class SprParams(ctypes.Structure):
         ("M", ctypes.c_int32), ("r", ctypes.c_int32),
         ("lambda_", ctypes.c_double),
         ("partition", ctypes.c_int32), ("init", ctypes.c_int32), ("weights", ctypes.c_int32),
+        ("probes", ctypes.c_int32), ("head0", ctypes.c_int32),
     ]
 
 
@@ -128,7 +130,8 @@ def _strides(t: torch.Tensor):
 
 def make_params(Q, K=None, V=None, O=None, *, Ms, p, Gk, Gq, iters=10, seed=0, route_mode="tau",
                 tau=0.9, rho_target=0.25, M=64, r=8, lam=1e-3, scale=0.0,
-                partition="response", init="seeded", weights="coverage") -> SprParams:
+                partition="response", init="seeded", weights="coverage",
+                probes="stratified", head0=0) -> SprParams:
     """spr_params for tensors shaped [B, H, N, d] (strides taken from them)."""
     B, H, N, d = Q.shape
     prm = SprParams()
@@ -151,6 +154,10 @@ def make_params(Q, K=None, V=None, O=None, *, Ms, p, Gk, Gq, iters=10, seed=0, r
     if weights not in ("coverage", "uniform"):
         raise ValueError(f"weights must be 'coverage' or 'uniform', not {weights!r}")
     prm.weights = WEIGHTS_COVERAGE if weights == "coverage" else WEIGHTS_UNIFORM
+    if probes not in ("stratified", "ranked"):
+        raise ValueError(f"probes must be 'stratified' or 'ranked', not {probes!r}")
+    prm.probes = PROBES_STRATIFIED if probes == "stratified" else PROBES_RANKED
+    prm.head0 = int(head0)
     return prm
 
 

@@ -93,6 +93,8 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_GBITS] = BH * Gm * nword * 4;
   sz[B_BK16] = BH * 2 * (size_t)lloyd_ncrows((int)Gk) * 64 * 2;
   sz[B_ZHL] = BH * N * 64 * 2;
+  sz[B_PDIST] = BH * N * 4;  // written only with ranked probes
+  sz[B_FITW] = BH * d * d * 4;
   size_t off = 0;
   for (int i = 0; i < B_COUNT_; ++i) {
     L->off[i] = off;
@@ -181,6 +183,8 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.gbits = AT(uint32_t*, B_GBITS);
   P.bk16 = AT(bf16*, B_BK16);
   P.zhl = AT(bf16*, B_ZHL);
+  P.pdist = AT(float*, B_PDIST);
+  P.fitw = AT(float*, B_FITW);
 #undef AT
   return P;
 }
@@ -236,6 +240,10 @@ spr_status sparsepr_check_params(const spr_params* p) {
     return SPR_EINVAL;
   if (p->init != SPR_INIT_SEEDED && p->init != SPR_INIT_WARM) return SPR_EINVAL;
   if (p->weights != SPR_WEIGHTS_COVERAGE && p->weights != SPR_WEIGHTS_UNIFORM) return SPR_EINVAL;
+  if (p->probes != SPR_PROBES_STRATIFIED && p->probes != SPR_PROBES_RANKED) return SPR_EINVAL;
+  if (p->probes == SPR_PROBES_RANKED && p->partition != SPR_PARTITION_RESPONSE)
+    return SPR_EUNSUPPORTED;  // no query-response coordinates to rank in
+  if (p->head0 < 0 || p->head0 > (1 << 30)) return SPR_EINVAL;
   return SPR_OK;
 }
 
@@ -349,7 +357,7 @@ spr_status sparsepr_workspace_view(const spr_params* prm, int32_t which, size_t*
   static const int map[SPR_VIEW_COUNT] = {
       B_LABK, B_LABQ, B_PERMK, B_PERMQ, B_KVOFF, B_QOFF, B_ROWPTR, B_COLIDX, B_PPOS,
       B_PIDX, B_PW,   B_OSP,   B_ODN,   B_W,     B_CENTK, B_CENTQ, B_CT,    B_RMS,
-      B_ENTRY, B_FITU, B_FITB, B_FITBV};
+      B_ENTRY, B_FITU, B_FITB, B_FITBV, B_PDIST};
   if (which < 0 || which >= SPR_VIEW_COUNT) return SPR_EINVAL;
   if (offset) *offset = L.off[map[which]];
   if (bytes) *bytes = L.bytes[map[which]];

@@ -1,10 +1,10 @@
 // Routed attention under renormalized hard drop, fused with the exact dense
 // probe rows [paperlayer §1, §4 "Sparse Execution"; App. A.2].
 //
-// Work items come from the device-built list: a tile of up to 128 permuted
+// Work items come from the device-built list: up to ATT_ITEM (256) permuted
 // query rows of one query group plus the merged key ranges of the K/V groups
-// routed to that group, or a tile of up to 128 probe rows with the single key
-// range [0, N).  Each row's softmax is taken over exactly the keys of its
+// routed to that group, or up to 256 probe rows with the single key range
+// [0, N).  This kernel takes an item's rows 128 at a time.  Each row's softmax is taken over exactly the keys of its
 // ranges (renormalised hard drop); keys past a range end are masked.
 //
 // This file holds the mma.sync (m16n8k16 bf16) implementation: 8 warps x 16
@@ -52,7 +52,10 @@ __global__ void __launch_bounds__(256, 1) k_attend_mma(AttArgs a) {
     __syncthreads();
     if (idx_s >= n_items) break;
     const int4 it = item_s;
-    const int bh = it.x, q0 = it.y, nrows = it.z, grp = it.w;
+    const int bh = it.x, grp = it.w;
+    // an item holds up to ATT_ITEM rows: they are taken 128 at a time
+    for (int h0 = 0; h0 < it.z; h0 += ATT_BM) {
+    const int q0 = it.y + h0, nrows = min(ATT_BM, it.z - h0);
     const bf16* qsrc = grp >= 0 ? a.Qp + ((size_t)bh * a.N + q0) * D
                                 : a.qprobe + ((size_t)bh * a.M + q0) * D;
     int rbeg = 0, rend = 1;
@@ -223,6 +226,7 @@ __global__ void __launch_bounds__(256, 1) k_attend_mma(AttArgs a) {
       atomicAdd(reinterpret_cast<unsigned long long*>(&a.stats[bh].tile_pairs),
                 (unsigned long long)ntiles * BN * ATT_BM);
     __syncthreads();
+    }
   }
 }
 

@@ -595,7 +595,8 @@ template <int W>
 __global__ void __launch_bounds__(W) k_lloyd_reduce(const float* slots, const int32_t* slot_cnt,
                                                     const uint32_t* tmask, uint32_t* gbits, int G,
                                                     int ntile, int nword, float* cent, bf16* bk,
-                                                    float* beta, int ncrows) {
+                                                    float* beta, int ncrows, const float* A,
+                                                    bf16* bq, int split_rows) {
   __shared__ int list[32 * W];
   __shared__ int shs[32];
   const int g = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
@@ -624,14 +625,30 @@ __global__ void __launch_bounds__(W) k_lloyd_reduce(const float* slots, const in
       list[i] = tl * LL_SLOTS + rk;
     }
     __syncthreads();
+    // two interleaved fp64 chains (even entries into s0, odd into s1, added in
+    // order at the end), eight loads in flight ahead of the adds
     int i = 0;
-    for (; i + 1 < n; i += 2) {  // two interleaved fp64 chains, added in order at the end
+    for (; i + 8 <= n; i += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = sb[(size_t)list[i + u] * W + c];
+#pragma unroll
+      for (int u = 0; u < 8; u += 2) {
+        s0 += (double)v[u];
+        s1 += (double)v[u + 1];
+      }
+    }
+    for (; i + 1 < n; i += 2) {
       s0 += (double)sb[(size_t)list[i] * W + c];
       s1 += (double)sb[(size_t)list[i + 1] * W + c];
     }
     if (i < n) s0 += (double)sb[(size_t)list[i] * W + c];
-    for (int q = 0; q < n; ++q) cnt += cb[list[q]];
-    __syncthreads();
+    // rows: one count per listed tile, summed over the block
+    int cpart = 0;
+    for (int q = c; q < n; q += W) cpart += cb[list[q]];
+    int ctot;
+    block_exscan_small(cpart, shs, &ctot);
+    cnt += ctot;
   }
   float* cg = cent + ((size_t)bh * G + g) * W;
   float v = cg[c];
@@ -643,6 +660,29 @@ __global__ void __launch_bounds__(W) k_lloyd_reduce(const float* slots, const in
     bf16* hi = bk + (((size_t)bh * 2 + 0) * ncrows + g) * 64;
     bf16* lo = bk + (((size_t)bh * 2 + 1) * ncrows + g) * 64;
     key_operand_row(v, c, hi, lo, beta + (size_t)bh * G + g);
+  }
+  if (A != nullptr) {
+    // query mode: the next assignment's operand row Bq_g = A a_g (A symmetric,
+    // j ascending) split into bf16 hi + lo, and beta_g = a_g . Bq_g / 2
+    __shared__ float av[W];
+    __shared__ float red[W / 32];
+    av[c] = v;
+    __syncthreads();
+    const float* Ab = A + (size_t)bh * W * W;
+    float sv = 0.f;
+    for (int j = 0; j < W; ++j) sv += Ab[(size_t)j * W + c] * av[j];
+    const bf16 hi = __float2bfloat16_rn(sv);
+    const bf16 lo = __float2bfloat16_rn(sv - __bfloat162float(hi));
+    bq[(((size_t)bh * 2 + 0) * split_rows + g) * W + c] = hi;
+    bq[(((size_t)bh * 2 + 1) * split_rows + g) * W + c] = lo;
+    const float t = warp_sum(sv * v);
+    if ((c & 31) == 0) red[c >> 5] = t;
+    __syncthreads();
+    if (c == 0) {
+      float q = 0.f;
+      for (int w = 0; w < W / 32; ++w) q += red[w];
+      beta[(size_t)bh * G + g] = 0.5f * q;
+    }
   }
 }
 
@@ -785,16 +825,19 @@ cudaError_t lloyd_step(const LloydStep& s, cudaStream_t st) {
       spr_launch(k_lloyd_reduce<64>, rg, 64, 0, st, static_cast<const float*>(s.slots),
                  static_cast<const int32_t*>(s.slot_cnt), static_cast<const uint32_t*>(s.tmask),
                  s.gbits, s.G, ntile, nword, s.cent, static_cast<bf16*>(nullptr),
-                 static_cast<float*>(nullptr), 0);
+                 s.A ? const_cast<float*>(s.beta) : static_cast<float*>(nullptr), 0, s.A,
+                 s.A ? const_cast<bf16*>(s.bq) : static_cast<bf16*>(nullptr), s.split_rows);
     else
       spr_launch(k_lloyd_reduce<128>, rg, 128, 0, st, static_cast<const float*>(s.slots),
                  static_cast<const int32_t*>(s.slot_cnt), static_cast<const uint32_t*>(s.tmask),
                  s.gbits, s.G, ntile, nword, s.cent, static_cast<bf16*>(nullptr),
-                 static_cast<float*>(nullptr), 0);
+                 s.A ? const_cast<float*>(s.beta) : static_cast<float*>(nullptr), 0, s.A,
+                 s.A ? const_cast<bf16*>(s.bq) : static_cast<bf16*>(nullptr), s.split_rows);
   } else {
     spr_launch(k_lloyd_reduce<LL_KW>, rg, LL_KW, 0, st, static_cast<const float*>(s.slots),
                static_cast<const int32_t*>(s.slot_cnt), static_cast<const uint32_t*>(s.tmask),
-               s.gbits, s.G, ntile, nword, s.cent, s.bk, const_cast<float*>(s.beta), NC);
+               s.gbits, s.G, ntile, nword, s.cent, s.bk, const_cast<float*>(s.beta), NC,
+               static_cast<const float*>(nullptr), static_cast<bf16*>(nullptr), 0);
   }
   return cudaGetLastError();
 }

@@ -82,7 +82,7 @@ size_t na_bytes_needed(int64_t BH, int64_t N, int64_t Gq) {
 
 // One thread per (head, query group): check the group's offsets and every key
 // range the attention kernels will follow, and store the group's tile count
-// (ceil(rows / 128) when it has rows and at least one range, else 0).  A bad
+// (ceil(rows / ATT_ITEM) when it has rows and at least one range, else 0).  A bad
 // index stores 0 and sets the error word with info = {head, group, 0 query
 // offsets | 1 range pointers | 2 a key range}.  Block 0 first resets the
 // header's cursor and counts (the error word is reset by the host-side
@@ -113,14 +113,14 @@ __global__ void __launch_bounds__(256) k_na_check(const int32_t* qoff, const int
           ok = false;
         }
       }
-      if (ok && q1 > q0 && r1 > r0) c = (q1 - q0 + ATT_BM - 1) / ATT_BM;
+      if (ok && q1 > q0 && r1 > r0) c = (q1 - q0 + ATT_ITEM - 1) / ATT_ITEM;
     }
   }
   counts[e] = c;
 }
 
 // One block: unless the check above found a bad index, the exclusive scan of
-// the tile counts and the work list (query tiles of at most 128 rows of each
+// the item counts and the work list (items of at most ATT_ITEM rows of each
 // group, in head-major, group-major order).
 __global__ void __launch_bounds__(1024) k_na_plan(const int32_t* qoff, const int32_t* counts,
                                                   int BH, int Gq, int max_items, int4* items,
@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(1024) k_na_plan(const int32_t* qoff, const int
     const int bh = e / Gq, i = e - bh * Gq;
     const int s = qoff[(size_t)bh * (Gq + 1) + i], en = qoff[(size_t)bh * (Gq + 1) + i + 1];
     for (int t = 0; t < c; ++t) {
-      const int q0 = s + t * ATT_BM;
-      items[k++] = make_int4(bh, q0, min(ATT_BM, en - q0), i);
+      const int q0 = s + t * ATT_ITEM;
+      items[k++] = make_int4(bh, q0, min(ATT_ITEM, en - q0), i);
     }
   }
   if (tid == 0) hdr->n_items = total;

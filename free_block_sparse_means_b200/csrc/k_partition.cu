@@ -87,7 +87,7 @@ __global__ void k_keyweights(const float* evals, const float* evecs, const float
 // 0xD1B54A32D192ED03).  One block per (bh, which); a small open-addressing map
 // stores the displaced entries of the virtual identity array.
 // ---------------------------------------------------------------------------
-__global__ void k_init_idx(int N, int Gk, int Gq, uint64_t seed, int32_t* init_k,
+__global__ void k_init_idx(int N, int Gk, int Gq, uint64_t seed, int head0, int32_t* init_k,
                            int32_t* init_q) {
   constexpr int CAP = 2048;
   __shared__ int keys[CAP], vals[CAP];
@@ -112,7 +112,8 @@ __global__ void k_init_idx(int N, int Gk, int Gq, uint64_t seed, int32_t* init_k
     keys[s] = k;
     vals[s] = v;
   };
-  uint64_t x = seed ^ ((uint64_t)(2 * bh + which + 1) * 0xD1B54A32D192ED03ull);
+  // the stream of head head0 + bh (heads of one call are numbered from head0)
+  uint64_t x = seed ^ ((uint64_t)(2 * ((int64_t)head0 + bh) + which + 1) * 0xD1B54A32D192ED03ull);
   for (int i = 0; i < G; ++i) {
     x += 0x9E3779B97F4A7C15ull;
     uint64_t z = x;
@@ -156,17 +157,31 @@ __global__ void k_warm_centk(const float* Craw, const float* W, int G, int D, in
 // Per (bh, g): base of each chunk within the group (exclusive scan over
 // chunks), group sizes, and group offsets (exclusive scan over g).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_chunk_scan(const int32_t* chunk_cnt, int nchunk, int G,
-                                                    int N, int32_t* cbase, int32_t* off,
-                                                    int32_t* counts) {
+__global__ void __launch_bounds__(256) k_chunk_scan(const int32_t* __restrict__ chunk_cnt,
+                                                    int nchunk, int G, int N,
+                                                    int32_t* __restrict__ cbase,
+                                                    int32_t* __restrict__ off,
+                                                    int32_t* __restrict__ counts) {
   __shared__ int wsum[8];
   const int bh = blockIdx.x, g = threadIdx.x;
   int tot = 0;
   if (g < G) {
-    for (int c = 0; c < nchunk; ++c) {
-      const size_t i = ((size_t)bh * nchunk + c) * G + g;
-      cbase[i] = tot;
-      tot += chunk_cnt[i];
+    const int32_t* src = chunk_cnt + (size_t)bh * nchunk * G + g;
+    int32_t* dst = cbase + (size_t)bh * nchunk * G + g;
+    int c = 0;
+    for (; c + 8 <= nchunk; c += 8) {  // eight loads in flight ahead of the running sum
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = src[(size_t)(c + u) * G];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        dst[(size_t)(c + u) * G] = tot;
+        tot += v[u];
+      }
+    }
+    for (; c < nchunk; ++c) {
+      dst[(size_t)c * G] = tot;
+      tot += src[(size_t)c * G];
     }
     counts[(size_t)bh * G + g] = tot;
   }
@@ -289,19 +304,16 @@ __global__ void k_gmean_fin(const double* part, const int32_t* off, int G, float
 template <int PP>
 __global__ void __launch_bounds__(256) k_obj_z(const float* Z, int N, int G, const float* cent,
                                                const int32_t* lab, int nchunk, double* part) {
+  static_assert(PP == 32, "one lane per coordinate");
   __shared__ double red[8];
-  const int bh = blockIdx.y, chunk = blockIdx.x;
+  const int bh = blockIdx.y, chunk = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // warp w takes rows w, w + 8, ... of the chunk (128-byte coalesced rows);
+  // each lane sums its coordinate's squared differences, then the warp adds
   double acc = 0.0;
-  for (int n = chunk * CHUNK + threadIdx.x; n < min(N, (chunk + 1) * CHUNK); n += 256) {
+  for (int n = chunk * CHUNK + warp; n < min(N, (chunk + 1) * CHUNK); n += 8) {
     const int g = lab[(size_t)bh * N + n];
-    const float* z = Z + ((size_t)bh * N + n) * PP;
-    const float* c = cent + ((size_t)bh * G + g) * PP;
-    float s = 0.f;
-    for (int k = 0; k < PP; ++k) {
-      const float t = z[k] - c[k];
-      s += t * t;
-    }
-    acc += s;
+    const float t = Z[((size_t)bh * N + n) * PP + lane] - cent[((size_t)bh * G + g) * PP + lane];
+    acc += (double)(t * t);
   }
   acc = warp_sum(acc);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
@@ -524,8 +536,8 @@ __global__ void __launch_bounds__(256) k_query_rms(RmsArgs a) {
 // Initial query centroids: a_g = (s / rms_n) q_n at the seeded rows.
 __global__ void k_init_centq(TensorView Q, int N, int G, int D, const int32_t* init,
                              const float* rms, float scale, float* centq) {
-  const int bh = blockIdx.x;
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+  const int bh = blockIdx.x;  // grid (BH, y): blocks of a head share its rows
+  for (int e = blockIdx.y * blockDim.x + threadIdx.x; e < G * D; e += blockDim.x * gridDim.y) {
     const int g = e / D, c = e % D;
     const int n = init[(size_t)bh * G + g];
     centq[(size_t)bh * G * D + e] = scale / rms[(size_t)bh * N + n] * bf2f(Q.row(bh, n)[c]);
@@ -617,11 +629,12 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
   const int ggrid = num_sms() * 8;
   cudaError_t e;
   spr_launch(k_semantic_setup, dim3(64, BH), 256, 0, st, P.Amat, P.rms, D, N, scale);
-  spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
+  spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, p.head0, P.initk,
+             P.initq);
   auto lloyd = [&](const TensorView& X, int G, const int32_t* init, float* cent,
                    int32_t* lab) -> cudaError_t {
     if (p.init != SPR_INIT_WARM)  // warm: cent holds the previous call's raw-row centroids
-      spr_launch(k_init_centq, BH, 256, 0, st, X, N, G, D, init, P.rms, scale, cent);
+      spr_launch(k_init_centq, dim3(BH, 32), 256, 0, st, X, N, G, D, init, P.rms, scale, cent);
     if (cudaMemsetAsync(P.gbits, 0, L.bytes[B_GBITS], st) != cudaSuccess) return cudaGetLastError();
     LloydStep ls{};
     ls.mode = KM_QUERY;
@@ -646,9 +659,10 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
     ls.slot_cnt_bytes = L.bytes[B_SLOTCNT];
     ls.tmask_bytes = L.bytes[B_TMASK];
     ls.gbits_bytes = L.bytes[B_GBITS];
+    ls.A = P.Amat;  // each update also prepares the next iteration's operand
+    spr_launch(k_qprep, dim3(BH, G), D, 0, st, P.Amat, cent, G, D, P.counts, P.beta, P.bq16,
+               split_rows, nullptr);
     for (int it = 0; it < p.iters; ++it) {
-      spr_launch(k_qprep, dim3(BH, G), D, 0, st, P.Amat, cent, G, D, P.counts, P.beta, P.bq16,
-                 split_rows, nullptr);
       const cudaError_t e2 = lloyd_step(ls, st);
       if (e2 != cudaSuccess) return e2;
     }
@@ -700,7 +714,8 @@ static cudaError_t partition_d(const spr_params& p, const Layout& L, const Ptrs&
   if ((e = launch_eig(P.MK, BH, D, p.p, P.eval, P.evec, P.trace, st)) != cudaSuccess) return e;
   spr_launch(k_keyweights, BH, 256, 0, st, P.eval, P.evec, P.trace, D, p.p, pp, P.W);
   if ((e = launch_project(K, N, D, pp, BH, P.W, P.Z, P.zhl, P.hdr, st)) != cudaSuccess) return e;
-  spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, P.initk, P.initq);
+  spr_launch(k_init_idx, dim3(BH, 2), 128, 0, st, N, p.Gk, p.Gq, p.seed, p.head0, P.initk,
+             P.initq);
   if (p.init == SPR_INIT_WARM)  // the previous call's centroids, mapped (Craw still holds them)
     spr_launch(k_warm_centk, BH, 256, 0, st, P.Craw, P.W, p.Gk, D, pp, P.centk);
   else
@@ -763,14 +778,20 @@ spr_launch(k_obj_z<32>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.l
   ra.rms = P.rms;
   ra.un2 = P.un2;
   ra.part = P.part;
-  {
+  if (D == 128) {  // tcgen05; its per-tile sums use the k-means partial-sum area (idle here)
+    if ((e = launch_rms_tc(Q, p.B, p.H, N, nchunk, split_rows, P.bq16, scale, P.stats, P.rms,
+                           P.un2, reinterpret_cast<double*>(P.csum), P.part, P.hdr, st)) !=
+        cudaSuccess)
+      return e;
+  } else {
     const size_t sm = (size_t)2 * D * D * 2 + ATT_BM * D * 2 + 64;
     cudaFuncSetAttribute(k_query_rms<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     spr_launch(k_query_rms<D>, dim3(nchunk, BH), 256, sm, st, ra);
   }
   // Query k-means in the head dimension
   if (p.init != SPR_INIT_WARM)  // warm: centq keeps the previous call's head-dim centroids
-    spr_launch(k_init_centq, BH, 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale, P.centq);
+    spr_launch(k_init_centq, dim3(BH, 32), 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale,
+               P.centq);
   if (cudaMemsetAsync(P.gbits, 0, L.bytes[B_GBITS], st) != cudaSuccess) return cudaGetLastError();
   {
     LloydStep qs{};
@@ -796,11 +817,11 @@ spr_launch(k_obj_z<32>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.l
     qs.slot_cnt_bytes = L.bytes[B_SLOTCNT];
     qs.tmask_bytes = L.bytes[B_TMASK];
     qs.gbits_bytes = L.bytes[B_GBITS];
-    for (int it = 0; it < p.iters; ++it) {
-      spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta,
-                 P.bq16, split_rows, nullptr);
+    qs.A = P.Amat;  // each update also prepares the next iteration's operand
+    spr_launch(k_qprep, dim3(BH, p.Gq), D, 0, st, P.Amat, P.centq, p.Gq, D, P.counts, P.beta,
+               P.bq16, split_rows, nullptr);
+    for (int it = 0; it < p.iters; ++it)
       if ((e = lloyd_step(qs, st)) != cudaSuccess) return e;
-    }
   }
   if ((e = label_hist(P.labq, N, p.Gq, nchunk, BH, P.chunk, P.hdr, st)) != cudaSuccess) return e;
   // group-major query order of the final labels

@@ -510,6 +510,13 @@ static cudaError_t reconstruct_d(const spr_params& p, const Layout& L, const Ptr
   } else {
     spr_launch(k_fit_zero, num_sms(), 256, 0, st, P.fitB, P.fitBv, D, BH);
   }
+  if (D == 128) {  // the tensor-core application
+    cudaError_t e = launch_apply_tc(p, L, P, O, R, st);
+    if (e != cudaSuccess) return e;
+    spr_launch(k_stats, (BH + 127) / 128, 128, 0, st, P.stats, P.part,
+               P.part + (size_t)BH * 2 * (L.nchunk + 1), L.nchunk, p.Gq, N, M, BH);
+    return cudaGetLastError();
+  }
   const int RA = (R + 1) & ~1;
   const size_t sm = (size_t)(2 * D * RA + D * APPLY_XT + 4 * RA * APPLY_XT) * 4;
   cudaFuncSetAttribute(k_apply<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

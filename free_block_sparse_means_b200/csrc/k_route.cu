@@ -180,39 +180,23 @@ __global__ void __launch_bounds__(1024) k_route_budget(const double* tail, const
   const int ncell = Gq * Gk;
   const double* R = tail + (size_t)bh * ncell;
   auto bits = [](double r) -> long long { return r < 0.0 ? -1ll : __double_as_longlong(r); };
-  // the first RB_CACHE cells of every thread stay in registers (bit pattern,
-  // pair count) for the whole search; more cells are read again each round
-  constexpr int RB_CACHE = 8;
-  long long cb[RB_CACHE];
-  long long cw[RB_CACHE];
-  long long tmin = 0x7FF0000000000000ll, tmax = -1;
-#pragma unroll
-  for (int q = 0; q < RB_CACHE; ++q) {
-    const int t = tid + q * 1024;
-    cb[q] = -1;
-    cw[q] = 0;
-    if (t < ncell) {
-      const int i = t / Gk, j = t - i * Gk;
-      if (nqs[i] > 0 && nks[j] > 0) {
-        cb[q] = bits(R[t]);
-        cw[q] = (long long)nqs[i] * nks[j];
-      }
-    }
-  }
-  auto cost = [&](long long T) {
+  auto live_cell = [&](int t) {
+    const int i = t / Gk, j = t - i * Gk;
+    return nqs[i] > 0 && nks[j] > 0;
+  };
+  auto weight = [&](int t) -> long long {
+    const int i = t / Gk, j = t - i * Gk;
+    return (long long)nqs[i] * nks[j];
+  };
+  auto cost = [&](long long T) {  // pairs of the live cells at or above pattern T
     long long c = 0;
-#pragma unroll
-    for (int q = 0; q < RB_CACHE; ++q) c += cb[q] >= T ? cw[q] : 0ll;
-    for (int t = tid + RB_CACHE * 1024; t < ncell; t += 1024) {
-      const int i = t / Gk, j = t - i * Gk;
-      if (nqs[i] > 0 && nks[j] > 0 && bits(R[t]) >= T) c += (long long)nqs[i] * nks[j];
-    }
+    for (int t = tid; t < ncell; t += 1024)
+      if (live_cell(t) && bits(R[t]) >= T) c += weight(t);
     return block_reduce(c, shl, [](long long a, long long b) { return a + b; });
   };
-  // the search runs between the smallest and largest live tail patterns
+  long long tmin = 0x7FF0000000000000ll, tmax = -1;
   for (int t = tid; t < ncell; t += 1024) {
-    const int i = t / Gk, j = t - i * Gk;
-    if (nqs[i] > 0 && nks[j] > 0) {
+    if (live_cell(t)) {
       const long long b = bits(R[t]);
       tmin = b < tmin ? b : tmin;
       tmax = b > tmax ? b : tmax;
@@ -220,20 +204,125 @@ __global__ void __launch_bounds__(1024) k_route_budget(const double* tail, const
   }
   tmin = block_reduce(tmin, shl, [](long long a, long long b) { return a < b ? a : b; });
   tmax = block_reduce(tmax, shl, [](long long a, long long b) { return a > b ? a : b; });
-  // cost(T) is non-increasing in T; cost(tmax + 1) = 0.
-  long long Tstar;
-  if (tmax < 0 || (double)cost(tmin) <= budget) {
-    Tstar = tmax < 0 ? 0 : tmin;
-  } else {
-    long long lo = tmin, hi = tmax + 1;  // cost(lo) > budget >= cost(hi)
-    while (hi - lo > 1) {
-      const long long mid = lo + (hi - lo) / 2;
-      if ((double)cost(mid) <= budget)
-        hi = mid;
-      else
-        lo = mid;
+  // cost(T) is non-increasing in T.  T* = B* + 1 with B* the largest live
+  // pattern whose cost exceeds the budget; T* = tmin when every live cell fits.
+  // B* is located with 1024 sample patterns (every (ncell / 1024)-th cell,
+  // sorted): each live cell's pairs go to the bin of samples around its
+  // pattern, suffix sums over the bins give the bin holding B*, and B* is
+  // found exactly among that bin's cells (or, past RB_LIST of them, by
+  // bisection over the bin's pattern range).
+  constexpr int RB_LIST = 1536;
+  __shared__ long long samp[1024];
+  __shared__ unsigned long long binw[1025];
+  __shared__ long long lb[RB_LIST];
+  __shared__ long long lw[RB_LIST];
+  __shared__ int nl_s;
+  {
+    const int t = (int)(((long long)tid * ncell) / 1024);
+    samp[tid] = (t < ncell && live_cell(t)) ? bits(R[t]) : -1;
+  }
+  binw[tid] = 0ull;
+  if (tid == 0) {
+    binw[1024] = 0ull;
+    nl_s = 0;
+  }
+  __syncthreads();
+  for (int k = 2; k <= 1024; k <<= 1) {  // bitonic sort of the samples, ascending
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const int ixj = tid ^ j;
+      if (ixj > tid) {
+        const long long a = samp[tid], b = samp[ixj];
+        if ((a > b) == ((tid & k) == 0)) {
+          samp[tid] = b;
+          samp[ixj] = a;
+        }
+      }
+      __syncthreads();
     }
-    Tstar = hi;
+  }
+  auto bin_of = [&](long long b) {  // samples <= b: 0 .. 1024
+    int lo = 0, hi = 1024;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (samp[mid] <= b) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
+  for (int t = tid; t < ncell; t += 1024)
+    if (live_cell(t)) atomicAdd(&binw[bin_of(bits(R[t]))], (unsigned long long)weight(t));
+  __syncthreads();
+  // suffix sums S(k) = sum of bins k .. 1024 (non-increasing in k): thread
+  // tid holds S(1023 - tid) from a prefix scan over the bins in reverse order
+  const long long s_top = (long long)binw[1024];
+  long long mine;
+  {
+    const int lane = tid & 31, w = tid >> 5;
+    long long inc = (long long)binw[1023 - tid];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long u = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += u;
+    }
+    if (lane == 31) shl[w] = inc;
+    __syncthreads();
+    long long before = 0;
+    for (int i = 0; i < w; ++i) before += shl[i];
+    __syncthreads();
+    mine = before + inc + s_top;
+  }
+  // k* = the largest bin with S(k*) > budget: bins 0 .. k* are exactly those
+  const int above = (int)block_reduce((long long)((double)mine > budget ? 1 : 0), shl,
+                                      [](long long a, long long b) { return a + b; });
+  const bool top_over = (double)s_top > budget;
+  long long Tstar;
+  if (tmax < 0) {
+    Tstar = 0;
+  } else if (above == 0 && !top_over) {
+    Tstar = tmin;  // every live cell fits
+  } else {
+    const int kst = top_over ? 1024 : above - 1;
+    // the cost of the cells in the bins above k*: S(k* + 1)
+    long long part = 0;
+    for (int k = kst + 1 + tid; k <= 1024; k += 1024) part += (long long)binw[k];
+    const long long c_above = block_reduce(part, shl, [](long long a, long long b) { return a + b; });
+    for (int t = tid; t < ncell; t += 1024) {
+      if (live_cell(t)) {
+        const long long b = bits(R[t]);
+        if (bin_of(b) == kst) {
+          const int at = atomicAdd(&nl_s, 1);
+          if (at < RB_LIST) {
+            lb[at] = b;
+            lw[at] = weight(t);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    const int nl = nl_s;
+    long long bstar = -1;
+    if (nl <= RB_LIST) {
+      // cost(b) for each listed pattern: the cells above the bin plus the
+      // listed cells at or above b; B* = the largest with cost > budget
+      for (int e = tid; e < nl; e += 1024) {
+        long long c = c_above;
+        for (int f = 0; f < nl; ++f) c += lb[f] >= lb[e] ? lw[f] : 0ll;
+        if ((double)c > budget && lb[e] > bstar) bstar = lb[e];
+      }
+      bstar = block_reduce(bstar, shl, [](long long a, long long b) { return a > b ? a : b; });
+    } else {
+      // bisection over the bin's pattern range [lo, hi): cost(lo) > budget >= cost(hi)
+      long long lo = kst > 0 ? samp[kst - 1] : tmin, hi = kst < 1024 ? samp[kst] : tmax + 1;
+      if (lo < tmin) lo = tmin;
+      while (hi - lo > 1) {
+        const long long mid = lo + (hi - lo) / 2;
+        if ((double)cost(mid) <= budget)
+          hi = mid;
+        else
+          lo = mid;
+      }
+      bstar = hi - 1;
+    }
+    Tstar = bstar + 1;
   }
   double kept_min = INFINITY;
   int only_top = 1;
@@ -380,9 +469,134 @@ __global__ void __launch_bounds__(256) k_probes(const int32_t* qoff, const int32
   }
 }
 
-// Attention work list: probe tiles of every head first (they span all keys),
-// then the query tiles of every (head, query group) with routed cells.
-// Items: {bh, q0, nrows, grp} with grp = -1 for a probe tile (q0 = probe slot).
+// Distance-ranked probes (reading R16): the squared distance of permuted query
+// pos (original row n) to its group's centroid in query-response coordinates,
+//   ||u_n - c_g||^2 = ||u_n||^2 - 2 (f_n q_n . Bq_g - beta_g),
+// with f_n = scale / rms_n, Bq_g = A a_g (bf16 hi + lo rows) and beta_g =
+// ||c_g||^2 / 2 from the final query centroids a_g, ||u_n||^2 from the RMS
+// pass.  One warp per permuted row: lane l holds D / 32 coordinates.
+template <int D>
+__global__ void __launch_bounds__(256) k_probe_dist(const bf16* Qp, const int32_t* permq,
+                                                    const int32_t* labq, const float* rms,
+                                                    const float* un2, const bf16* bq,
+                                                    const float* beta, int N, int G,
+                                                    int split_rows, float scale, int BH,
+                                                    float* dist) {
+  constexpr int V = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (w >= (long long)BH * N) return;
+  const int bh = (int)(w / N), pos = (int)(w - (long long)bh * N);
+  const int n = permq[(size_t)bh * N + pos];
+  const int g = labq[(size_t)bh * N + n];
+  const bf16* q = Qp + ((size_t)bh * N + pos) * D + lane * V;
+  const bf16* bh_row = bq + (((size_t)bh * 2 + 0) * split_rows + g) * D + lane * V;
+  const bf16* bl_row = bq + (((size_t)bh * 2 + 1) * split_rows + g) * D + lane * V;
+  float acc = 0.f;
+#pragma unroll
+  for (int v = 0; v < V; ++v)
+    acc = fmaf(__bfloat162float(q[v]),
+               __bfloat162float(bh_row[v]) + __bfloat162float(bl_row[v]), acc);
+  acc = warp_sum(acc);
+  if (lane == 0) {
+    const float f = scale / rms[(size_t)bh * N + n];
+    const float score = fmaf(f, acc, -beta[(size_t)bh * G + g]);
+    dist[(size_t)bh * N + pos] = fmaf(-2.f, score, un2[(size_t)bh * N + n]);
+  }
+}
+
+// Orderable 64-bit key of (distance, original row): smaller distance first,
+// ties to the lower row; NaN sorts last.
+__device__ __forceinline__ unsigned long long dist_key(float d, int row) {
+  uint32_t b = __float_as_uint(d);
+  if (d != d) b = 0xffffffffu;
+  else b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return ((unsigned long long)b << 32) | (uint32_t)row;
+}
+
+// Replace each query group's stratified probe rows by its m_g rows nearest
+// the centroid (reading R16; counts and weights unchanged).  Grid (Gq, BH),
+// 256 threads.  The group's slots are the entries of the ascending probe
+// list inside its position range; the m_g smallest keys are found one at a
+// time (the k-th smallest is the smallest key above the (k-1)-th), then
+// written in ascending position order.
+__global__ void __launch_bounds__(256) k_probes_ranked(const int32_t* qoff, const int32_t* permq,
+                                                       const float* dist, int Gq, int N, int M,
+                                                       int32_t* ppos, int32_t* pidx,
+                                                       int32_t* pslot) {
+  __shared__ int sel[MAX_PROBES];
+  __shared__ unsigned long long shk[8];
+  __shared__ int shp[8];
+  const int g = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+  const int q0 = qoff[(size_t)bh * (Gq + 1) + g], q1 = qoff[(size_t)bh * (Gq + 1) + g + 1];
+  if (q1 <= q0 || M == 0) return;
+  int32_t* pp = ppos + (size_t)bh * M;
+  auto lower = [&](int x) {  // first probe slot whose position is >= x
+    int lo = 0, hi = M;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (pp[mid] < x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
+  const int base = lower(q0), m = lower(q1) - base;
+  if (m <= 0) return;
+  // the stratified rows lose their slots
+  for (int t = tid; t < m; t += 256) pslot[(size_t)bh * N + pp[base + t]] = -1;
+  const float* dg = dist + (size_t)bh * N;
+  const int32_t* pq = permq + (size_t)bh * N;
+  unsigned long long last = 0ull;
+  for (int k = 0; k < m; ++k) {
+    unsigned long long best = ~0ull;
+    int bpos = -1;
+    for (int pos = q0 + tid; pos < q1; pos += 256) {
+      const unsigned long long key = dist_key(dg[pos], pq[pos]);
+      if ((k == 0 || key > last) && key < best) {
+        best = key;
+        bpos = pos;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long ok = __shfl_xor_sync(0xffffffffu, best, o);
+      const int op = __shfl_xor_sync(0xffffffffu, bpos, o);
+      if (ok < best) {
+        best = ok;
+        bpos = op;
+      }
+    }
+    if ((tid & 31) == 0) {
+      shk[tid >> 5] = best;
+      shp[tid >> 5] = bpos;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int i = 1; i < 8; ++i)
+        if (shk[i] < shk[0]) {
+          shk[0] = shk[i];
+          shp[0] = shp[i];
+        }
+      sel[k] = shp[0];
+    }
+    __syncthreads();
+    last = shk[0];
+    __syncthreads();
+  }
+  // ascending positions: each chosen position's rank among the chosen
+  for (int t = tid; t < m; t += 256) {
+    const int pos = sel[t];
+    int rank = 0;
+    for (int u = 0; u < m; ++u) rank += sel[u] < pos;
+    pp[base + rank] = pos;
+    pidx[(size_t)bh * M + base + rank] = pq[pos];
+    pslot[(size_t)bh * N + pos] = base + rank;
+  }
+}
+
+// Attention work list: probe items of every head first (they span all keys),
+// then the query items of every (head, query group) with routed cells; an
+// item holds up to ATT_ITEM rows.
+// Items: {bh, q0, nrows, grp} with grp = -1 for probe rows (q0 = probe slot).
 __global__ void __launch_bounds__(1024) k_worklist(const int32_t* qoff, const int32_t* rowptr,
                                                    int BH, int Gq, int M, int max_items,
                                                    int4* items, Header* hdr) {
@@ -392,11 +606,11 @@ __global__ void __launch_bounds__(1024) k_worklist(const int32_t* qoff, const in
   const int per = (nent + 1023) / 1024;
   const int e0 = tid * per, e1 = min(nent, e0 + per);
   auto count = [&](int e) -> int {
-    if (e < BH) return (M + ATT_BM - 1) / ATT_BM;
+    if (e < BH) return (M + ATT_ITEM - 1) / ATT_ITEM;
     const int bh = (e - BH) / Gq, i = (e - BH) % Gq;
     const int nq = qoff[(size_t)bh * (Gq + 1) + i + 1] - qoff[(size_t)bh * (Gq + 1) + i];
     const int nc = rowptr[(size_t)bh * (Gq + 1) + i + 1] - rowptr[(size_t)bh * (Gq + 1) + i];
-    return (nq > 0 && nc > 0) ? (nq + ATT_BM - 1) / ATT_BM : 0;
+    return (nq > 0 && nc > 0) ? (nq + ATT_ITEM - 1) / ATT_ITEM : 0;
   };
   int local = 0;
   for (int e = e0; e < e1; ++e) local += count(e);
@@ -413,13 +627,13 @@ __global__ void __launch_bounds__(1024) k_worklist(const int32_t* qoff, const in
     const int c = count(e);
     for (int t = 0; t < c; ++t) {
       if (e < BH) {
-        const int q0 = t * ATT_BM;
-        items[k++] = make_int4(e, q0, min(ATT_BM, M - q0), -1);
+        const int q0 = t * ATT_ITEM;
+        items[k++] = make_int4(e, q0, min(ATT_ITEM, M - q0), -1);
       } else {
         const int bh = (e - BH) / Gq, i = (e - BH) % Gq;
         const int s = qoff[(size_t)bh * (Gq + 1) + i], en = qoff[(size_t)bh * (Gq + 1) + i + 1];
-        const int q0 = s + t * ATT_BM;
-        items[k++] = make_int4(bh, q0, min(ATT_BM, en - q0), i);
+        const int q0 = s + t * ATT_ITEM;
+        items[k++] = make_int4(bh, q0, min(ATT_ITEM, en - q0), i);
       }
     }
   }
@@ -459,6 +673,22 @@ cudaError_t launch_route(const spr_params& p, const Layout& L, const Ptrs& P, cu
   spr_launch(k_probes, BH, 256, 0, st, P.qoff, P.permq, p.Gq, p.N, p.M,
              p.weights == SPR_WEIGHTS_UNIFORM ? 1 : 0, P.ppos, P.pidx, P.pw,
              P.pslot, P.stats);
+  if (p.probes == SPR_PROBES_RANKED && p.M > 0) {
+    const int split_rows = bq_rows(p.Gk > p.Gq ? p.Gk : p.Gq, D);
+    const float fscale = (float)scale;
+    const long long warps = (long long)BH * p.N;
+    const int grid = (int)((warps * 32 + 255) / 256);
+    if (D == 64)
+      spr_launch(k_probe_dist<64>, grid, 256, 0, st, static_cast<const bf16*>(P.Qp), P.permq,
+                 P.labq, P.rms, P.un2, static_cast<const bf16*>(P.bq16), P.beta, p.N, p.Gq,
+                 split_rows, fscale, BH, P.pdist);
+    else
+      spr_launch(k_probe_dist<128>, grid, 256, 0, st, static_cast<const bf16*>(P.Qp), P.permq,
+                 P.labq, P.rms, P.un2, static_cast<const bf16*>(P.bq16), P.beta, p.N, p.Gq,
+                 split_rows, fscale, BH, P.pdist);
+    spr_launch(k_probes_ranked, dim3(p.Gq, BH), 256, 0, st, P.qoff, P.permq,
+               static_cast<const float*>(P.pdist), p.Gq, p.N, p.M, P.ppos, P.pidx, P.pslot);
+  }
   if (p.M > 0) {
     const int grid = num_sms() * 4;
     if (D == 64)

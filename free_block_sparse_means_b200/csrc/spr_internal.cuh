@@ -16,7 +16,8 @@ constexpr int CHUNK = 512;         // rows per histogram chunk (k-means, permuta
 constexpr int MAX_GROUPS = 256;    // Gk, Gq upper bound
 constexpr int MAX_P = 32;          // eigen-coordinate upper bound (coordinates padded to 32)
 constexpr int MAX_PROBES = 4096;   // M upper bound
-constexpr int ATT_BM = 128;        // query rows per attention work item
+constexpr int ATT_BM = 128;        // query rows per attention tile
+constexpr int ATT_ITEM = 128;      // query rows per attention work item (one tile)
 
 // Device error word codes (first error wins; info words carry details).
 enum : int32_t {
@@ -35,7 +36,7 @@ enum Buf : int {
   B_QBAR, B_LOGIT, B_ENTRY, B_TOP, B_SEL, B_ROWPTR, B_COLIDX, B_RUNPTR, B_RUNS, B_PPOS,
   B_PIDX, B_PW, B_PSLOT, B_QPROBE, B_ITEMS, B_OSP, B_ODN, B_FITU, B_FITB, B_FITBV,
   B_GRAM, B_AXX, B_RXBAR, B_PROJ, B_PART, B_CSUM, B_XP, B_RP, B_PMEAN, B_CRAW64, B_QBAR64,
-  B_SLOTCNT, B_TMASK, B_GBITS, B_BK16, B_ZHL, B_COUNT_
+  B_SLOTCNT, B_TMASK, B_GBITS, B_BK16, B_ZHL, B_PDIST, B_FITW, B_COUNT_
 };
 
 struct Layout {
@@ -79,6 +80,8 @@ struct Ptrs {
   uint32_t *tmask, *gbits;  // k-means update bookkeeping
   bf16* bk16;               // key k-means operand [BH][2][round32(Gk)][64]
   bf16* zhl;                // key coordinates as bf16 hi | lo rows [BH][N][64]
+  float* pdist;             // ranked probes: distance of each permuted query [BH][N]
+  float* fitw;              // W^T = (B U_r^T)^T of the fit [BH][d][d] (d = 128 path)
   int2* runs;
   int4* items;
   uint8_t *sel, *top;
@@ -114,6 +117,16 @@ cudaError_t attend_preload();
 cudaError_t attend_tc_preload();
 cudaError_t launch_reconstruct(const spr_params& p, const Layout& L, const Ptrs& P,
                                bf16* O, cudaStream_t st);
+// Query-response RMS and ||u_hat||^2 on the tensor cores (d = 128), with the
+// chunk sums of ||u_hat||^2 into part (tpart: BH * ceil(N / 128) * 4 doubles).
+cudaError_t launch_rms_tc(const TensorView& Q, int B, int H, int N, int nchunk, int split_rows,
+                          const bf16* bsplit, float scale, const spr_head_stats* stats,
+                          float* rms, float* un2, double* tpart, double* part, Header* hdr,
+                          cudaStream_t st);
+// Residual application on the tensor cores (d = 128): O = x + b + x W per
+// unprobed permuted row, the dense row per probe, bf16 in the original order.
+cudaError_t launch_apply_tc(const spr_params& p, const Layout& L, const Ptrs& P, bf16* O, int R,
+                            cudaStream_t st);
 // Leading eigenpairs of `count` symmetric n x n matrices (fp32, row-major):
 // evals[m * n + k] for the K largest (descending), evecs[(m * n + row) * n + k]
 // the matching unit eigenvectors as columns, trace[m] the trace (may be null).
@@ -135,6 +148,8 @@ struct LloydStep {
   const bf16* bq;      // query mode: [BH][2][split_rows][d] operand (hi, lo)
   bf16* bk;            // key mode: [BH][2][lloyd_ncrows(G)][64] operand (hi, lo)
   const float* rms;    // query mode: row RMS (factor scale / rms)
+  const float* A;      // query mode, optional: A = C~^T C~ [BH][d][d]; the update then also
+                       // writes the next iteration's operand bq and beta (as k_qprep does)
   float scale;
   const float* beta;   // [BH][G]: query beta_g (k_qprep); key ||c_g||^2 / 2 (written by the update)
   float* cent;         // [BH][G][width] centroids, updated in place
@@ -250,7 +265,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // exp2 through the hardware approximation instruction.
 __device__ __forceinline__ float ex2(float x) {
   float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));  // pure: free to schedule
   return y;
 }
 

@@ -93,6 +93,23 @@ enum { SPR_INIT_SEEDED = 0, SPR_INIT_WARM = 1 };
 enum { SPR_WEIGHTS_COVERAGE = 0, SPR_WEIGHTS_UNIFORM = 1 };
 
 /*
+ * Which rows of a query group become its probes.  The per-group counts m_g
+ * (stratified apportionment) and the weights are the same for both.
+ * SPR_PROBES_STRATIFIED takes m_g rows evenly spaced through the group in the
+ * permuted order (the method's stratified selection [paperlayer App. A.2]).
+ * SPR_PROBES_RANKED takes the group's m_g rows nearest its centroid in
+ * query-response coordinates (squared distance ||u_n - c_g||^2, ties to the
+ * lower original query index): the distance-ranked selection of the
+ * probe-selection ablation [paperlayer §4 "Probe-Fitted Residual
+ * Reconstruction" (probes drawn from query partitions and query-response
+ * coordinates); §5 "Ablations", Table 4].  The distance is evaluated in fp32
+ * as ||u_n||^2 - 2 (u_n . c_g - ||c_g||^2 / 2) from the final query
+ * centroids; SPR_PARTITION_SEMANTIC has no query-response coordinates and
+ * returns SPR_EUNSUPPORTED with it.
+ */
+enum { SPR_PROBES_STRATIFIED = 0, SPR_PROBES_RANKED = 1 };
+
+/*
  * Parameters of one call.  Shapes: B batches, H heads, N tokens (N_q = N_k =
  * N, full-sequence attention [paperlayer §2]), head dim d in {64, 128}.
  *
@@ -124,6 +141,11 @@ typedef struct {
                          semantic mode ignores Ms and p */
   int32_t init;       /* SPR_INIT_SEEDED (0, default) or SPR_INIT_WARM */
   int32_t weights;    /* SPR_WEIGHTS_COVERAGE (0, default) or SPR_WEIGHTS_UNIFORM */
+  int32_t probes;     /* SPR_PROBES_STRATIFIED (0, default) or SPR_PROBES_RANKED */
+  int32_t head0;      /* global index of this call's first (batch, head), 0..2^30: the
+                         k-means initial rows of flattened head bh come from the stream
+                         of head head0 + bh, so a call split over head ranges (each
+                         with its own head0) draws exactly what one call would */
 } spr_params;
 
 /* Per-(batch, head) results, copied out by sparsepr_get_stats. */
@@ -244,7 +266,10 @@ typedef enum {
   SPR_VIEW_FIT_B = 20,   /* [BH, d, d] fp32 ridge coefficients B (first r_eff
                             columns); the correction of a row x is b + (x B) U_r^T */
   SPR_VIEW_FIT_BVEC = 21,/* [BH, d] fp32 intercept b = Rbar - (xbar B) U_r^T */
-  SPR_VIEW_COUNT = 22
+  SPR_VIEW_PROBE_DIST = 22,/* [BH, N] fp32 squared distance of each permuted query
+                            to its group's centroid in query-response
+                            coordinates (written with SPR_PROBES_RANKED only) */
+  SPR_VIEW_COUNT = 23
 } spr_view;
 
 spr_status sparsepr_workspace_view(const spr_params* prm, int32_t which, size_t* offset,

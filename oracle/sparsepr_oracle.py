@@ -543,12 +543,15 @@ def rho_exec(counts_q, counts_k, row_ptr, col_idx, M):
 # Whole call
 # ---------------------------------------------------------------------------
 def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
-                  rows=None, want_dense=False, warm=None):
+                  rows=None, want_dense=False, warm=None, probe_pos=None):
     """One (batch, head) SparsePR call, fp64, following the pages' order.
 
     Driven mode: ``lab_k`` / ``lab_q`` (and optionally ``csr``) replace the
     oracle's own clustering (routing) so that everything downstream is
-    recomputed from given assignments.  ``rows`` limits the routed attention
+    recomputed from given assignments; ``probe_pos`` likewise replaces the
+    selected probe positions (ascending, with the selection's own per-group
+    counts; for ranked selection, where rows whose distances tie at the cut
+    may be taken either way).  ``rows`` limits the routed attention
     and the output to those original rows (probe rows are always computed).
     ``warm`` (reading R13) is the ``warm_state`` a previous call returned:
     both k-means then start from its centroids instead of seeded rows.
@@ -650,7 +653,15 @@ def sparsepr_head(Q, K, V, prm: Params, bh=0, lab_k=None, lab_q=None, csr=None,
     if prm.probe_select == "ranked":  # reading R16: nearest to the own query centroid
         dist = ((Xq - Cu[lab_q]) ** 2).sum(axis=1)
         out["probe_dist"] = dist
+        out["probe_u2"] = (Xq * Xq).sum(axis=1)  # ||u||^2, the scale of a fp32 evaluation
     probe_pos, probe_idx, wts, m_g = select_probes(counts_q, q_off, perm_q, prm.M, dist)
+    if probe_pos is not None:  # driven: another valid choice of the same per-group counts
+        given = np.asarray(probe_pos, np.int64)
+        grp = np.searchsorted(np.asarray(q_off, np.int64), given, side="right") - 1
+        if (len(given) != len(probe_pos) or (np.diff(given) <= 0).any()
+                or not (np.bincount(grp, minlength=prm.Gq) == m_g).all()):
+            raise ValueError("driven probe positions do not match the per-group counts")
+        probe_pos, probe_idx = given, np.asarray(perm_q)[given]
     if prm.weights == "uniform" and len(wts):  # the unweighted estimator (reading R14)
         wts = np.full(len(wts), 1.0 / len(wts))
     routed, probe_pairs, rho = rho_exec(counts_q, counts_k, row_ptr, col_idx, prm.M)

@@ -47,6 +47,7 @@ class Workload:
     center_scale: float = 2.0
     partition: str = "response"  # or "semantic" (the comparator)
     weights: str = "coverage"  # or "uniform" (probe weights of the fit)
+    probes: str = "stratified"  # or "ranked" (probe rows nearest their centroid)
 
     @property
     def N(self) -> int:

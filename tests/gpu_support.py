@@ -37,7 +37,7 @@ LABEL_AGREE = 0.99
 def oracle_params(wl, **kw) -> Params:
     d = dict(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
              tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index,
-             weights=wl.weights)
+             weights=wl.weights, probe_select=wl.probes)
     d.update(kw)
     return Params(**d)
 
@@ -53,7 +53,7 @@ def run_gpu(wl, N=None, heads=None, inputs=None, check=None, partition=None):
     prm = spr.make_params(Qd, Kd, Vd, Od, Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
                           seed=wl.index, route_mode=wl.route_mode, tau=wl.tau,
                           rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
-                          partition=partition, weights=wl.weights)
+                          partition=partition, weights=wl.weights, probes=wl.probes)
     ws = spr.alloc_workspace(prm)
     spr.sparsepr_call(prm, Qd, Kd, Vd, Od, ws)
     stats, err = spr.sparsepr_get_stats(prm, ws)
@@ -97,6 +97,8 @@ def collect(prm, ws, Q, K, V, Od, stats, check=None):
     if M > 0:
         out.update(probe_pos=view("probe_pos", i32, (BH, M)), probe_idx=view("probe_idx", i32, (BH, M)),
                    probe_w=view("probe_w", f32, (BH, M)), o_probe=view("o_probe", f32, (BH, M, d)))
+        if prm.probes == spr._binding.PROBES_RANKED:
+            out["probe_dist"] = view("probe_dist", f32, (BH, N))
     return out
 
 
@@ -186,6 +188,12 @@ def check_head(g, wl, bh, rows=None, report=None):
         assert not (diff & ~fr).any(), f"route differs off near-ties at {np.argwhere(diff & ~fr)[:5]}"
         near = int(diff.sum())
         orc = sparsepr_head(q, k, v, prm, bh=bh, lab_k=lab_k, lab_q=lab_q, csr=(rp, ci), rows=rows)
+    probe_swaps = 0
+    if wl.M > 0 and wl.probes == "ranked":
+        probe_swaps = check_ranked_probes(g, orc, bh)
+        if probe_swaps:
+            orc = sparsepr_head(q, k, v, prm, bh=bh, lab_k=lab_k, lab_q=lab_q, csr=gpu_csr(g, bh)
+                                if near else None, rows=rows, probe_pos=g["probe_pos"][bh])
     st = g["stats"][bh]
     assert st["routed_pairs"] == orc["routed_pairs"], "routed pairs"
     assert st["probe_pairs"] == orc["probe_pairs"], "probe pairs"
@@ -206,7 +214,7 @@ def check_head(g, wl, bh, rows=None, report=None):
     e_sp = rel_l2(osp_gpu, orc["O_sp"])
     e_out = rel_l2(g["O"][bh][want], orc["O"])
     res = dict(bh=bh, near_ties=near, live_cells=int(live.sum()), obj_k_rel=ek, obj_q_rel=eq,
-               hard_drop_rel=e_sp, out_rel=e_out)
+               hard_drop_rel=e_sp, out_rel=e_out, probe_swaps=probe_swaps)
     if wl.M > 0:
         res["probe_rel"] = rel_l2(g["o_probe"][bh].astype(np.float64), orc["probe_dense"])
     if report is not None:
@@ -218,6 +226,44 @@ def check_head(g, wl, bh, rows=None, report=None):
     if wl.M > 0:
         assert res["probe_rel"] <= OUT_TOL, f"probe rows rel-L2 {res['probe_rel']}"
     return res, orc
+
+
+DIST_TOL = 2e-5  # ranked probes: fp32 distance error, relative to the group's largest ||u||^2
+
+
+def check_ranked_probes(g, orc, bh):
+    """Distance-ranked probes (reading R16).  The GPU's fp32 distances
+    ||u||^2 - 2 (u.c - ||c||^2 / 2) against the oracle's fp64 ||u - c||^2
+    (both in permuted order), within DIST_TOL of the group's largest ||u||^2
+    (the size the fp32 cancellation error scales with); then, per group,
+    the GPU's m_g rows against the oracle's: a row taken by one side only must
+    sit within twice that tolerance of the oracle's cut (the m_g-th smallest
+    distance).  Returns the number of rows taken differently."""
+    perm, qoff = g["perm_q"][bh].astype(np.int64), orc["q_off"]
+    d_orc = orc["probe_dist"][perm]
+    d_gpu = g["probe_dist"][bh].astype(np.float64)
+    u2 = orc["probe_u2"][perm]
+    swaps = 0
+    gp = g["probe_pos"][bh].astype(np.int64)
+    op = orc["probe_pos"].astype(np.int64)
+    for gi in range(len(qoff) - 1):
+        a, b = int(qoff[gi]), int(qoff[gi + 1])
+        if b <= a:
+            continue
+        scale = float(u2[a:b].max())
+        tol = DIST_TOL * max(scale, 1e-30)
+        err = np.abs(d_gpu[a:b] - d_orc[a:b])
+        assert (err <= tol).all(), f"probe distance group {gi}: max err {err.max()} > {tol}"
+        sg = set(gp[(gp >= a) & (gp < b)].tolist())
+        so = set(op[(op >= a) & (op < b)].tolist())
+        assert len(sg) == len(so), f"probe count group {gi}"
+        if sg == so or not so:
+            continue
+        cut = max(d_orc[p] for p in so)
+        for p in sg ^ so:
+            assert abs(d_orc[p] - cut) <= 2 * tol, f"probe group {gi}: row at {p} is off the cut"
+        swaps += len(sg - so)
+    return swaps
 
 
 def check_kmeans_independent(g, wl, bh, report=None):

@@ -49,10 +49,11 @@ def test_struct_layout_matches_c(tmp_path):
 #include <stddef.h>
 #include "sparsepr.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(spr_params),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(spr_params),
          offsetof(spr_params, scale), offsetof(spr_params, seed), offsetof(spr_params, tau),
          offsetof(spr_params, M), offsetof(spr_params, lambda), offsetof(spr_params, partition),
-         offsetof(spr_params, init), offsetof(spr_params, weights), sizeof(spr_head_stats),
+         offsetof(spr_params, init), offsetof(spr_params, weights), offsetof(spr_params, probes),
+         offsetof(spr_params, head0), sizeof(spr_head_stats),
          offsetof(spr_head_stats, gk_nonempty));
   return 0;
 }
@@ -62,8 +63,8 @@ int main(void) {
     got = list(map(int, subprocess.check_output([str(exe)]).split()))
     P, S = spr.SprParams, spr.SprHeadStats
     want = [ctypes.sizeof(P), P.scale.offset, P.seed.offset, P.tau.offset, P.M.offset,
-            P.lambda_.offset, P.partition.offset, P.init.offset, P.weights.offset, ctypes.sizeof(S),
-            S.gk_nonempty.offset]
+            P.lambda_.offset, P.partition.offset, P.init.offset, P.weights.offset,
+            P.probes.offset, P.head0.offset, ctypes.sizeof(S), S.gk_nonempty.offset]
     assert got == want
 
 
@@ -89,7 +90,13 @@ def test_validation(lib):
     assert spr.sparsepr_check_params(_params(p=33)) == spr._binding.SPR_EUNSUPPORTED
     assert spr.sparsepr_check_params(_params(p=7)) == 0
     assert spr.sparsepr_check_params(_params(partition="semantic")) == 0
-    for field in ("partition", "init", "weights"):
+    # distance-ranked probes need the query-response coordinates
+    assert spr.sparsepr_check_params(_params(probes="ranked")) == 0
+    assert spr.sparsepr_check_params(_params(probes="ranked", partition="semantic")) == \
+        spr._binding.SPR_EUNSUPPORTED
+    assert spr.sparsepr_check_params(_params(head0=23)) == 0
+    assert spr.sparsepr_check_params(_params(head0=-1)) == spr._binding.SPR_EINVAL
+    for field in ("partition", "init", "weights", "probes"):
         prm = _params()
         setattr(prm, field, 2)
         assert spr.sparsepr_check_params(prm) == spr._binding.SPR_EINVAL, field
@@ -98,6 +105,7 @@ def test_validation(lib):
     # the options do not change the workspace a call needs
     n = spr.sparsepr_workspace_size(_params())
     assert spr.sparsepr_workspace_size(_params(init="warm", weights="uniform", partition="semantic")) == n
+    assert spr.sparsepr_workspace_size(_params(probes="ranked")) == n
 
 
 def test_entry_points_reject_before_any_gpu_work(lib):
