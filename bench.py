@@ -172,55 +172,89 @@ def blas_cores():
         return os.cpu_count() or 1
 
 
-ORACLE_WHOLE_HEAD_MAX_N = 16384  # longer heads: attention rows sampled and extrapolated
+ORACLE_WHOLE_HEAD_MAX_N = 16384  # longer heads: attention on sampled query groups, scaled
 
 
-def oracle_head_seconds(wl, bh, sample_rows=2048):
-    """Seconds the fp64 oracle takes for one whole head (independent mode).
+class OracleHead:
+    """The fp64 oracle on one head of a workload, as it stands.
 
-    Up to ORACLE_WHOLE_HEAD_MAX_N tokens the head runs whole.  Longer heads
-    run the whole partition, route, probes (exact dense rows) and fit, but
-    the hard-drop attention of only `sample_rows` rows; that part's time is
-    measured on its own (the oracle's hard_drop_attention on the sampled
-    rows) and scaled to all N rows (rows are independent, each costs about
-    the same).  Returns (seconds, description of the sample).
-    """
-    from oracle import Params, hard_drop_attention, sparsepr_head
-    prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode=wl.route_mode,
-                 tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index,
-                 partition=wl.partition, weights=wl.weights, probe_select=wl.probes)
-    Q, K, V = voronoi_qkv(wl, heads=[bh])
-    q, k, v = (t[0, 0].double().numpy() for t in (Q, K, V))
-    if wl.N <= ORACLE_WHOLE_HEAD_MAX_N:
+    Up to ORACLE_WHOLE_HEAD_MAX_N tokens a head runs whole.  Longer heads
+    run their partition, route, probes (exact dense rows) and fit once
+    (t_fixed); the hard-drop attention, which the oracle evaluates query group
+    by query group (one gather of the routed keys per group), is timed on
+    every row of a sample of whole query groups and scaled by routed pairs
+    (all groups / the sampled ones) to the whole head."""
+
+    def __init__(self, wl, bh):
+        import numpy as np
+        from oracle import Params, sparsepr_head
+        self.wl = wl
+        self.prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters,
+                          route_mode=wl.route_mode, tau=wl.tau, rho_target=wl.rho_target,
+                          M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index, partition=wl.partition,
+                          weights=wl.weights, probe_select=wl.probes)
+        Q, K, V = voronoi_qkv(wl, heads=[bh])
+        self.q, self.k, self.v = (t[0, 0].double().numpy() for t in (Q, K, V))
+        self.whole = wl.N <= ORACLE_WHOLE_HEAD_MAX_N
         t0 = time.perf_counter()
-        sparsepr_head(q, k, v, prm, bh=bh)
-        return time.perf_counter() - t0, "whole head"
-    import numpy as np
-    rows = np.sort(np.random.default_rng(bh).choice(wl.N, sample_rows, replace=False))
-    t0 = time.perf_counter()
-    out = sparsepr_head(q, k, v, prm, bh=bh, rows=rows)
-    t1 = time.perf_counter()
-    hard_drop_attention(q, k, v, out["lab_q"], out["lab_k"], out["row_ptr"], out["col_idx"],
-                        out["scale"], rows=rows)
-    t_rows = time.perf_counter() - t1
-    total = (t1 - t0) + t_rows * (wl.N / sample_rows - 1.0)
-    return total, (f"whole partition, route, probes and fit; hard-drop attention of "
-                   f"{sample_rows} sampled rows scaled to {wl.N}")
+        self.out = sparsepr_head(self.q, self.k, self.v, self.prm, bh=bh,
+                                 rows=None if self.whole else np.arange(min(16, wl.N)))
+        self.t_fixed = time.perf_counter() - t0
+        if not self.whole:
+            o = self.out
+            cq, ck, rp, ci = o["counts_q"], o["counts_k"], o["row_ptr"], o["col_idx"]
+            self.pairs = np.array([cq[i] * ck[ci[rp[i]:rp[i + 1]]].sum() for i in range(len(cq))],
+                                  np.float64)
+            self.live = np.nonzero(self.pairs > 0)[0]
+            self.rng = np.random.default_rng(bh)
+            t, p = self._time(self.live[:1])
+            self.per_pair = max(t / max(p, 1.0), 1e-15)
+
+    def _time(self, groups):
+        import numpy as np
+        from oracle import hard_drop_attention
+        o = self.out
+        rows = np.nonzero(np.isin(o["lab_q"], groups))[0]
+        t0 = time.perf_counter()
+        hard_drop_attention(self.q, self.k, self.v, o["lab_q"], o["lab_k"], o["row_ptr"],
+                            o["col_idx"], o["scale"], rows=rows)
+        return time.perf_counter() - t0, float(self.pairs[groups].sum())
+
+    def groups_for(self, seconds):
+        """Query groups whose attention takes about `seconds`."""
+        g = seconds / (self.per_pair * float(self.pairs[self.live].mean()))
+        return int(min(len(self.live), max(1, g)))
+
+    def head_seconds(self, groups=None):
+        """One estimate of the whole head's time (a fresh group sample)."""
+        if self.whole:
+            return self.t_fixed
+        gs = self.rng.choice(self.live, groups, replace=False)
+        t, p = self._time(gs)
+        return self.t_fixed + t * float(self.pairs.sum()) / p
+
+    def describe(self, groups=None):
+        if self.whole:
+            return "whole head"
+        return (f"partition, route, probes and fit of the head; hard-drop attention of every "
+                f"row of {groups} random query groups, scaled by routed pairs")
 
 
 def oracle_baseline(wl, budget_s=10.0):
     """The oracle as it stands on heads of the workload, ~budget_s of CPU work
-    (at least one head), scaled to all heads."""
+    beyond one head's fixed part (at least one head), scaled to all heads."""
     heads, t_tot, how = 0, 0.0, ""
     while heads < wl.BH and (heads == 0 or t_tot < budget_s):
-        t, how = oracle_head_seconds(wl, heads)
-        t_tot += t
+        h = OracleHead(wl, heads)
+        g = None if h.whole else h.groups_for(budget_s / 2)
+        t_tot += h.head_seconds(g)
+        how = h.describe(g)
         heads += 1
     flops = 4.0 * wl.d * wl.N * wl.N * heads
     return {"value": flops / t_tot / 1e12, "unit": "TFLOP/s (dense-equivalent)",
             "cores": blas_cores(), "kind": "oracle",
             "sample": f"{heads} of {wl.BH} heads of {wl.name} ({how}), fp64 numpy, "
-                      f"{t_tot:.1f} s"}
+                      f"{t_tot:.1f} s estimated"}
 
 
 def partition_bytes(wl):
@@ -249,16 +283,26 @@ def config_of(wl, world):
             "l2": "flushed (256 MiB write) before every timed call"}
 
 
+REF_BUDGET_S = 120.0  # wall-clock target of a whole reference-arm run (steps + warm-up)
+
+
 def run_reference(args, wl):
-    """The oracle as the reference arm: one whole head of the workload per step."""
+    """The oracle as the reference arm, on a bounded sample of the workload
+    (OracleHead): head 0 is set up once; every step is a fresh estimate of its
+    time (whole head, or a fresh sample of whole query groups sized so that
+    the warm-up and the steps take about REF_BUDGET_S)."""
     world, rank, _ = dist_info()
     if rank != 0:
         return 0
-    times, how = [], ""
-    for s in range(args.warmup + args.steps):
-        t, how = oracle_head_seconds(wl, s % wl.BH, sample_rows=args.ref_rows)
+    nsteps = args.warmup + args.steps
+    h = OracleHead(wl, 0)
+    g = None if h.whole else h.groups_for(max(REF_BUDGET_S - h.t_fixed, 10.0) / nsteps)
+    times = []
+    for s in range(nsteps):
+        t = h.head_seconds(g) if not h.whole else OracleHead(wl, s % wl.BH).t_fixed
         if s >= args.warmup:
             times.append(t)
+    sample = f"head 0 of {wl.name}: {h.describe(g)} (fp64 numpy)"
     t = statistics.mean(times)
     val = 4.0 * wl.d * wl.N * wl.N / t / 1e12
     unit = "TFLOP/s (dense-equivalent)"
@@ -268,7 +312,7 @@ def run_reference(args, wl):
             "data": "synthetic", "impl": "reference",
             "config": dict(config_of(wl, 1), kmeans_start="seeded"),
             "cpu_baseline": {"value": val, "unit": unit, "cores": blas_cores(), "kind": "oracle",
-                             "sample": f"one head of {wl.name} per step ({how})"},
+                             "sample": sample},
             "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -507,7 +551,7 @@ def run_ours(args, wl):
     # the output crosses PCIe inside the timed region
     Qh, Kh, Vh = (t.pin_memory() for t in (Qc, Kc, Vc))
     Oh = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
-    e2e_chunk = max(1, -(-wl.BH // E2E_CHUNKS))
+    e2e_chunk = max(1, -(-wl.BH // args.e2e_chunks))
     pipe = spr.HostPipeline(shape, e2e_chunk, device=dev, Ms=wl.Ms, p=wl.p, Gk=wl.Gk,
                             Gq=wl.Gq, iters=wl.iters, seed=wl.index, route_mode=wl.route_mode,
                             tau=wl.tau, rho_target=wl.rho_target, M=wl.M, r=wl.r, lam=wl.lam,
@@ -646,8 +690,6 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
-    ap.add_argument("--ref-rows", type=int, default=2048,
-                    help="reference arm on long workloads: attention rows sampled per head")
     ap.add_argument("--warm-iters", type=int, default=0,
                     help="T > 0: the first warm-up call is seeded, every later call starts its "
                          "k-means from the previous call's centroids and runs T iterations")
@@ -661,6 +703,8 @@ def main(argv=None):
                     help="add the O1 pooled-support and O2 retained-mass diagnostics")
     ap.add_argument("--rho", type=float, default=0.0,
                     help="executed-pair density target (0: the workload's), for density sweeps")
+    ap.add_argument("--e2e-chunks", type=int, default=E2E_CHUNKS,
+                    help="head chunks of the pipelined host-buffer call timed as e2e")
     ap.add_argument("--sweep", action="store_true",
                     help="density x probe budget x rank sweep (one JSON line per point; "
                          "default workload: sweep)")

@@ -19,9 +19,7 @@
 //               MN-major B operand.  A tile whose key range ends early is
 //               multiplied only up to its last 16-key block.
 //   warps 4..7  one thread per query row (= TMEM lane): scaled, masked row
-//               max, exp2 (a quarter of a full tile's exponentials on the FMA
-//               pipe, the rest on the multi-function unit), row sums, P back
-//               to TMEM; O is rescaled in TMEM only
+//               max, exp2, row sums, P back to TMEM; O is rescaled in TMEM only
 //               when the running max grows by more than 2^8 (the final
 //               normalisation uses the same stale max, so this is exact);
 //               epilogue O / l to global memory.
@@ -47,29 +45,6 @@ constexpr uint32_t BOX_BYTES = TBN * 64 * 2;   // one 64-column swizzled box: 16
 constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, TMEM_COLS = 512;
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s
 constexpr size_t SMEM_BYTES = 1024 + (1 + 2 * NST) * TILE_BYTES + 512;
-
-// Coefficients of 2^f on [-1/2, 1/2] (degree 3), fitted for relative error by
-// iteratively reweighted least squares (Lawson's algorithm) on Chebyshev
-// nodes: maximum relative error 7.5e-5, far below the bf16 rounding (2^-9)
-// that P is stored with.  Written out by free_block_sparse_means_b200/exp2_fit.py.
-constexpr float EXP2_C0 = 0.999928073f, EXP2_C1 = 0.693260995f, EXP2_C2 = 0.242611143f,
-                EXP2_C3 = 0.055171627f;
-
-// 2^x for x <= 0 on the FMA and integer pipes (Cody & Waite's reduction
-// x = n + f, n = round(x)): adding 1.5 * 2^23 rounds x to an integer in the
-// low mantissa bits of t (round to nearest), f = x - n lies in [-1/2, 1/2],
-// 2^f comes from the polynomial and 2^n is added to its exponent field.  The
-// shift t << 23 keeps exactly n << 23 (the bits of 1.5 * 2^23 shift out).
-// x is clamped at -125 so that the result stays a normal number; below that
-// 2^x is far under anything a bf16 probability can hold next to the row max
-// (which is 1).  Only full tiles use it (no masked keys there).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, EXP2_C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
 
 struct TcArgs {
   const int4* items;
@@ -372,41 +347,19 @@ __global__ void __launch_bounds__(256, 1)
         const float corr = rescale ? ex2(m - m_use) : 1.f;
         const float neg = -m_use;
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (nvalid == TBN) {
-          // full tile: every fourth exponential on the FMA pipe (exp2_poly),
-          // the rest on the multi-function unit
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 2; ++h) {
+          if (64 * h < nvalid) {  // uniform across the warp: one tile for all rows
             uint32_t pr[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const float x0 = fmaf(__uint_as_float(sr[64 * h + 2 * c]), a.scale_log2, neg);
-              const float x1 = fmaf(__uint_as_float(sr[64 * h + 2 * c + 1]), a.scale_log2, neg);
-              const float p0 = ex2(x0);
-              const float p1 = (c & 1) ? exp2_poly(x1) : ex2(x1);
+              const float p0 = ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c]), a.scale_log2, neg));
+              const float p1 = ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c + 1]), a.scale_log2, neg));
               sum4[c & 3] += p0 + p1;
               pr[c] = pack_bf16(p0, p1);
             }
             __syncwarp();
             tc::tmem_st32(scol + 32 * h, pr);
-          }
-        } else {
-          // partial tile: masked keys carry -inf, which ex2 maps to exactly 0
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (64 * h < nvalid) {  // uniform across the warp: one tile for all rows
-              uint32_t pr[32];
-#pragma unroll
-              for (int c = 0; c < 32; ++c) {
-                const float p0 = ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c]), a.scale_log2, neg));
-                const float p1 =
-                    ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c + 1]), a.scale_log2, neg));
-                sum4[c & 3] += p0 + p1;
-                pr[c] = pack_bf16(p0, p1);
-              }
-              __syncwarp();
-              tc::tmem_st32(scol + 32 * h, pr);
-            }
           }
         }
         const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);

@@ -416,6 +416,7 @@ __global__ void __launch_bounds__(LU_WARPS * 32) k_lloyd_update(LuArgs a) {
   constexpr int VPL = W / 32;                        // update values per lane
   constexpr int INVALID = 0x7fffffff;
   __shared__ float rowf_all[LU_WARPS][LL_TILE];
+  __shared__ int keys_all[LU_WARPS][LL_TILE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * LU_WARPS + warp;
   if (t >= a.BH * a.ntile) return;
@@ -458,17 +459,21 @@ __global__ void __launch_bounds__(LU_WARPS * 32) k_lloyd_update(LuArgs a) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) nkeys += __popc(__ballot_sync(0xffffffffu, key[q] != INVALID));
   warp_sort128(key, lane);
-  // run starts (a label differing from the previous position's)
-  uint32_t sb[4];
+  // the sorted keys, position p = 32 q + lane, for the in-order pass below
+  int* keys = keys_all[warp];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    int pk = __shfl_up_sync(0xffffffffu, key[q], 1);
-    const int carry = q > 0 ? __shfl_sync(0xffffffffu, key[q > 0 ? q - 1 : 0], 31) : -1;
-    if (lane == 0) pk = q > 0 ? carry : -1;
-    const bool st = key[q] != INVALID && (pk < 0 || (pk >> 7) != (key[q] >> 7));
-    sb[q] = __ballot_sync(0xffffffffu, st);
+  for (int q = 0; q < 4; ++q) keys[32 * q + lane] = key[q];
+  __syncwarp();  // keys and row factors visible to the whole warp
+  // row r of the tile: lane's VPL values at xbase + r * xstride
+  const char* xbase;
+  int64_t xstride;
+  if constexpr (MODE == KM_QUERY) {
+    xbase = reinterpret_cast<const char*>(a.X.row(bh, n0) + lane * VPL);
+    xstride = a.X.sn * 2;
+  } else {
+    xbase = reinterpret_cast<const char*>(a.Z + ((size_t)bh * a.N + n0) * LL_KW + lane);
+    xstride = LL_KW * 4;
   }
-  __syncwarp();  // row factors visible to the whole warp
   float acc[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
@@ -487,58 +492,49 @@ __global__ void __launch_bounds__(LU_WARPS * 32) k_lloyd_update(LuArgs a) {
       atomicOr(a.gbits + ((size_t)bh * a.G + cur_g) * a.nword + (tl >> 5), 1u << (tl & 31));
     }
   };
-  constexpr int UB = 8;  // rows loaded ahead of the in-order sums
+  // sorted positions in order, UB rows loaded ahead of the sums; a label
+  // change in the sorted order starts the next run (slot)
+  constexpr int UB = 8;
+  for (int p0 = 0; p0 < nkeys; p0 += UB) {
+    const int pe = min(UB, nkeys - p0);
+    int kk[UB];
+    float x[UB][VPL];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int base = 32 * q;
-    if (base >= nkeys) break;
-    const int cnt_q = min(32, nkeys - base);
-    for (int u0 = 0; u0 < cnt_q; u0 += UB) {
-      int kk[UB];
-      float x[UB][VPL];
-#pragma unroll
-      for (int e = 0; e < UB; ++e) {
-        kk[e] = __shfl_sync(0xffffffffu, key[q], (u0 + e) & 31);
-        const int rr = kk[e] & 127;
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) x[e][v] = 0.f;
-        if (u0 + e < cnt_q) {
-          const int n = n0 + rr;
-          if constexpr (MODE == KM_QUERY && VPL == 4) {  // bf16 -> fp32 is a shift
-            const uint2 raw = *reinterpret_cast<const uint2*>(a.X.row(bh, n) + lane * 4);
-            x[e][0] = __uint_as_float(raw.x << 16);
-            x[e][1] = __uint_as_float(raw.x & 0xffff0000u);
-            x[e][2] = __uint_as_float(raw.y << 16);
-            x[e][3] = __uint_as_float(raw.y & 0xffff0000u);
-          } else if constexpr (MODE == KM_QUERY) {
-            const uint32_t raw = *reinterpret_cast<const uint32_t*>(a.X.row(bh, n) + lane * 2);
-            x[e][0] = __uint_as_float(raw << 16);
-            x[e][1] = __uint_as_float(raw & 0xffff0000u);
-          } else {
-            x[e][0] = a.Z[((size_t)bh * a.N + n) * LL_KW + lane];
-          }
-        }
+    for (int e = 0; e < UB; ++e) {
+      kk[e] = e < pe ? keys[p0 + e] : keys[p0];
+      const char* src = xbase + (int64_t)(kk[e] & 127) * xstride;
+      if constexpr (MODE == KM_QUERY && VPL == 4) {  // bf16 -> fp32 is a shift
+        const uint2 raw = *reinterpret_cast<const uint2*>(src);
+        x[e][0] = __uint_as_float(raw.x << 16);
+        x[e][1] = __uint_as_float(raw.x & 0xffff0000u);
+        x[e][2] = __uint_as_float(raw.y << 16);
+        x[e][3] = __uint_as_float(raw.y & 0xffff0000u);
+      } else if constexpr (MODE == KM_QUERY) {
+        const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
+        x[e][0] = __uint_as_float(raw << 16);
+        x[e][1] = __uint_as_float(raw & 0xffff0000u);
+      } else {
+        x[e][0] = *reinterpret_cast<const float*>(src);
       }
+    }
 #pragma unroll
-      for (int e = 0; e < UB; ++e) {
-        const int u = u0 + e;
-        if (u < cnt_q) {
-          const int p = base + u;
-          if ((sb[q] >> u) & 1u) {
-            if (run >= 0) flush(p - run_start);
-            ++run;
-            run_start = p;
-            cur_g = kk[e] >> 7;
+    for (int e = 0; e < UB; ++e) {
+      if (e < pe) {
+        const int g = kk[e] >> 7;
+        if (g != cur_g) {
+          if (run >= 0) flush(p0 + e - run_start);
+          ++run;
+          run_start = p0 + e;
+          cur_g = g;
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
-          }
-          if (MODE == KM_QUERY) {
-            const float f = rowf[kk[e] & 127];
+          for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
+        }
+        if constexpr (MODE == KM_QUERY) {
+          const float f = rowf[kk[e] & 127];
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) acc[v] = fmaf(f, x[e][v], acc[v]);
-          } else {
-            acc[0] += x[e][0];
-          }
+          for (int v = 0; v < VPL; ++v) acc[v] = fmaf(f, x[e][v], acc[v]);
+        } else {
+          acc[0] += x[e][0];
         }
       }
     }
