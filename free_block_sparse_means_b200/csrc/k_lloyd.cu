@@ -615,9 +615,15 @@ __global__ void __launch_bounds__(W) k_lloyd_reduce(const float* slots, const in
     __syncthreads();
     for (int i = c; i < n; i += W) {  // slot of g in each listed tile: its rank among the labels
       const int tl = list[i];
-      const uint32_t* m = mb + (size_t)tl * 8;
-      int rk = __popc(m[g >> 5] & ((1u << (g & 31)) - 1u));
-      for (int j = 0; j < (g >> 5); ++j) rk += __popc(m[j]);
+      const uint4* m4 = reinterpret_cast<const uint4*>(mb + (size_t)tl * 8);
+      const uint4 ma = m4[0], mc = m4[1];  // the tile's eight mask words, two loads
+      const uint32_t mw[8] = {ma.x, ma.y, ma.z, ma.w, mc.x, mc.y, mc.z, mc.w};
+      int rk = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t keep = j < (g >> 5) ? 0xffffffffu : j == (g >> 5) ? (1u << (g & 31)) - 1u : 0u;
+        rk += __popc(mw[j] & keep);
+      }
       list[i] = tl * LL_SLOTS + rk;
     }
     __syncthreads();
@@ -666,6 +672,7 @@ __global__ void __launch_bounds__(W) k_lloyd_reduce(const float* slots, const in
     __syncthreads();
     const float* Ab = A + (size_t)bh * W * W;
     float sv = 0.f;
+#pragma unroll 16
     for (int j = 0; j < W; ++j) sv += Ab[(size_t)j * W + c] * av[j];
     const bf16 hi = __float2bfloat16_rn(sv);
     const bf16 lo = __float2bfloat16_rn(sv - __bfloat162float(hi));
