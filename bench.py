@@ -369,6 +369,26 @@ def quality_vs_dense(spr, prm, ws, Q, K, V, O, wl, rows_per_head=1024, seed=0):
             "o3_orthogonal_energy_rel": e_orth / den}
 
 
+def dense_sdpa_context(Q, K, V, wl, ms_per_call, flush, stream, reps=3):
+    """Context only, outside the timed region: dense attention on the same
+    inputs with torch's scaled_dot_product_attention (a library kernel), the
+    time a call without any sparsity would take on this GPU."""
+    import torch.nn.functional as F
+    F.scaled_dot_product_attention(Q, K, V)  # warm-up (backend selection)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        F.scaled_dot_product_attention(Q, K, V)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    flop = 4.0 * wl.d * wl.N * wl.N * wl.BH
+    return {"kernel": "torch scaled_dot_product_attention (dense, bf16)", "ms": ms,
+            "tflops": flop / (ms * 1e-3) / 1e12, "sparsepr_speedup": ms / ms_per_call}
+
+
 def support_and_mass(P, keep, alpha=0.9, pool=8):
     """O1 / O2 on sampled query rows (measurement only, torch).
 
@@ -594,6 +614,7 @@ def run_ours(args, wl):
                            f"of one chunk overlapping the computation of the next"},
             "gpu_launches": int(n1 - n0), "clocks": clocks, "device_error": err}
     line["rel_l2_vs_dense"] = quality_vs_dense(spr, prm, ws, Q, K, V, O, wl)
+    line["dense_context"] = dense_sdpa_context(Q, K, V, wl, ms_per_call, flush, stream)
     if args.diagnostics:
         line["diagnostics"] = diagnostics(spr, prm, ws, Q, K, V, wl)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

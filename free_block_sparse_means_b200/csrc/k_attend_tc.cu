@@ -1,5 +1,5 @@
 // Routed attention on the 5th-generation tensor cores (tcgen05, TMEM, TMA) for
-// head dimension 128 [paperlayer §1, §4 "Sparse Execution"; App. A.2].
+// head dimensions 64 and 128 [paperlayer §1, §4 "Sparse Execution"; App. A.2].
 //
 // Each work item is a tile of up to 128 query rows (one query group's rows in
 // the group-major layout, or 128 gathered probe rows) plus its key ranges (the
@@ -37,14 +37,17 @@ namespace spr {
 
 namespace {
 
-constexpr int TBM = 128, TBN = 128, TD = 128;
+constexpr int TBM = 128, TBN = 128;  // query rows and keys per tile
 constexpr int NST = 3;                         // K/V pipeline stages
 constexpr int NITQ = 4;                        // item ring slots
-constexpr uint32_t TILE_BYTES = TBN * TD * 2;  // one Q, K or V tile: 32 KB
 constexpr uint32_t BOX_BYTES = TBN * 64 * 2;   // one 64-column swizzled box: 16 KB
 constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, TMEM_COLS = 512;
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s
-constexpr size_t SMEM_BYTES = 1024 + (1 + 2 * NST) * TILE_BYTES + 512;
+// one Q, K or V tile of head dimension TD (TD / 64 boxes) and the CTA's shared memory
+template <int TD>
+__host__ __device__ constexpr uint32_t tile_bytes() { return TBN * TD * 2; }
+template <int TD>
+__host__ __device__ constexpr size_t smem_bytes() { return 1024 + (1 + 2 * NST) * (size_t)tile_bytes<TD>() + 512; }
 
 struct TcArgs {
   const int4* items;
@@ -95,10 +98,13 @@ struct TileIter {
 
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
+template <int TD>
 __global__ void __launch_bounds__(256, 1)
     k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQprobe,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 TcArgs a) {
+  constexpr uint32_t TILE_BYTES = tile_bytes<TD>();
+  constexpr int NBOX = TD / 64;  // 64-column boxes per row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -178,8 +184,8 @@ __global__ void __launch_bounds__(256, 1)
         tc::mbar_expect_tx(q_full, TILE_BYTES);
         const CUtensorMap* qm = it.w >= 0 ? &tmQ : &tmQprobe;
         const int qrow = it.w >= 0 ? it.x * a.N + it.y : it.x * a.M + it.y;
-        tc::tma_load_2d(sQ, qm, 0, qrow, q_full);
-        tc::tma_load_2d(sQ + BOX_BYTES, qm, 64, qrow, q_full);
+        for (int j = 0; j < NBOX; ++j)
+          tc::tma_load_2d(sQ + j * BOX_BYTES, qm, 64 * j, qrow, q_full);
         ++q_loads;
         for (; I.valid; I.next(), ++kv) {
           const int s = kv % NST;
@@ -192,10 +198,10 @@ __global__ void __launch_bounds__(256, 1)
           uint8_t* vd = kd + TILE_BYTES;
           tc::mbar_expect_tx(kv_full + s, 2 * TILE_BYTES);
           const int krow = it.x * a.N + I.t0;
-          tc::tma_load_2d(kd, &tmK, 0, krow, kv_full + s);
-          tc::tma_load_2d(kd + BOX_BYTES, &tmK, 64, krow, kv_full + s);
-          tc::tma_load_2d(vd, &tmV, 0, krow, kv_full + s);
-          tc::tma_load_2d(vd + BOX_BYTES, &tmV, 64, krow, kv_full + s);
+          for (int j = 0; j < NBOX; ++j) {
+            tc::tma_load_2d(kd + j * BOX_BYTES, &tmK, 64 * j, krow, kv_full + s);
+            tc::tma_load_2d(vd + j * BOX_BYTES, &tmV, 64 * j, krow, kv_full + s);
+          }
         }
       }
       if (*abort_s) {  // let our copies in flight land before the block exits
@@ -457,7 +463,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 // Row-major [rows, 128] bf16 tensor, 64 x 128 boxes, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows) {
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, int TD) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)TD, (cuuint64_t)rows};
@@ -471,10 +477,10 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows) {
 
 }  // namespace
 
-// The tcgen05 path serves d = 128 unless SPR_ATTEND=mma selects the mma.sync
-// kernel (kept for d = 64 and for side-by-side checks).
+// The tcgen05 path serves d = 64 and 128 unless SPR_ATTEND=mma selects the
+// mma.sync kernel (kept for side-by-side checks).
 bool attend_tc_enabled(int d) {
-  if (d != 128) return false;
+  if (d != 64 && d != 128) return false;
   const char* e = getenv("SPR_ATTEND");
   return !(e && strcmp(e, "mma") == 0);
 }
@@ -482,16 +488,19 @@ bool attend_tc_enabled(int d) {
 cudaError_t attend_tc_preload() {
   if (!get_encode()) return cudaErrorInvalidValue;
   cudaFuncAttributes fa;
-  return cudaFuncGetAttributes(&fa, k_attend_tc);
+  cudaError_t e = cudaFuncGetAttributes(&fa, k_attend_tc<64>);
+  return e != cudaSuccess ? e : cudaFuncGetAttributes(&fa, k_attend_tc<128>);
 }
 
 cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P,
                              cudaStream_t st) {
   CUtensorMap mQ, mQp, mK, mV;
   const uint64_t rows = (uint64_t)L.BH * p.N;
-  if (!make_map(&mQ, P.Qp, rows) || !make_map(&mK, P.Kp, rows) || !make_map(&mV, P.Vp, rows))
+  if (!make_map(&mQ, P.Qp, rows, p.d) || !make_map(&mK, P.Kp, rows, p.d) ||
+      !make_map(&mV, P.Vp, rows, p.d))
     return cudaErrorInvalidValue;
-  if (!make_map(&mQp, P.qprobe, (uint64_t)L.BH * (p.M > 0 ? p.M : 1))) return cudaErrorInvalidValue;
+  if (!make_map(&mQp, P.qprobe, (uint64_t)L.BH * (p.M > 0 ? p.M : 1), p.d))
+    return cudaErrorInvalidValue;
   TcArgs a;
   a.items = P.items;
   a.runptr = P.runptr;
@@ -506,10 +515,14 @@ cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P
   a.odn = P.odn;
   a.hdr = P.hdr;
   a.stats = P.stats;
-  cudaError_t e = cudaFuncSetAttribute(k_attend_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  auto go = [&](auto kern, size_t smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    spr_launch(kern, num_sms(), 256, smem, st, mQ, mQp, mK, mV, a);
+    return cudaSuccess;
+  };
+  cudaError_t e = p.d == 64 ? go(k_attend_tc<64>, smem_bytes<64>()) : go(k_attend_tc<128>, smem_bytes<128>());
   if (e != cudaSuccess) return e;
-  spr_launch(k_attend_tc, num_sms(), 256, SMEM_BYTES, st, mQ, mQp, mK, mV, a);
   return cudaGetLastError();
 }
 

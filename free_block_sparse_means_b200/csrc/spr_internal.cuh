@@ -107,7 +107,7 @@ cudaError_t launch_partition(const spr_params& p, const Layout& L, const Ptrs& P
                              cudaStream_t st);
 cudaError_t launch_route(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st);
 cudaError_t launch_attend(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st);
-// tcgen05 routed attention (head dim 128); attend_tc_enabled says whether
+// tcgen05 routed attention (head dims 64 and 128); attend_tc_enabled says whether
 // launch_attend uses it for this head dim.
 cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P, cudaStream_t st);
 bool attend_tc_enabled(int d);
