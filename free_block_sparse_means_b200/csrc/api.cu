@@ -42,7 +42,7 @@ bool make_layout(const spr_params* p, Layout* L) {
   sz[B_PERMQ] = BH * N * 4;
   sz[B_QOFF] = BH * (Gq + 1) * 4;
   sz[B_KP] = BH * N * d * 2;
-  sz[B_VP] = BH * N * d * 2;
+  sz[B_VP] = BH * vt_ld(N) * d * 2;  // [BH][N][d], or transposed [BH][d][vt_ld(N)]
   sz[B_QP] = BH * N * d * 2;
   sz[B_CRAW] = BH * Gk * d * 4;
   sz[B_CT] = BH * Gk * d * 4;
@@ -137,6 +137,7 @@ Ptrs resolve(const Layout& L, void* ws) {
   P.qoff = AT(int32_t*, B_QOFF);
   P.Kp = AT(bf16*, B_KP);
   P.Vp = AT(bf16*, B_VP);
+  P.Vt = attend_tc_enabled(L.d) ? P.Vp : nullptr;
   P.Qp = AT(bf16*, B_QP);
   P.Craw = AT(float*, B_CRAW);
   P.Ct = AT(float*, B_CT);

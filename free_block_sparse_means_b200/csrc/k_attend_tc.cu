@@ -16,8 +16,10 @@
 //               thread: S = Q K^T (A and B K-major in shared memory) into the
 //               S buffer of the tile, and O += P V with P read from TMEM (the
 //               bf16 probabilities the softmax wrote over S) and V as an
-//               MN-major B operand.  A tile whose key range ends early is
-//               multiplied only up to its last 16-key block.
+//               MN-major B operand.  S of a tile whose key range ends early
+//               is computed only up to its last 16-key block; PV always
+//               covers the tile's 128 keys (P is zero past the valid ones),
+//               so that each group of products issues as straight-line code.
 //   warps 4..7  one thread per query row (= TMEM lane): scaled, masked row
 //               max, exp2, row sums, P back to TMEM; O is rescaled in TMEM only
 //               when the running max grows by more than 2^8 (the final
@@ -41,7 +43,7 @@ constexpr int TBM = 128, TBN = 128;  // query rows and keys per tile
 constexpr int NST = 3;                         // K/V pipeline stages
 constexpr int NITQ = 4;                        // item ring slots
 constexpr uint32_t BOX_BYTES = TBN * 64 * 2;   // one 64-column swizzled box: 16 KB
-constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, TMEM_COLS = 512;
+constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, Q_COL = 384, TMEM_COLS = 512;
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s
 // one Q, K or V tile of head dimension TD (TD / 64 boxes) and the CTA's shared memory
 template <int TD>
@@ -61,34 +63,48 @@ struct TcArgs {
   spr_head_stats* stats;
 };
 
-// Key tiles of one item: for each key range [x, y), tiles start at x, x+128, ...
+// Key tiles of one item: for each key range [x, y), the first tile starts at x
+// rounded down to 8 keys, the next ones 128 keys apart.  The transposed values
+// are addressed by key, and a tile's first key must sit on a 16-byte boundary;
+// the first lo keys of a range's first tile lie before the range and are
+// masked.  Both value layouts use the same tiles, so that they sum in the same
+// order.  The range after the current one is loaded when the current one
+// starts, so that moving to it waits on no global load.
 struct TileIter {
   const int2* runs;
-  int r, rend, t0;
-  int2 run;
+  int r, rend, t0, lo;
+  int2 run, nxt;
   bool valid;
+  __device__ void start_run() {
+    t0 = run.x & ~7;
+    lo = run.x - t0;
+  }
   __device__ void init(const TcArgs& a, const int4& it) {
     runs = nullptr;
     r = 0;
     rend = 1;
     run = make_int2(0, a.N);
+    nxt = make_int2(0, 0);
     if (it.w >= 0) {
       r = a.runptr[(size_t)it.x * (a.Gq + 1) + it.w];
       rend = a.runptr[(size_t)it.x * (a.Gq + 1) + it.w + 1];
       runs = a.runs + (size_t)it.x * a.Gq * a.Gk;
       run = r < rend ? runs[r] : make_int2(0, 0);
+      if (r + 1 < rend) nxt = runs[r + 1];
     }
-    t0 = run.x;
+    start_run();
     valid = r < rend && run.x < run.y;
   }
   __device__ int nvalid() const { return min(TBN, run.y - t0); }
   __device__ void next() {
     t0 += TBN;
+    lo = 0;
     if (t0 >= run.y) {
       ++r;
       if (r < rend) {
-        run = runs[r];
-        t0 = run.x;
+        run = nxt;
+        start_run();
+        if (r + 1 < rend) nxt = runs[r + 1];
       } else {
         valid = false;
       }
@@ -98,13 +114,41 @@ struct TileIter {
 
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
-template <int TD>
+// Packed two-lane fp32 arithmetic (sm_100): one instruction for two scores.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n.reg .b64 ra, rb, rc, rd;\n"
+      "mov.b64 ra, {%2, %3};\nmov.b64 rb, {%4, %4};\nmov.b64 rc, {%5, %5};\n"
+      "fma.rn.ftz.f32x2 rd, ra, rb, rc;\nmov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n.reg .b64 ra, rd;\n"
+      "mov.b64 ra, {%2, %3};\nmov.b64 rd, {%0, %1};\n"
+      "add.rn.ftz.f32x2 rd, rd, ra;\nmov.b64 {%0, %1}, rd;\n}\n"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+// three-input maximum (sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// VT: the values are transposed, [BH][d][vt_ld(N)] (tmV maps them), Q is copied
+// into TMEM and both products take their A operand from TMEM and a K-major B
+// from shared memory.  Without VT the values are [BH][N][d] and PV reads them
+// as an MN-major B: a stream that mixes K-major and MN-major operands runs the
+// tensor cores at about half rate.
+template <int TD, bool VT>
 __global__ void __launch_bounds__(256, 1)
     k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQprobe,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 TcArgs a) {
   constexpr uint32_t TILE_BYTES = tile_bytes<TD>();
   constexpr int NBOX = TD / 64;  // 64-column boxes per row
+  constexpr uint32_t VBOX = TD * 128;  // VT: one box of 64 keys x TD rows of the transposed values
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -117,12 +161,12 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* kv_empty = bars + 2 + NST;  // [NST]
   uint64_t* s_full = bars + 2 + 2 * NST;   // [2]
   uint64_t* p_full = bars + 4 + 2 * NST;   // [2]
-  uint64_t* o_done = bars + 6 + 2 * NST;
-  uint64_t* o_free = bars + 7 + 2 * NST;
-  uint64_t* drain = bars + 8 + 2 * NST;
-  uint64_t* it_full = bars + 9 + 2 * NST;           // [NITQ]
-  uint64_t* it_empty = bars + 9 + 2 * NST + NITQ;   // [NITQ]
-  int* it_ring = reinterpret_cast<int*>(bars + 9 + 2 * NST + 2 * NITQ);  // [NITQ]
+  uint64_t* o_done = bars + 6 + 2 * NST;   // [2]: PV(g) of the g-th tile commits o_done[g & 1]
+  uint64_t* o_free = bars + 8 + 2 * NST;
+  uint64_t* drain = bars + 9 + 2 * NST;
+  uint64_t* it_full = bars + 10 + 2 * NST;           // [NITQ]
+  uint64_t* it_empty = bars + 10 + 2 * NST + NITQ;   // [NITQ]
+  int* it_ring = reinterpret_cast<int*>(bars + 10 + 2 * NST + 2 * NITQ);  // [NITQ]
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(it_ring + NITQ);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
@@ -144,6 +188,7 @@ __global__ void __launch_bounds__(256, 1)
       tc::mbar_init(it_empty + s, 1 + 128);  // the MMA thread and every softmax thread
     }
     tc::mbar_init(o_done, 1);
+    tc::mbar_init(o_done + 1, 1);
     tc::mbar_init(o_free, 128);
     tc::mbar_init(drain, 1);
     *abort_s = 0;
@@ -200,8 +245,11 @@ __global__ void __launch_bounds__(256, 1)
           const int krow = it.x * a.N + I.t0;
           for (int j = 0; j < NBOX; ++j) {
             tc::tma_load_2d(kd + j * BOX_BYTES, &tmK, 64 * j, krow, kv_full + s);
-            tc::tma_load_2d(vd + j * BOX_BYTES, &tmV, 64 * j, krow, kv_full + s);
+            if (!VT) tc::tma_load_2d(vd + j * BOX_BYTES, &tmV, 64 * j, krow, kv_full + s);
           }
+          if (VT)  // keys t0 .. t0 + 127 of the TD rows of this head (t0 is a multiple of 8)
+            for (int j = 0; j < 2; ++j)
+              tc::tma_load_2d(vd + j * VBOX, &tmV, I.t0 + 64 * j, it.x * TD, kv_full + s);
         }
       }
       if (*abort_s) {  // let our copies in flight land before the block exits
@@ -213,8 +261,20 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ);
-      int kv = 0, pg = 0;
+      // The issuing thread shares its scheduler with a softmax warp, so its
+      // per-tile instruction count bounds the product stream: descriptors are
+      // formed once and advanced by constant offsets (the start address field
+      // is address >> 4 and never carries), and stages and phases rotate.
+      constexpr uint32_t STAGE_D = (2 * TILE_BYTES) >> 4;  // descriptor step between stages
+      const uint64_t qdesc = tc::smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kdesc0 = tc::smem_desc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t vdesc0 = VT ? tc::smem_desc_sw128(smem_u32(sKV + TILE_BYTES), 16, 1024)
+                                 : tc::smem_desc_sw128(smem_u32(sKV + TILE_BYTES), BOX_BYTES, 1024);
+      const uint32_t idPV = tc::idesc_bf16(TBM, TD, VT ? 0 : 1);
+      int ss = 0, ps = 0;          // K/V stage of the next S and the next PV product
+      uint32_t sph = 0;            // kv_full phase of stage ss
+      uint32_t sb = 0, pb = 0;     // S buffer of the next S and of the next PV product
+      uint32_t pbph = 0;           // p_full phase of buffer pb
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int slot = k % NITQ;
@@ -227,35 +287,43 @@ __global__ void __launch_bounds__(256, 1)
         Is.init(a, it);
         Ip.init(a, it);
         if (!tc::mbar_wait(q_full, k & 1, abort_s, WAIT_NS)) break;
-        int kv_s = kv, sg = pg;
-        auto issue_s = [&]() -> bool {
-          const int s = kv_s % NST;
-          if (!tc::mbar_wait(kv_full + s, (kv_s / NST) & 1, abort_s, WAIT_NS)) return false;
+        if (VT) {  // Q into TMEM; its shared-memory tile is free once copied
           tc::tc_fence_after();
-          const int n16 = (Is.nvalid() + 15) & ~15;
-          const uint32_t idS = tc::idesc_bf16(TBM, n16, 0);
-          const uint32_t d = tbase + ((sg & 1) ? S_COL1 : S_COL0);
-          const uint32_t k_addr = smem_u32(sKV + (size_t)(2 * s) * TILE_BYTES);
+#pragma unroll
+          for (int ks = 0; ks < TD / 16; ++ks)
+            tc::tmem_cp_128x256b(tbase + Q_COL + ks * 8,
+                                 qdesc + (((ks >> 2) * BOX_BYTES + (ks & 3) * 32) >> 4));
+          tc::mma_commit(q_empty);
+        }
+        auto issue_s = [&]() -> bool {
+          if (!tc::mbar_wait(kv_full + ss, sph, abort_s, WAIT_NS)) return false;
+          tc::tc_fence_after();
+          const uint32_t idS = tc::idesc_bf16(TBM, (Is.nvalid() + 15) & ~15, 0);
+          const uint32_t d = tbase + sb * S_COL1;
+          const uint64_t kd = kdesc0 + (uint64_t)(ss * STAGE_D);
 #pragma unroll
           for (int ks = 0; ks < TD / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * BOX_BYTES + (ks & 3) * 32;
-            tc::mma_ss(d, tc::smem_desc_sw128(q_addr + off, 16, 1024),
-                       tc::smem_desc_sw128(k_addr + off, 16, 1024), idS, ks > 0);
+            const uint32_t off = ((ks >> 2) * BOX_BYTES + (ks & 3) * 32) >> 4;
+            if (VT)
+              tc::mma_ts(d, tbase + Q_COL + ks * 8, kd + off, idS, ks > 0);
+            else
+              tc::mma_ss(d, qdesc + off, kd + off, idS, ks > 0);
           }
-          tc::mma_commit(s_full + (sg & 1));
-          ++kv_s;
-          ++sg;
+          tc::mma_commit(s_full + sb);
+          if (++ss == NST) {
+            ss = 0;
+            sph ^= 1u;
+          }
+          sb ^= 1u;
           return true;
         };
         for (int j = 0; j < 2 && Is.valid && ok; ++j) {
           ok = issue_s();
           Is.next();
         }
-        const uint32_t idPV = tc::idesc_bf16(TBM, TD, 1);
         bool first = true;
         for (; Ip.valid && ok; Ip.next()) {
-          const int b = pg & 1;
-          if (!tc::mbar_wait(p_full + b, (pg >> 1) & 1, abort_s, WAIT_NS)) {
+          if (!tc::mbar_wait(p_full + pb, pbph, abort_s, WAIT_NS)) {
             ok = false;
             break;
           }
@@ -264,25 +332,27 @@ __global__ void __launch_bounds__(256, 1)
             break;
           }
           tc::tc_fence_after();
-          const int s = kv % NST;
-          const uint32_t v_addr = smem_u32(sKV + (size_t)(2 * s + 1) * TILE_BYTES);
-          const uint32_t p_col = tbase + (b ? S_COL1 : S_COL0);
-          const int nk = (Ip.nvalid() + 15) >> 4;  // 16-key blocks holding valid keys
-          for (int kk = 0; kk < nk; ++kk)
-            tc::mma_ts(tbase + O_COL, p_col + kk * 8,
-                       tc::smem_desc_sw128(v_addr + kk * 2048, BOX_BYTES, 1024), idPV,
-                       !(first && kk == 0));
-          tc::mma_commit(kv_empty + s);
-          tc::mma_commit(o_done);
+          const uint64_t vd = vdesc0 + (uint64_t)(ps * STAGE_D);
+          const uint32_t p_col = tbase + pb * S_COL1;
+          // every 16-key block of the tile, as straight-line code (a branch
+          // between products slows their issue); P is zero past the valid keys
+#pragma unroll
+          for (int kk = 0; kk < TBN / 16; ++kk) {
+            const uint32_t voff = VT ? ((kk >> 2) * VBOX + (kk & 3) * 32) >> 4 : kk * (2048 >> 4);
+            tc::mma_ts(tbase + O_COL, p_col + kk * 8, vd + voff, idPV, !(first && kk == 0));
+          }
+          tc::mma_commit(kv_empty + ps);
+          tc::mma_commit(o_done + pb);
           first = false;
-          ++kv;
-          ++pg;
+          if (++ps == NST) ps = 0;
+          pb ^= 1u;
+          if (pb == 0) pbph ^= 1u;
           if (Is.valid) {
             ok = issue_s();
             Is.next();
           }
         }
-        tc::mma_commit(q_empty);
+        if (!VT) tc::mma_commit(q_empty);  // the last S product has read the Q tile
       }
       // drain: every MMA issued so far completes before TMEM is released
       tc::mma_commit(drain);
@@ -292,7 +362,7 @@ __global__ void __launch_bounds__(256, 1)
     // ------------------------------------------------------------ softmax
     const int row = threadIdx.x - 128;                          // query row in the tile
     const uint32_t lane_f = (uint32_t)((warp & 3) * 32) << 16;  // TMEM lane field
-    int pg = 0, pvseen = 0;
+    int pg = 0;  // tiles this CTA has processed: the g of the tile below
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int slot = k % NITQ;
@@ -335,13 +405,22 @@ __global__ void __launch_bounds__(256, 1)
           for (int c = 0; c < TBN; ++c)
             if (c >= nvalid) sr[c] = f2u(-INFINITY);
         }
+        if (I.lo > 0) {  // keys before the range in its first, 8-aligned tile
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            if (c < I.lo) sr[c] = f2u(-INFINITY);
+        }
         float mx8[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) mx8[q] = __uint_as_float(sr[q]);
+        for (int q = 0; q < 8; ++q)
+          mx8[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
 #pragma unroll
-        for (int c = 8; c < TBN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+        for (int c = 16; c < TBN; c += 16)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            mx8[q] = max3(mx8[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + 8 + q]));
+        const float mx = fmaxf(max3(mx8[0], mx8[1], mx8[2]),
+                               max3(max3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) *
                          a.scale_log2;
         const float mn = fmaxf(m, mx);
         float m_use = m;
@@ -359,39 +438,58 @@ __global__ void __launch_bounds__(256, 1)
             uint32_t pr[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const float p0 = ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c]), a.scale_log2, neg));
-              const float p1 = ex2(fmaf(__uint_as_float(sr[64 * h + 2 * c + 1]), a.scale_log2, neg));
-              sum4[c & 3] += p0 + p1;
+              float x0, x1;
+              fma2(x0, x1, __uint_as_float(sr[64 * h + 2 * c]),
+                   __uint_as_float(sr[64 * h + 2 * c + 1]), a.scale_log2, neg);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              add2(sum4[2 * (c & 1)], sum4[2 * (c & 1) + 1], p0, p1);
               pr[c] = pack_bf16(p0, p1);
             }
             __syncwarp();
             tc::tmem_st32(scol + 32 * h, pr);
+          } else {  // no valid key in this half: P = 0 for the PV product
+            uint32_t z[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) z[c] = 0u;
+            __syncwarp();
+            tc::tmem_st32(scol + 32 * h, z);
           }
         }
         const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-        if (!first) {  // O holds PV of the previous tile once it is done
-          const bool got_o = tc::mbar_wait(o_done, pvseen & 1, abort_s, WAIT_NS);
+        // P(g) is released without waiting for PV(g - 1): only a rescale of O
+        // has to wait for it.  Waiting here for PV(g - 2), done long before,
+        // keeps at most two phases of o_done[g & 1] in play, so that every
+        // parity wait on it (here, the rescale's and the epilogue's) is exact.
+        if (pg >= 2) {
+          const bool got = tc::mbar_wait(o_done + (pg & 1), ((pg - 2) >> 1) & 1, abort_s, WAIT_NS);
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+        }
+        // the rescale is per row, the TMEM access per warp: a warp rescales
+        // when any of its rows needs it (the others multiply by 1), once
+        // PV(g - 1) has finished accumulating into O
+        if (__any_sync(0xffffffffu, rescale)) {
+          const bool got_o =
+              tc::mbar_wait(o_done + ((pg - 1) & 1), ((pg - 1) >> 1) & 1, abort_s, WAIT_NS);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
             break;
           }
-          ++pvseen;
           tc::tc_fence_after();
-          // the rescale is per row, the TMEM access per warp: a warp rescales
-          // when any of its rows needs it (the others multiply by 1)
-          if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-            for (int c = 0; c < TD / 32; ++c) {
-              uint32_t o[32];
-              __syncwarp();
-              tc::tmem_ld32(tbase + lane_f + O_COL + 32 * c, o);
-              tc::tmem_wait_ld();
+          for (int c = 0; c < TD / 32; ++c) {
+            uint32_t o[32];
+            __syncwarp();
+            tc::tmem_ld32(tbase + lane_f + O_COL + 32 * c, o);
+            tc::tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = f2u(__uint_as_float(o[e]) * corr);
-              __syncwarp();
-              tc::tmem_st32(tbase + lane_f + O_COL + 32 * c, o);
-            }
+            for (int e = 0; e < 32; ++e) o[e] = f2u(__uint_as_float(o[e]) * corr);
+            __syncwarp();
+            tc::tmem_st32(tbase + lane_f + O_COL + 32 * c, o);
           }
         }
         l = l * corr + sum;
@@ -407,13 +505,13 @@ __global__ void __launch_bounds__(256, 1)
         tc::mbar_arrive(o_free);
         continue;
       }
-      const bool got_o = tc::mbar_wait(o_done, pvseen & 1, abort_s, WAIT_NS);
+      const int gl = pg - 1;  // the item's last tile: its PV completes after all others
+      const bool got_o = tc::mbar_wait(o_done + (gl & 1), (gl >> 1) & 1, abort_s, WAIT_NS);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got_o)) {
         ok = false;
         break;
       }
-      ++pvseen;
       tc::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       float* dst = it.w >= 0 ? a.osp + ((size_t)it.x * a.N + it.y + row) * TD
@@ -475,6 +573,20 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, int TD) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Transposed values [BH * TD rows][ld keys] (ld a multiple of 8), boxes of 64
+// keys x TD rows, 128-byte swizzle.
+bool make_map_vt(CUtensorMap* m, const void* ptr, uint64_t BH, int TD, uint64_t ld) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)ld, (cuuint64_t)(BH * TD)};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)TD};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 // The tcgen05 path serves d = 64 and 128 unless SPR_ATTEND=mma selects the
@@ -488,16 +600,20 @@ bool attend_tc_enabled(int d) {
 cudaError_t attend_tc_preload() {
   if (!get_encode()) return cudaErrorInvalidValue;
   cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, k_attend_tc<64>);
-  return e != cudaSuccess ? e : cudaFuncGetAttributes(&fa, k_attend_tc<128>);
+  cudaError_t e = cudaFuncGetAttributes(&fa, k_attend_tc<64, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, k_attend_tc<128, false>);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, k_attend_tc<64, true>);
+  return e != cudaSuccess ? e : cudaFuncGetAttributes(&fa, k_attend_tc<128, true>);
 }
 
 cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P,
                              cudaStream_t st) {
   CUtensorMap mQ, mQp, mK, mV;
   const uint64_t rows = (uint64_t)L.BH * p.N;
+  const bool vt = P.Vt != nullptr;
   if (!make_map(&mQ, P.Qp, rows, p.d) || !make_map(&mK, P.Kp, rows, p.d) ||
-      !make_map(&mV, P.Vp, rows, p.d))
+      !(vt ? make_map_vt(&mV, P.Vt, (uint64_t)L.BH, p.d, (uint64_t)vt_ld(p.N))
+           : make_map(&mV, P.Vp, rows, p.d)))
     return cudaErrorInvalidValue;
   if (!make_map(&mQp, P.qprobe, (uint64_t)L.BH * (p.M > 0 ? p.M : 1), p.d))
     return cudaErrorInvalidValue;
@@ -521,7 +637,12 @@ cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P
     spr_launch(kern, num_sms(), 256, smem, st, mQ, mQp, mK, mV, a);
     return cudaSuccess;
   };
-  cudaError_t e = p.d == 64 ? go(k_attend_tc<64>, smem_bytes<64>()) : go(k_attend_tc<128>, smem_bytes<128>());
+  cudaError_t e;
+  if (p.d == 64)
+    e = vt ? go(k_attend_tc<64, true>, smem_bytes<64>()) : go(k_attend_tc<64, false>, smem_bytes<64>());
+  else
+    e = vt ? go(k_attend_tc<128, true>, smem_bytes<128>())
+           : go(k_attend_tc<128, false>, smem_bytes<128>());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -341,6 +341,53 @@ __global__ void __launch_bounds__(256) k_gather_rows(TensorView src, const int32
   }
 }
 
+// Transposed gather: dst[bh][c][n] = src(bh, perm[bh][n])[c] for the values in
+// the group-major key order, rows of vt_ld(N) keys (the tail past N is zero).
+// One block per 64 keys of one head: the 64 source rows are read whole into
+// shared memory, and each of the D output rows gets its 64 keys as eight
+// 16-byte stores.  Row stride of the staging tile: D + 8 elements, so that the
+// column reads of the transpose spread over the banks.
+template <int D>
+__global__ void __launch_bounds__(256) k_gather_vt(TensorView src, const int32_t* perm, int N,
+                                                   bf16* dst) {
+  constexpr int KB = 64, LD = D + 8;
+  __shared__ __align__(16) bf16 tile[KB * LD];
+  const int bh = blockIdx.y, n0 = blockIdx.x * KB;
+  const int64_t ld = vt_ld(N);
+  for (int e = threadIdx.x; e < KB * (D / 8); e += 256) {
+    const int r = e / (D / 8), c = e % (D / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (n0 + r < N) {
+      const int n = perm[(int64_t)bh * N + n0 + r];
+      v = reinterpret_cast<const uint4*>(src.row(bh, n))[c];
+    }
+    *reinterpret_cast<uint4*>(tile + r * LD + c * 8) = v;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < D * (KB / 8); e += 256) {
+    const int c = e / (KB / 8), k8 = e % (KB / 8);
+    if (n0 + k8 * 8 >= ld) continue;  // past the padded row
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint16_t lo = reinterpret_cast<const uint16_t*>(tile)[(k8 * 8 + 2 * i) * LD + c];
+      const uint16_t hi = reinterpret_cast<const uint16_t*>(tile)[(k8 * 8 + 2 * i + 1) * LD + c];
+      w[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    *reinterpret_cast<uint4*>(dst + ((int64_t)bh * D + c) * ld + n0 + k8 * 8) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// The values in the group-major key order, in the layout the attention reads.
+template <int D>
+void gather_values(TensorView V, const Ptrs& P, int N, int BH, int ggrid, cudaStream_t st) {
+  if (P.Vt)
+    spr_launch(k_gather_vt<D>, dim3((N + 63) / 64, BH), 256, 0, st, V, P.permk, N, P.Vt);
+  else
+    spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
+}
+
 // ---------------------------------------------------------------------------
 // Centred nonempty K/V centroids [paperlayer App. B.2]: Ctilde rows (compacted,
 // ascending group index) = c_j - mean over nonempty j of c_j.
@@ -677,7 +724,7 @@ static cudaError_t partition_semantic_d(const spr_params& p, const Layout& L, co
   spr_launch(k_obj_rows<D>, dim3(nchunk, BH), 256, 0, st, K, N, p.Gk, P.Craw, P.labk, nchunk, 0,
              P.part);
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
-  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
+  gather_values<D>(V, P, N, BH, ggrid, st);
   spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.gpart);
   spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.gpart, P.kvoff, p.Gk, P.Craw, P.craw64);
   spr_launch(k_center, BH, 256, 0, st, P.Craw, P.counts, p.Gk, D, P.Ct, P.stats);
@@ -758,7 +805,7 @@ spr_launch(k_obj_z<32>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.l
   // Paired K/V groups: permuted keys and values, raw-key centroids
   const int ggrid = sms * 8;
   spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, K, P.permk, N, BH, P.Kp);
-  spr_launch(k_gather_rows<D>, ggrid, 256, 0, st, V, P.permk, N, BH, P.Vp);
+  gather_values<D>(V, P, N, BH, ggrid, st);
   spr_launch(k_gmean_part<D>, dim3(p.Gk, BH, GM_SLICES), 256, 0, st, P.Kp, P.kvoff, N, p.Gk, P.gpart);
   spr_launch(k_gmean_fin<D>, dim3(p.Gk, BH), D, 0, st, P.gpart, P.kvoff, p.Gk, P.Craw, P.craw64);
   // P.counts holds |K_j| now; keep a copy of key counts in kv_off differences.

@@ -86,7 +86,15 @@ struct Ptrs {
   int4* items;
   uint8_t *sel, *top;
   bf16 *Kp, *Vp, *Qp, *bq16, *qprobe;
+  // Vp holds V in the group-major key order, [BH][N][d]; when the tensor-core
+  // attention runs (attend_tc_enabled), the partition writes it transposed
+  // instead, [BH][d][vt_ld(N)], and Vt points at it (null otherwise).
+  bf16* Vt;
 };
+
+// Row length of the transposed V: N rounded up to 8 keys (16 bytes), so that
+// every row starts 16-byte aligned for the tensor-memory-access unit.
+__host__ __device__ inline int64_t vt_ld(int64_t N) { return (N + 7) & ~int64_t(7); }
 
 Ptrs resolve(const Layout& L, void* ws);
 
