@@ -43,7 +43,8 @@ constexpr int TBM = 128, TBN = 128;  // query rows and keys per tile
 constexpr int NST = 3;                         // K/V pipeline stages
 constexpr int NITQ = 4;                        // item ring slots
 constexpr uint32_t BOX_BYTES = TBN * 64 * 2;   // one 64-column swizzled box: 16 KB
-constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, Q_COL = 384, TMEM_COLS = 512;
+constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, Q_COL = 384, X_COL = 448, TMEM_COLS = 512;
+constexpr int ATT_THREADS = 384;  // producer, MMA issuer, two idle warps, eight softmax warps
 constexpr uint64_t WAIT_NS = 2000000000ull;  // 2 s
 // one Q, K or V tile of head dimension TD (TD / 64 boxes) and the CTA's shared memory
 template <int TD>
@@ -142,7 +143,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // as an MN-major B: a stream that mixes K-major and MN-major operands runs the
 // tensor cores at about half rate.
 template <int TD, bool VT>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(ATT_THREADS, 1)
     k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQprobe,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 TcArgs a) {
@@ -166,7 +167,9 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* drain = bars + 9 + 2 * NST;
   uint64_t* it_full = bars + 10 + 2 * NST;           // [NITQ]
   uint64_t* it_empty = bars + 10 + 2 * NST + NITQ;   // [NITQ]
-  int* it_ring = reinterpret_cast<int*>(bars + 10 + 2 * NST + 2 * NITQ);  // [NITQ]
+  uint64_t* pair_bar = bars + 10 + 2 * NST + 2 * NITQ;      // [4] softmax pairs, once per tile
+  uint64_t* ep_bar = bars + 14 + 2 * NST + 2 * NITQ;        // [4] softmax pairs, once per item
+  int* it_ring = reinterpret_cast<int*>(bars + 18 + 2 * NST + 2 * NITQ);  // [NITQ]
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(it_ring + NITQ);
   volatile int* abort_s = reinterpret_cast<volatile int*>(tmem_base_s + 1);
 
@@ -181,15 +184,19 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(s_full + s, 1);
-      tc::mbar_init(p_full + s, 128);
+      tc::mbar_init(p_full + s, 256);
     }
     for (int s = 0; s < NITQ; ++s) {
       tc::mbar_init(it_full + s, 1);
-      tc::mbar_init(it_empty + s, 1 + 128);  // the MMA thread and every softmax thread
+      tc::mbar_init(it_empty + s, 1 + 256);  // the MMA thread and every softmax thread
+    }
+    for (int s = 0; s < 4; ++s) {
+      tc::mbar_init(pair_bar + s, 64);
+      tc::mbar_init(ep_bar + s, 64);
     }
     tc::mbar_init(o_done, 1);
     tc::mbar_init(o_done + 1, 1);
-    tc::mbar_init(o_free, 128);
+    tc::mbar_init(o_free, 256);
     tc::mbar_init(drain, 1);
     *abort_s = 0;
     tc::fence_barrier_init();
@@ -360,9 +367,19 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int row = threadIdx.x - 128;                          // query row in the tile
-    const uint32_t lane_f = (uint32_t)((warp & 3) * 32) << 16;  // TMEM lane field
+    // Two warps per quarter of the rows: warps 4 + q and 8 + q both hold rows
+    // 32q .. 32q + 31 (their TMEM lanes); the first takes keys 0 .. 63 of
+    // every tile, the second keys 64 .. 127, so that each scheduler runs two
+    // softmax warps and one's bookkeeping overlaps the other's exponentials.
+    // The pair agrees on each tile's row max, and adds its row sums at the
+    // end of an item, through TMEM columns X_COL.. and a pair barrier.
+    const int q = warp & 3, hh = (warp - 4) >> 2;               // row quarter, key half
+    const int row = 32 * q + lane;                              // query row in the tile
+    const uint32_t lane_f = (uint32_t)(q * 32) << 16;           // TMEM lane field
+    const uint32_t xcol = tbase + lane_f + X_COL;
+    constexpr int OH = TD / 2;                                  // O columns of one half
     int pg = 0;  // tiles this CTA has processed: the g of the tile below
+    int ng = 0;  // items with tiles this CTA has processed
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int slot = k % NITQ;
@@ -392,36 +409,54 @@ __global__ void __launch_bounds__(256, 1)
           break;
         }
         tc::tc_fence_after();
-        uint32_t sr[TBN];
+        uint32_t sr[64];  // keys 64 hh .. 64 hh + 63 of the tile
 #pragma unroll
-        for (int c = 0; c < TBN / 32; ++c)
-          if (c < nch) tc::tmem_ld32(scol + 32 * c, sr + 32 * c);
+        for (int c = 0; c < 2; ++c)
+          if (2 * hh + c < nch) tc::tmem_ld32(scol + 64 * hh + 32 * c, sr + 32 * c);
         tc::tmem_wait_ld();
-        // row max of the raw scores (the scale is positive), in eight
-        // independent chains; keys past the tile's valid count (partial
-        // tiles only) are masked to -inf
-        if (nvalid < TBN) {
+        // keys past the tile's valid count, and keys before the range in its
+        // first, 8-aligned tile, are masked to -inf
+        if (nvalid < 64 * hh + 64) {
 #pragma unroll
-          for (int c = 0; c < TBN; ++c)
-            if (c >= nvalid) sr[c] = f2u(-INFINITY);
+          for (int c = 0; c < 64; ++c)
+            if (64 * hh + c >= nvalid) sr[c] = f2u(-INFINITY);
         }
-        if (I.lo > 0) {  // keys before the range in its first, 8-aligned tile
+        if (hh == 0 && I.lo > 0) {
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             if (c < I.lo) sr[c] = f2u(-INFINITY);
         }
+        // max of the raw scores of this half (the scale is positive)
         float mx8[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          mx8[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
+        for (int e = 0; e < 8; ++e)
+          mx8[e] = fmaxf(__uint_as_float(sr[e]), __uint_as_float(sr[e + 8]));
 #pragma unroll
-        for (int c = 16; c < TBN; c += 16)
+        for (int c = 16; c < 64; c += 16)
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            mx8[q] = max3(mx8[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + 8 + q]));
-        const float mx = fmaxf(max3(mx8[0], mx8[1], mx8[2]),
-                               max3(max3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) *
-                         a.scale_log2;
+          for (int e = 0; e < 8; ++e)
+            mx8[e] = max3(mx8[e], __uint_as_float(sr[c + e]), __uint_as_float(sr[c + 8 + e]));
+        const float mxh = fmaxf(max3(mx8[0], mx8[1], mx8[2]),
+                                max3(max3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+        // exchange with the other half of the row: column X_COL + 2 b + hh
+        // holds this half's max of tile g; it is next written at tile g + 2,
+        // after the pair barrier of tile g + 1, which needs this thread's
+        // read below
+        __syncwarp();
+        tc::tmem_st1(xcol + 2 * b + hh, f2u(mxh));
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::mbar_arrive(pair_bar + q);
+        const bool got_x = tc::mbar_wait(pair_bar + q, pg & 1, abort_s, WAIT_NS);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got_x)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const float mxo = __uint_as_float(tc::tmem_ld1(xcol + 2 * b + (1 - hh)));
+        tc::tmem_wait_ld();
+        const float mx = fmaxf(mxh, mxo) * a.scale_log2;  // the same value in both halves
         const float mn = fmaxf(m, mx);
         float m_use = m;
         bool rescale = false;
@@ -432,28 +467,25 @@ __global__ void __launch_bounds__(256, 1)
         const float corr = rescale ? ex2(m - m_use) : 1.f;
         const float neg = -m_use;
         float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (64 * hh < nvalid) {  // uniform across the warp: one tile for all rows
+          uint32_t pr[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (64 * h < nvalid) {  // uniform across the warp: one tile for all rows
-            uint32_t pr[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              float x0, x1;
-              fma2(x0, x1, __uint_as_float(sr[64 * h + 2 * c]),
-                   __uint_as_float(sr[64 * h + 2 * c + 1]), a.scale_log2, neg);
-              const float p0 = ex2(x0), p1 = ex2(x1);
-              add2(sum4[2 * (c & 1)], sum4[2 * (c & 1) + 1], p0, p1);
-              pr[c] = pack_bf16(p0, p1);
-            }
-            __syncwarp();
-            tc::tmem_st32(scol + 32 * h, pr);
-          } else {  // no valid key in this half: P = 0 for the PV product
-            uint32_t z[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) z[c] = 0u;
-            __syncwarp();
-            tc::tmem_st32(scol + 32 * h, z);
+          for (int c = 0; c < 32; ++c) {
+            float x0, x1;
+            fma2(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]),
+                 a.scale_log2, neg);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            add2(sum4[2 * (c & 1)], sum4[2 * (c & 1) + 1], p0, p1);
+            pr[c] = pack_bf16(p0, p1);
           }
+          __syncwarp();
+          tc::tmem_st32(scol + 32 * hh, pr);
+        } else {  // no valid key in this half: P = 0 for the PV product
+          uint32_t z[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) z[c] = 0u;
+          __syncwarp();
+          tc::tmem_st32(scol + 32 * hh, z);
         }
         const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
         // P(g) is released without waiting for PV(g - 1): only a rescale of O
@@ -469,8 +501,9 @@ __global__ void __launch_bounds__(256, 1)
           }
         }
         // the rescale is per row, the TMEM access per warp: a warp rescales
-        // when any of its rows needs it (the others multiply by 1), once
-        // PV(g - 1) has finished accumulating into O
+        // its half of O's columns when any of its rows needs it (the others
+        // multiply by 1; both halves of a row decide alike), once PV(g - 1)
+        // has finished accumulating into O
         if (__any_sync(0xffffffffu, rescale)) {
           const bool got_o =
               tc::mbar_wait(o_done + ((pg - 1) & 1), ((pg - 1) >> 1) & 1, abort_s, WAIT_NS);
@@ -481,15 +514,15 @@ __global__ void __launch_bounds__(256, 1)
           }
           tc::tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < TD / 32; ++c) {
+          for (int c = 0; c < OH / 32; ++c) {
             uint32_t o[32];
             __syncwarp();
-            tc::tmem_ld32(tbase + lane_f + O_COL + 32 * c, o);
+            tc::tmem_ld32(tbase + lane_f + O_COL + OH * hh + 32 * c, o);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = f2u(__uint_as_float(o[e]) * corr);
             __syncwarp();
-            tc::tmem_st32(tbase + lane_f + O_COL + 32 * c, o);
+            tc::tmem_st32(tbase + lane_f + O_COL + OH * hh + 32 * c, o);
           }
         }
         l = l * corr + sum;
@@ -512,15 +545,33 @@ __global__ void __launch_bounds__(256, 1)
         ok = false;
         break;
       }
+      // the row sum of both halves (column X_COL + 4 + hh, next written at the
+      // next item's end, after this item's pair barrier has been passed by both)
+      __syncwarp();
+      tc::tmem_st1(xcol + 4 + hh, f2u(l));
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(ep_bar + q);
+      const bool got_e = tc::mbar_wait(ep_bar + q, ng & 1, abort_s, WAIT_NS);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got_e)) {
+        ok = false;
+        break;
+      }
+      ++ng;
       tc::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* dst = it.w >= 0 ? a.osp + ((size_t)it.x * a.N + it.y + row) * TD
-                             : a.odn + ((size_t)it.x * a.M + it.y + row) * TD;
+      const float lo_ = __uint_as_float(tc::tmem_ld1(xcol + 4 + (1 - hh)));
+      tc::tmem_wait_ld();
+      const float lt = hh == 0 ? l + lo_ : lo_ + l;  // the same sum in both halves
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      float* dst = (it.w >= 0 ? a.osp + ((size_t)it.x * a.N + it.y + row) * TD
+                              : a.odn + ((size_t)it.x * a.M + it.y + row) * TD) +
+                   OH * hh;
 #pragma unroll
-      for (int c = 0; c < TD / 32; ++c) {
+      for (int c = 0; c < OH / 32; ++c) {
         uint32_t o[32];
         __syncwarp();
-        tc::tmem_ld32(tbase + lane_f + O_COL + 32 * c, o);
+        tc::tmem_ld32(tbase + lane_f + O_COL + OH * hh + 32 * c, o);
         tc::tmem_wait_ld();
         if (row < it.z) {
           float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
@@ -533,7 +584,7 @@ __global__ void __launch_bounds__(256, 1)
       }
       tc::tc_fence_before();
       tc::mbar_arrive(o_free);
-      if (row == 0)
+      if (row == 0 && hh == 0)
         atomicAdd(reinterpret_cast<unsigned long long*>(&a.stats[it.x].tile_pairs), exec_pairs);
     }
   }
@@ -634,7 +685,7 @@ cudaError_t launch_attend_tc(const spr_params& p, const Layout& L, const Ptrs& P
   auto go = [&](auto kern, size_t smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    spr_launch(kern, num_sms(), 256, smem, st, mQ, mQp, mK, mV, a);
+    spr_launch(kern, num_sms(), ATT_THREADS, smem, st, mQ, mQp, mK, mV, a);
     return cudaSuccess;
   };
   cudaError_t e;
