@@ -453,133 +453,6 @@ __global__ void __launch_bounds__(256) k_amat(const float* Ct, int G, int D,
   }
 }
 
-// ---------------------------------------------------------------------------
-// Query-response RMS on the tensor cores (mma.sync m16n8k16 bf16, fp32
-// accumulation), reading R4: per query row the quadratic form q A q with
-// A = Ctilde^T Ctilde split into bf16 hi + lo (the products carry ~16 bits
-// of the fp32 A); rms = sqrt(s^2 qAq / G'k + eps) and ||u_hat||^2 =
-// s^2 qAq / rms^2 (their chunk sums feed the query objective).
-// One block per CHUNK rows (sub-tiles of 128), 8 warps x 16 rows.
-// ---------------------------------------------------------------------------
-struct RmsArgs {
-  TensorView Q;
-  int N, nchunk, split_rows;
-  const bf16* bsplit;   // [BH][2][split_rows][D]: rows of A, bf16 hi then lo
-  float scale;
-  const spr_head_stats* stats;
-  float* rms;
-  float* un2;
-  double* part;
-};
-
-template <int D>
-__global__ void __launch_bounds__(256) k_query_rms(RmsArgs a) {
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  extern __shared__ __align__(128) uint8_t rsm[];
-  uint8_t* Bhi = rsm;
-  uint8_t* Blo = Bhi + D * D * 2;
-  uint8_t* Qs = Blo + D * D * 2;
-  double* red = reinterpret_cast<double*>(Qs + ATT_BM * D * 2);
-  const int bh = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31, gid = lane >> 2, tig = lane & 3;
-  // B operand = A, swizzled rows
-  const bf16* bsrc = a.bsplit + (size_t)bh * 2 * a.split_rows * D;
-  for (int e = tid; e < D * CH; e += 256) {
-    const int r = e / CH, c = e % CH;
-    *reinterpret_cast<uint4*>(Bhi + swz<CH>(r, c)) = reinterpret_cast<const uint4*>(bsrc + (size_t)r * D)[c];
-    *reinterpret_cast<uint4*>(Blo + swz<CH>(r, c)) =
-        reinterpret_cast<const uint4*>(bsrc + ((size_t)a.split_rows + r) * D)[c];
-  }
-  const float gk = (float)max(1, a.stats[bh].gk_nonempty);
-  double un2acc = 0.0;
-  for (int sub = 0; sub < CHUNK / ATT_BM; ++sub) {
-    const int row0 = chunk * CHUNK + sub * ATT_BM;
-    if (row0 >= a.N) break;
-    __syncthreads();  // previous tile consumed
-    for (int e = tid; e < ATT_BM * CH; e += 256) {
-      const int r = e / CH, c = e % CH, n = row0 + r;
-      const bf16* src = a.Q.row(bh, n < a.N ? n : 0) + c * 8;
-      cp_async16(Qs + swz<CH>(r, c), src, n < a.N ? 16 : 0);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    // A fragments for this warp's 16 rows
-    uint32_t af[D / 16][4];
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int c = ks * 2 + (lane >> 4);
-      ldsm_x4(af[ks][0], af[ks][1], af[ks][2], af[ks][3], Qs + swz<CH>(r, c));
-    }
-    const int r_lo = row0 + warp * 16 + gid, r_hi = r_lo + 8;
-    float quad_lo = 0.f, quad_hi = 0.f;
-    for (int nc = 0; nc < D; nc += 32) {
-      float acc[4][4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {  // two n-tile pairs of 16 columns
-          const int brow = nc + pr * 16 + (lane & 7) + (lane >> 4) * 8;
-          const int bc = ks * 2 + ((lane >> 3) & 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(b0, b1, b2, b3, Bhi + swz<CH>(brow, bc));
-          mma16816(acc[pr * 2], af[ks], b0, b1);
-          mma16816(acc[pr * 2 + 1], af[ks], b2, b3);
-          ldsm_x4(b0, b1, b2, b3, Blo + swz<CH>(brow, bc));
-          mma16816(acc[pr * 2], af[ks], b0, b1);
-          mma16816(acc[pr * 2 + 1], af[ks], b2, b3);
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {  // (qA)_col q_col, from the swizzled tile
-        const int col = nc + t * 8 + 2 * tig;
-        const int rl = warp * 16 + gid, rh = rl + 8;
-        const bf16* ql = reinterpret_cast<const bf16*>(Qs + swz<CH>(rl, col / 8)) + (col & 7);
-        const bf16* qh = reinterpret_cast<const bf16*>(Qs + swz<CH>(rh, col / 8)) + (col & 7);
-        quad_lo += acc[t][0] * bf2f(ql[0]) + acc[t][1] * bf2f(ql[1]);
-        quad_hi += acc[t][2] * bf2f(qh[0]) + acc[t][3] * bf2f(qh[1]);
-      }
-    }
-    quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 1);
-    quad_lo += __shfl_xor_sync(0xffffffffu, quad_lo, 2);
-    quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 1);
-    quad_hi += __shfl_xor_sync(0xffffffffu, quad_hi, 2);
-    if (tig == 0) {
-      const float s2 = a.scale * a.scale;
-      if (r_lo < a.N) {
-        const float ms = s2 * fmaxf(quad_lo, 0.f) / gk;
-        const float rr = sqrtf(ms + 1e-6f);
-        a.rms[(size_t)bh * a.N + r_lo] = rr;
-        const float u2 = s2 * fmaxf(quad_lo, 0.f) / (rr * rr);
-        a.un2[(size_t)bh * a.N + r_lo] = u2;
-        un2acc += u2;
-      }
-      if (r_hi < a.N) {
-        const float ms = s2 * fmaxf(quad_hi, 0.f) / gk;
-        const float rr = sqrtf(ms + 1e-6f);
-        a.rms[(size_t)bh * a.N + r_hi] = rr;
-        const float u2 = s2 * fmaxf(quad_hi, 0.f) / (rr * rr);
-        a.un2[(size_t)bh * a.N + r_hi] = u2;
-        un2acc += u2;
-      }
-    }
-  }
-  __syncthreads();
-  un2acc = warp_sum(un2acc);
-  if (lane == 0) red[warp] = un2acc;
-  __syncthreads();
-  if (tid == 0) {
-    double s = 0.0;
-    for (int i = 0; i < 8; ++i) s += red[i];
-    a.part[((size_t)bh * 2 + 1) * (a.nchunk + 1) + chunk] = s;
-  }
-}
-
 // Initial query centroids: a_g = (s / rms_n) q_n at the seeded rows.
 __global__ void k_init_centq(TensorView Q, int N, int G, int D, const int32_t* init,
                              const float* rms, float scale, float* centq) {
@@ -814,27 +687,11 @@ spr_launch(k_obj_z<32>, dim3(nchunk, BH), 256, 0, st, P.Z, N, p.Gk, P.centk, P.l
   spr_launch(k_amat, dim3(BH, (D / 32) * (D / 32)), 256, 0, st, P.Ct, p.Gk, D, P.stats, P.Amat, P.bq16,
                                                          split_rows);
   // Query-response RMS (tensor-core quadratic form)
-  RmsArgs ra{};
-  ra.Q = Q;
-  ra.N = N;
-  ra.nchunk = nchunk;
-  ra.split_rows = split_rows;
-  ra.bsplit = P.bq16;
-  ra.scale = scale;
-  ra.stats = P.stats;
-  ra.rms = P.rms;
-  ra.un2 = P.un2;
-  ra.part = P.part;
-  if (D == 128) {  // tcgen05; its per-tile sums use the k-means partial-sum area (idle here)
-    if ((e = launch_rms_tc(Q, p.B, p.H, N, nchunk, split_rows, P.bq16, scale, P.stats, P.rms,
-                           P.un2, reinterpret_cast<double*>(P.csum), P.part, P.hdr, st)) !=
-        cudaSuccess)
-      return e;
-  } else {
-    const size_t sm = (size_t)2 * D * D * 2 + ATT_BM * D * 2 + 64;
-    cudaFuncSetAttribute(k_query_rms<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    spr_launch(k_query_rms<D>, dim3(nchunk, BH), 256, sm, st, ra);
-  }
+  // tcgen05; its per-tile sums use the k-means partial-sum area (idle here)
+  if ((e = launch_rms_tc(Q, p.B, p.H, N, D, nchunk, split_rows, P.bq16, scale, P.stats, P.rms,
+                         P.un2, reinterpret_cast<double*>(P.csum), P.part, P.hdr, st)) !=
+      cudaSuccess)
+    return e;
   // Query k-means in the head dimension
   if (p.init != SPR_INIT_WARM)  // warm: centq keeps the previous call's head-dim centroids
     spr_launch(k_init_centq, dim3(BH, 32), 256, 0, st, Q, N, p.Gq, D, P.initq, P.rms, scale,

@@ -1,5 +1,5 @@
 // Query-response RMS on the tensor cores [paperlayer App. B.2, C.1] for head
-// dimension 128.
+// dimensions 64 and 128.
 //
 // u = s C~ q has ||u||^2 = s^2 q^T A q with A = C~^T C~ (d x d, symmetric),
 // so every row needs one quadratic form: rms = sqrt(s^2 q^T A q / G'_k +
@@ -7,10 +7,10 @@
 //
 // k_rms_tc is persistent, one CTA per SM over a contiguous range of the
 // flattened (head, 128-row tile) sequence:
-//   warp 0 lane 0   TMA: the head's A as bf16 hi and lo rows (two 64-column
-//                   boxes each) and the query tiles ([B, H, N, d] view,
+//   warp 0 lane 0   TMA: the head's A as bf16 hi and lo rows (d / 64 boxes of
+//                   64 columns each) and the query tiles ([B, H, N, d] view,
 //                   strided) into a 4-stage ring;
-//   warp 1          owns TMEM (two 128-column buffers); one thread issues
+//   warp 1          owns TMEM (two d-column buffers); one thread issues
 //                   T = q A_hi + q A_lo (tcgen05.mma kind::f16, bf16
 //                   operands, fp32 accumulation; q is exact in bf16, the
 //                   split carries ~16 bits of A);
@@ -30,14 +30,21 @@ namespace spr {
 
 namespace {
 
-constexpr int RT_D = 128;
 constexpr int RT_TM = 128;
-constexpr uint32_t RT_BOX = RT_TM * 128;      // 128 rows x 64 bf16: 16 KB
-constexpr uint32_t RT_TILE = 2 * RT_BOX;      // 128 x 128 bf16
+constexpr uint32_t RT_BOX = RT_TM * 128;      // 128 query rows x 64 bf16: 16 KB
 constexpr int RT_NS = 4;
 constexpr int RT_THREADS = 256;
 constexpr uint64_t RT_WAIT_NS = 2000000000ull;
-constexpr size_t RT_SMEM = 1024 + (size_t)(2 + RT_NS) * RT_TILE + 256;
+// per head dimension D: a query tile is D / 64 boxes, A (D x D) is D / 64
+// boxes of D rows x 64 columns
+template <int D>
+__host__ __device__ constexpr uint32_t rt_qtile() { return (D / 64) * RT_BOX; }
+template <int D>
+__host__ __device__ constexpr uint32_t rt_abox() { return D * 128; }
+template <int D>
+__host__ __device__ constexpr size_t rt_smem() {
+  return 1024 + 2 * (size_t)(D / 64) * rt_abox<D>() + (size_t)RT_NS * rt_qtile<D>() + 256;
+}
 
 struct RtArgs {
   int N, BH, H, ntile;
@@ -53,16 +60,19 @@ __device__ __forceinline__ uint32_t rt_swz(int r, int q) {  // 16-byte chunk q o
   return (uint32_t)(r * 128 + (((q ^ r) & 7) << 4));
 }
 
+template <int D>
 __global__ void __launch_bounds__(RT_THREADS, 1)
     k_rms_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmA,
              RtArgs a) {
   extern __shared__ uint8_t rt_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(rt_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint8_t* Ah = sm;                    // A hi: 2 boxes
-  uint8_t* Al = sm + RT_TILE;          // A lo: 2 boxes
-  uint8_t* Qs = sm + 2 * RT_TILE;      // [RT_NS] tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Qs + RT_NS * RT_TILE);
+  constexpr int NB = D / 64;
+  constexpr uint32_t QTILE = rt_qtile<D>(), ABOX = rt_abox<D>(), ATILE = NB * ABOX;
+  uint8_t* Ah = sm;                    // A hi: NB boxes
+  uint8_t* Al = sm + ATILE;            // A lo: NB boxes
+  uint8_t* Qs = sm + 2 * ATILE;        // [RT_NS] tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Qs + RT_NS * QTILE);
   uint64_t* q_full = bars;             // [4]
   uint64_t* q_empty = bars + 4;        // [4]
   uint64_t* t_full = bars + 8;         // [2]
@@ -99,7 +109,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     tc::prefetch_tmap(&tmA);
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_s, 2 * RT_D);
+    tc::tmem_alloc(tmem_s, 2 * D);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -115,20 +125,20 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         const int bh = head_of(t), tl = t - bh * a.ntile;
         if (t == tb || bh != head_of(t - 1)) {  // this head's A, hi and lo
           if (na > 0 && !tc::mbar_wait(a_free, (na - 1) & 1, abort_s, RT_WAIT_NS)) break;
-          tc::mbar_expect_tx(a_full, 2 * RT_TILE);
+          tc::mbar_expect_tx(a_full, 2 * ATILE);
           for (int h = 0; h < 2; ++h)
-            for (int j = 0; j < 2; ++j)
-              tc::tma_load_3d((h ? Al : Ah) + j * RT_BOX, &tmA, 64 * j, 0, 2 * bh + h, a_full);
+            for (int j = 0; j < NB; ++j)
+              tc::tma_load_3d((h ? Al : Ah) + j * ABOX, &tmA, 64 * j, 0, 2 * bh + h, a_full);
           ++na;
         }
         const int s = k % RT_NS;
         if (k >= RT_NS &&
             !tc::mbar_wait(q_empty + s, ((k / RT_NS) - 1) & 1, abort_s, RT_WAIT_NS))
           break;
-        tc::mbar_expect_tx(q_full + s, RT_TILE);
+        tc::mbar_expect_tx(q_full + s, QTILE);
         const int bb = bh / a.H, hh = bh - bb * a.H;
-        for (int j = 0; j < 2; ++j)
-          tc::tma_load_4d(Qs + s * RT_TILE + j * RT_BOX, &tmQ, 64 * j, tl * RT_TM, hh, bb,
+        for (int j = 0; j < NB; ++j)
+          tc::tma_load_4d(Qs + s * QTILE + j * RT_BOX, &tmQ, 64 * j, tl * RT_TM, hh, bb,
                           q_full + s);
         ++loads;
       }
@@ -141,7 +151,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ products
     if (lane == 0) {
-      const uint32_t idesc = tc::idesc_bf16(RT_TM, RT_D, 0);
+      const uint32_t idesc = tc::idesc_bf16(RT_TM, D, 0);
       const uint32_t ah = smem_u32(Ah), al = smem_u32(Al);
       int k = 0, na = 0;
       for (int t = tb; t < te; ++t, ++k) {
@@ -156,15 +166,16 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         if (!tc::mbar_wait(q_full + s, (k / RT_NS) & 1, abort_s, RT_WAIT_NS)) break;
         if (k >= 2 && !tc::mbar_wait(t_free + b, ((k >> 1) - 1) & 1, abort_s, RT_WAIT_NS)) break;
         tc::tc_fence_after();
-        const uint32_t d = tbase + (uint32_t)(b * RT_D);
-        const uint32_t q_addr = smem_u32(Qs + s * RT_TILE);
+        const uint32_t d = tbase + (uint32_t)(b * D);
+        const uint32_t q_addr = smem_u32(Qs + s * QTILE);
 #pragma unroll
-        for (int ks = 0; ks < RT_D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * RT_BOX + (ks & 3) * 32;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * RT_BOX + (ks & 3) * 32;   // query tile
+          const uint32_t offa = (ks >> 2) * ABOX + (ks & 3) * 32;    // A
           tc::mma_ss(d, tc::smem_desc_sw128(q_addr + off, 16, 1024),
-                     tc::smem_desc_sw128(ah + off, 16, 1024), idesc, ks > 0);
+                     tc::smem_desc_sw128(ah + offa, 16, 1024), idesc, ks > 0);
           tc::mma_ss(d, tc::smem_desc_sw128(q_addr + off, 16, 1024),
-                     tc::smem_desc_sw128(al + off, 16, 1024), idesc, 1);
+                     tc::smem_desc_sw128(al + offa, 16, 1024), idesc, 1);
         }
         tc::mma_commit(t_full + b);
         if (hend) tc::mma_commit(a_free);
@@ -187,13 +198,13 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
       got = __all_sync(0xffffffffu, got);
       if (!got) break;
       tc::tc_fence_after();
-      const uint8_t* qt = Qs + s * RT_TILE;
+      const uint8_t* qt = Qs + s * QTILE;
       float quad = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {  // columns 32c .. 32c + 31
+      for (int c = 0; c < D / 32; ++c) {  // columns 32c .. 32c + 31
         uint32_t v[32];
         __syncwarp();
-        tc::tmem_ld32(tbase + lane_f + (uint32_t)(b * RT_D + 32 * c), v);
+        tc::tmem_ld32(tbase + lane_f + (uint32_t)(b * D + 32 * c), v);
         tc::tmem_wait_ld();
         const uint8_t* box = qt + (c >> 1) * RT_BOX;
 #pragma unroll
@@ -233,7 +244,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
   if (tid == 0 && *abort_s) set_error(a.hdr, ERR_TIMEOUT, 22, blockIdx.x, 0);
   if (warp == 1) {
     __syncwarp();
-    tc::tmem_dealloc(tbase, 2 * RT_D);
+    tc::tmem_dealloc(tbase, 2 * D);
   }
 }
 
@@ -251,14 +262,15 @@ __global__ void k_un2_chunks(const double* tpart, int ntile, int nchunk, double*
 
 }  // namespace
 
-cudaError_t launch_rms_tc(const TensorView& Q, int B, int H, int N, int nchunk, int split_rows,
-                          const bf16* bsplit, float scale, const spr_head_stats* stats,
-                          float* rms, float* un2, double* tpart, double* part, Header* hdr,
-                          cudaStream_t st) {
+template <int D>
+cudaError_t launch_rms_tc_d(const TensorView& Q, int B, int H, int N, int nchunk, int split_rows,
+                            const bf16* bsplit, float scale, const spr_head_stats* stats,
+                            float* rms, float* un2, double* tpart, double* part, Header* hdr,
+                            cudaStream_t st) {
   const int BH = B * H;
   CUtensorMap mQ, mA;
   {
-    const uint64_t dims[4] = {(uint64_t)RT_D, (uint64_t)N, (uint64_t)H, (uint64_t)B};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)N, (uint64_t)H, (uint64_t)B};
     const uint64_t str[3] = {(uint64_t)Q.sn * 2, (uint64_t)Q.sh * 2, (uint64_t)Q.sb * 2};
     const uint32_t box[4] = {64, RT_TM, 1, 1};
     if (!encode_tmap(&mQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, Q.base, dims, str, box,
@@ -267,10 +279,10 @@ cudaError_t launch_rms_tc(const TensorView& Q, int B, int H, int N, int nchunk, 
   }
   {
     // [BH][2][split_rows][d] bf16: rows 0 .. d - 1 of A (hi, then lo)
-    const uint64_t dims[3] = {(uint64_t)RT_D, (uint64_t)split_rows, (uint64_t)(2 * BH)};
-    const uint64_t str[2] = {(uint64_t)RT_D * 2, (uint64_t)split_rows * RT_D * 2};
-    const uint32_t box[3] = {64, RT_TM, 1};
-    if (split_rows < RT_D ||
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)split_rows, (uint64_t)(2 * BH)};
+    const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)split_rows * D * 2};
+    const uint32_t box[3] = {64, (uint32_t)D, 1};
+    if (split_rows < D ||
         !encode_tmap(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, bsplit, dims, str, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
@@ -286,15 +298,28 @@ cudaError_t launch_rms_tc(const TensorView& Q, int B, int H, int N, int nchunk, 
   a.un2 = un2;
   a.tpart = tpart;
   a.hdr = hdr;
-  cudaError_t e =
-      cudaFuncSetAttribute(k_rms_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RT_SMEM);
+  cudaError_t e = cudaFuncSetAttribute(k_rms_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)rt_smem<D>());
   if (e != cudaSuccess) return e;
   const int T = BH * a.ntile;
   const int grid = T < num_sms() ? T : num_sms();
-  spr_launch(k_rms_tc, grid, RT_THREADS, RT_SMEM, st, mQ, mA, a);
+  spr_launch(k_rms_tc<D>, grid, RT_THREADS, rt_smem<D>(), st, mQ, mA, a);
   spr_launch(k_un2_chunks, dim3(nchunk, BH), 1, 0, st, static_cast<const double*>(tpart),
              a.ntile, nchunk, part);
   return cudaGetLastError();
+}
+
+cudaError_t launch_rms_tc(const TensorView& Q, int B, int H, int N, int D, int nchunk,
+                          int split_rows, const bf16* bsplit, float scale,
+                          const spr_head_stats* stats, float* rms, float* un2, double* tpart,
+                          double* part, Header* hdr, cudaStream_t st) {
+  if (D == 64)
+    return launch_rms_tc_d<64>(Q, B, H, N, nchunk, split_rows, bsplit, scale, stats, rms, un2,
+                               tpart, part, hdr, st);
+  if (D == 128)
+    return launch_rms_tc_d<128>(Q, B, H, N, nchunk, split_rows, bsplit, scale, stats, rms, un2,
+                                tpart, part, hdr, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace spr

@@ -125,12 +125,13 @@ cudaError_t attend_preload();
 cudaError_t attend_tc_preload();
 cudaError_t launch_reconstruct(const spr_params& p, const Layout& L, const Ptrs& P,
                                bf16* O, cudaStream_t st);
-// Query-response RMS and ||u_hat||^2 on the tensor cores (d = 128), with the
-// chunk sums of ||u_hat||^2 into part (tpart: BH * ceil(N / 128) * 4 doubles).
-cudaError_t launch_rms_tc(const TensorView& Q, int B, int H, int N, int nchunk, int split_rows,
-                          const bf16* bsplit, float scale, const spr_head_stats* stats,
-                          float* rms, float* un2, double* tpart, double* part, Header* hdr,
-                          cudaStream_t st);
+// Query-response RMS and ||u_hat||^2 on the tensor cores (head dimension D =
+// 64 or 128), with the chunk sums of ||u_hat||^2 into part (tpart: BH *
+// ceil(N / 128) * 4 doubles).
+cudaError_t launch_rms_tc(const TensorView& Q, int B, int H, int N, int D, int nchunk,
+                          int split_rows, const bf16* bsplit, float scale,
+                          const spr_head_stats* stats, float* rms, float* un2, double* tpart,
+                          double* part, Header* hdr, cudaStream_t st);
 // Residual application on the tensor cores (d = 128): O = x + b + x W per
 // unprobed permuted row, the dense row per probe, bf16 in the original order.
 cudaError_t launch_apply_tc(const spr_params& p, const Layout& L, const Ptrs& P, bf16* O, int R,
