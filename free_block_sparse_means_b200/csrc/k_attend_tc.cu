@@ -6,25 +6,36 @@
 // merged K/V groups routed to the query group, or [0, N) for probes).  Every
 // row's softmax is renormalised over exactly those keys (hard drop).
 //
-// One persistent CTA per SM, 8 warps:
+// One persistent CTA per SM, 12 warps:
 //   warp 0      producer: takes the next item from the global cursor and
 //               publishes it in a 4-slot shared-memory ring for the other
 //               roles; TMA-loads the Q tile once per item and K and V tiles of
-//               128 keys into a three-stage ring (128-byte-swizzled boxes of 64
-//               columns).
-//   warp 1      owns TMEM (512 columns: S0, S1, O) and issues the MMAs from one
-//               thread: S = Q K^T (A and B K-major in shared memory) into the
-//               S buffer of the tile, and O += P V with P read from TMEM (the
-//               bf16 probabilities the softmax wrote over S) and V as an
-//               MN-major B operand.  S of a tile whose key range ends early
-//               is computed only up to its last 16-key block; PV always
-//               covers the tile's 128 keys (P is zero past the valid ones),
-//               so that each group of products issues as straight-line code.
-//   warps 4..7  one thread per query row (= TMEM lane): scaled, masked row
-//               max, exp2, row sums, P back to TMEM; O is rescaled in TMEM only
-//               when the running max grows by more than 2^8 (the final
-//               normalisation uses the same stale max, so this is exact);
-//               epilogue O / l to global memory.
+//               128 keys into a three-stage ring (128-byte-swizzled boxes).  A
+//               key range's first tile starts at its first key rounded down
+//               to 8 (see TileIter).
+//   warp 1      owns TMEM (S0, S1, O, Q and a few exchange columns) and
+//               issues every tensor-core operation from one thread.  With VT
+//               (the values stored transposed, the attention stage's layout):
+//               Q is copied into TMEM once per item (tcgen05.cp), S = Q K^T
+//               takes A from TMEM and B = the K tile, O += P V takes A = P
+//               from TMEM (the bf16 probabilities the softmax wrote over S)
+//               and B = the transposed value tile, so every operand the
+//               tensor cores read is K-major.  Without VT (caller-owned
+//               [N, d] values) S reads Q from shared memory and PV reads V as
+//               an MN-major B.  S of a tile whose key range ends early is
+//               computed only up to its last 16-key block; PV always covers
+//               the tile's 128 keys (P is zero past the valid ones), so that
+//               each group of products issues as straight-line code.
+//   warps 2, 3  idle.
+//   warps 4..11 the softmax, two warps per scheduler: warps 4 + q and 8 + q
+//               hold rows 32q .. 32q + 31 (their TMEM lanes), the first keys
+//               0 .. 63 of every tile, the second keys 64 .. 127.  Per tile:
+//               masked half-row max, agreed with the partner through TMEM and
+//               a pair barrier; exp2, row sums, P back to TMEM; O is rescaled
+//               in TMEM only when the running max grows by more than 2^8 (the
+//               final normalisation uses the same stale max, so this is
+//               exact); per item the pair adds its row sums and each writes
+//               its half of O / l to global memory.
 // Every mbarrier wait is bounded in time; a wait that runs out sets an abort
 // flag that ends every role, the device error word records a timeout, copies
 // and MMAs in flight are drained, and TMEM is freed.  TMEM loads and stores
