@@ -562,7 +562,13 @@ def run_ours(args, wl):
             "frac": att_achieved / peaks["bf16_tflops"], "peak_source": f"{peak_kind} bf16 burst",
             "traffic": profiled_traffic(wl.name, wl.BH),
             "algorithmic_flop_per_launch": 4.0 * wl.d * pairs,
-            "executed_tile_pairs": tile_pairs, "true_pairs": pairs}
+            "executed_tile_pairs": tile_pairs, "true_pairs": pairs,
+            # the same kernel against the sustained (power-capped) bf16 peak, and
+            # on executed tile pairs (padding included) against the burst peak
+            "frac_sustained": att_achieved / peaks.get("bf16_tflops_sustained",
+                                                       FALLBACK_PEAKS["bf16_tflops_sustained"]),
+            "frac_executed_pairs": (att_achieved * tile_pairs / pairs / peaks["bf16_tflops"]
+                                    if pairs > 0 else 0.0)}
     part_bytes = partition_bytes(wl)
     part_gbs = part_bytes / (stage_max[0] * 1e-3) / 1e9
     # end to end through the public API with host buffers (pinned): the
