@@ -119,3 +119,33 @@ def test_hunyuan_shape_rows_sample_runs():
     np.testing.assert_allclose(dense_attention(q[rows], k, v, full["scale"]),
                                sparsepr_head(q, k, v, prm, lab_k=full["lab_k"], lab_q=full["lab_q"],
                                              rows=rows, want_dense=True)["O_dense"], atol=0)
+
+
+def test_group_means_by_hand_and_empty_groups():
+    from oracle import group_means
+    X = np.array([[1.0, 2.0], [3.0, 6.0], [10.0, -4.0], [5.0, 5.0]])
+    lab = np.array([0, 0, 2, 0])
+    got = group_means(X, lab, 4, fallback=np.full((4, 2), 7.0))
+    # group 0: rows 0, 1, 3 -> (9/3, 13/3); group 2: row 2; groups 1, 3 keep the fallback
+    want = np.array([[3.0, 13.0 / 3.0], [7.0, 7.0], [10.0, -4.0], [7.0, 7.0]])
+    assert np.allclose(got, want, rtol=0, atol=1e-15)
+    assert np.isnan(group_means(X, lab, 4)[1]).all()  # no fallback: NaN
+
+
+def test_multi_head_call_slices_per_head_arguments():
+    """The [B, H, N, d] wrapper runs head (b, h) as flat head b*H + h: its seeded
+    k-means rows and its per-head keyword arrays follow that index."""
+    from oracle import sparsepr_call
+    wl = workload("tiny", B=2, H=2, grid=(1, 8, 16), centers=8, Gk=8, Gq=8, Ms=64, M=16, r=4)
+    Q, K, V = (t.double().numpy() for t in voronoi_qkv(wl))
+    prm = Params(Ms=wl.Ms, p=wl.p, Gk=wl.Gk, Gq=wl.Gq, iters=wl.iters, route_mode="tau",
+                 tau=wl.tau, M=wl.M, r=wl.r, lam=wl.lam, seed=wl.index)
+    rows = [np.arange(3 * bh, 3 * bh + 5) for bh in range(4)]
+    res = sparsepr_call(Q, K, V, prm, rows=rows)
+    for b in range(2):
+        for h in range(2):
+            bh = 2 * b + h
+            one = sparsepr_head(Q[b, h], K[b, h], V[b, h], prm, bh=bh, rows=rows[bh])
+            assert np.array_equal(res[bh]["lab_k"], one["lab_k"])
+            assert np.array_equal(res[bh]["lab_q"], one["lab_q"])
+            assert np.array_equal(res[bh]["O"], one["O"])
